@@ -1,0 +1,267 @@
+"""fp64 CPU oracle for the ZipMap global large-chunk TTT layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+reference leg of ``bench.py`` may call it.  It shares no code with the CUDA
+path (``recon_chunk_ttt_b200``); both only consume the seeded arrays of
+``recon_chunk_ttt_b200.workloads``.
+
+Sources (pages on the web, cited by title and section):
+  [review]  kimjy99, "[논문리뷰] ZipMap: Linear-Time Stateful 3D Reconstruction
+            via Test-Time Training", section 2 "Feature Backbone" (Eq. 1
+            SwiGLU fast weights, Eq. 2 virtual loss, Eq. 3 eta-weighted
+            gradient, Newton-Schulz + L2 renormalisation, apply o' = f(q),
+            ray-map queries) and section 3 "Streaming Reconstruction".
+  [notes]   67656.sbs reading notes "ZipMap：基于 Test-Time Training 的线性时间
+            有状态 3D 重建", section "TTT 模块：核心公式" (virtual objective,
+            one gradient step with per-token eta, SwiGLU, the linear-case
+            derivation) and "流式更新（streaming）".
+  [survey]  mhpn.cn survey of TTSA3R / LaCT / ZipMap / LoGeR, part "二、LaCT,
+            2、架构" (update = summed chunk gradient, then L2 normalisation).
+
+Everything is float64.  Inputs are the same (bf16-exact or fp32) values the
+GPU receives, upcast exactly.  Per head:
+  W1, W3 : [hidden, d]   (rows are the fan-in vectors of hidden units)
+  W2     : [d, hidden]
+  K, V, Q: [n, d] token-major
+  eta    : [n]
+
+Readings taken where the pages are silent or ambiguous (each is also listed in
+the design notes):
+  * SiLU(x) = x * sigmoid(x) with the logistic sigmoid (the pages name SiLU
+    without defining it).
+  * One gradient step (the review says one step; the notes say "one (or a
+    few)").
+  * The Eq. 3 sum runs over every image token of the chunk (its index letter
+    is a typo in the review).
+  * Renormalisation axis: row-wise (each row of W1, W3 of length d, each row
+    of W2 of length hidden) to the pre-update row norm, no epsilon; a zero
+    updated row is left as is.  "frobenius" (whole matrix per head, the
+    literal reading of the unindexed norm) and "off" are kept as switches.
+  * Newton-Schulz orthonormalisation of the gradient is not applied (the
+    layer as specified for this build omits it).
+  * Heads are independent fast-weight MLPs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+RENORM_OFF, RENORM_ROW, RENORM_FROB = 0, 1, 2
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def sigmoid(x):
+    """Logistic function, evaluated without overflow."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    ex = np.exp(x[~pos])
+    out[~pos] = ex / (1.0 + ex)
+    return out
+
+
+def silu(x):
+    """SiLU(x) = x * sigmoid(x)."""
+    x = _f64(x)
+    return x * sigmoid(x)
+
+
+def silu_prime(x):
+    """d/dx SiLU(x) = s + x s (1 - s), s = sigmoid(x)."""
+    x = _f64(x)
+    s = sigmoid(x)
+    return s * (1.0 + x * (1.0 - s))
+
+
+# --------------------------------------------------------------------------
+# Eq. 1 of [review] / "Fast-weight MLP：SwiGLU" of [notes]:
+#   f_W(x) = W2 [ SiLU(W1 x) ⊙ (W3 x) ]
+# --------------------------------------------------------------------------
+def fast_weight_mlp(W1, W2, W3, X):
+    """Rows of X are tokens; returns f_W(x) for each row.  [n, d] -> [n, d]."""
+    W1, W2, W3, X = map(_f64, (W1, W2, W3, X))
+    h1 = X @ W1.T              # [n, hidden]  = (W1 x)^T
+    h3 = X @ W3.T              # [n, hidden]  = (W3 x)^T
+    return (silu(h1) * h3) @ W2.T
+
+
+# --------------------------------------------------------------------------
+# Eq. 2 of [review] / "虚拟目标" of [notes]:  L_i = -f_W(k_i)^T v_i,
+# weighted by the per-token write strength eta_i (Eq. 3 of [review]).
+# --------------------------------------------------------------------------
+def virtual_loss(W1, W2, W3, K, V, eta):
+    """sum_i eta_i * L(f_W(k_i), v_i) with L = -f_W(k)^T v."""
+    F = fast_weight_mlp(W1, W2, W3, K)
+    return float(-np.sum(_f64(eta) * np.sum(F * _f64(V), axis=1)))
+
+
+def gradient(W1, W2, W3, K, V, eta):
+    """g = ∇_W sum_i eta_i L(f_W(k_i), v_i)  (Eq. 3 of [review]).
+
+    Chain rule for one token with h1 = W1 k, h3 = W3 k, a = SiLU(h1),
+    u = a ⊙ h3, L = -v^T W2 u:
+        dL/dW2 = -v u^T
+        dL/du  = -W2^T v =: du
+        dL/dh3 = du ⊙ a,          dL/dW3 = (du ⊙ a) k^T
+        dL/dh1 = du ⊙ h3 ⊙ SiLU'(h1),  dL/dW1 = (...) k^T
+    Summed over all tokens with weights eta_i.  Returns (G1, G2, G3) shaped
+    like (W1, W2, W3).
+    """
+    W1, W2, W3, K, V, eta = map(_f64, (W1, W2, W3, K, V, eta))
+    h1 = K @ W1.T
+    h3 = K @ W3.T
+    a = silu(h1)
+    u = a * h3
+    du = -(V @ W2)                      # row i = (-W2^T v_i)^T
+    dh3 = du * a
+    dh1 = du * h3 * silu_prime(h1)
+    e = eta[:, None]
+    G2 = -(V * e).T @ u                 # [d, hidden]
+    G1 = (dh1 * e).T @ K                # [hidden, d]
+    G3 = (dh3 * e).T @ K                # [hidden, d]
+    return G1, G2, G3
+
+
+def gradient_rows_w13(W1, W2, W3, K, V, eta, rows):
+    """Selected rows r of G1 and G3 only, by the same formulas as
+    ``gradient`` restricted to hidden unit r (each row needs only row r of W1
+    and W3 and column r of W2).  Returns (G1[rows], G3[rows])."""
+    W1, W2, W3, K, V, eta = map(_f64, (W1, W2, W3, K, V, eta))
+    rows = np.asarray(rows)
+    h1 = K @ W1[rows].T                 # [n, r]
+    h3 = K @ W3[rows].T
+    du = -(V @ W2[:, rows])
+    e = eta[:, None]
+    dh3 = du * silu(h1)
+    dh1 = du * h3 * silu_prime(h1)
+    return (dh1 * e).T @ K, (dh3 * e).T @ K
+
+
+def gradient_cols_w2(W1, W2, W3, K, V, eta, cols):
+    """Selected columns j of G2 only: G2[:, j] = -sum_i eta_i v_i u_i[j]."""
+    W1, W3, K, V, eta = map(_f64, (W1, W3, K, V, eta))
+    cols = np.asarray(cols)
+    u = silu(K @ W1[cols].T) * (K @ W3[cols].T)      # [n, c]
+    return -(V * eta[:, None]).T @ u                 # [d, c]
+
+
+# --------------------------------------------------------------------------
+# Update and L2 renormalisation ([review] section 2, the two-line update after
+# Eq. 3; [survey] LaCT 架构 "L2 归一化"):
+#   W' = W - g,   Ŵ = ||W|| * W' / ||W'||
+# --------------------------------------------------------------------------
+def renorm(W, Wp, mode):
+    """Rescale the updated matrix Wp to the norm of the pre-update W.
+    mode: RENORM_OFF, RENORM_ROW (each row to its own pre-update row norm)
+    or RENORM_FROB (whole matrix)."""
+    W, Wp = _f64(W), _f64(Wp)
+    if mode == RENORM_OFF:
+        return Wp.copy()
+    if mode == RENORM_ROW:
+        n_old = np.sqrt(np.sum(W * W, axis=-1, keepdims=True))
+        n_new = np.sqrt(np.sum(Wp * Wp, axis=-1, keepdims=True))
+        scale = np.divide(n_old, n_new, out=np.ones_like(n_new), where=n_new > 0)
+        return Wp * scale
+    if mode == RENORM_FROB:
+        n_old = np.sqrt(np.sum(W * W))
+        n_new = np.sqrt(np.sum(Wp * Wp))
+        return Wp * (n_old / n_new) if n_new > 0 else Wp.copy()
+    raise ValueError(f"unknown renorm mode {mode}")
+
+
+def update_head(W1, W2, W3, K, V, eta, renorm_mode=RENORM_ROW):
+    """One TTT update of one head: Ŵ = renorm(W - g)."""
+    G1, G2, G3 = gradient(W1, W2, W3, K, V, eta)
+    return (renorm(W1, _f64(W1) - G1, renorm_mode),
+            renorm(W2, _f64(W2) - G2, renorm_mode),
+            renorm(W3, _f64(W3) - G3, renorm_mode))
+
+
+def _split_heads(X, heads):
+    X = _f64(X)
+    n = X.shape[0]
+    return X.reshape(n, heads, -1)
+
+
+def ttt_update(W1, W2, W3, K, V, eta, renorm_mode=RENORM_ROW):
+    """All heads.  W1, W3: [H, hidden, d]; W2: [H, d, hidden];
+    K, V: [n, H*d]; eta: [n, H].  Returns (Ŵ1, Ŵ2, Ŵ3) in fp64."""
+    H = np.shape(W1)[0]
+    Kh, Vh = _split_heads(K, H), _split_heads(V, H)
+    eta = _f64(eta).reshape(-1, H)
+    out = [update_head(W1[h], W2[h], W3[h], Kh[:, h], Vh[:, h], eta[:, h],
+                       renorm_mode) for h in range(H)]
+    return tuple(np.stack([o[i] for o in out]) for i in range(3))
+
+
+def ttt_apply(W1, W2, W3, Q):
+    """o'_i = f_Ŵ(q_i) for every query row and head ([review] section 2,
+    the apply equation; ray-map queries use the same map).  Q: [m, H*d]."""
+    H = np.shape(W1)[0]
+    Qh = _split_heads(Q, H)
+    m = Qh.shape[0]
+    O = np.stack([fast_weight_mlp(W1[h], W2[h], W3[h], Qh[:, h])
+                  for h in range(H)], axis=1)
+    return O.reshape(m, -1)
+
+
+def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW):
+    """Streaming ([review] section 3, [notes] "流式更新"): for each frame t,
+    W^(t) = TTTUpdate(W^(t-1); the frame's tokens), then the frame's queries
+    read f_{W^(t)}.  Returns the final weights and the per-frame outputs
+    concatenated in frame order."""
+    n = np.shape(K)[0]
+    Ws = (_f64(W1), _f64(W2), _f64(W3))
+    outs = []
+    for s in range(0, n, frame_tokens):
+        e = min(n, s + frame_tokens)
+        Ws = ttt_update(*Ws, K[s:e], V[s:e], eta[s:e], renorm_mode)
+        outs.append(ttt_apply(*Ws, Q[s:e]))
+    return Ws, np.concatenate(outs, axis=0)
+
+
+# --------------------------------------------------------------------------
+# Linear fast weights ([notes], "为什么它像 attention（线性情形的直观推导）"):
+#   f_W(k) = W k,  L = -(W k)^T v  =>  ∇_W L = -v k^T
+# --------------------------------------------------------------------------
+def linear_gradient(W, K, V, eta):
+    """g = ∇_W sum_i eta_i (-(W k_i)^T v_i) = -sum_i eta_i v_i k_i^T."""
+    K, V, eta = map(_f64, (K, V, eta))
+    return -(V * eta[:, None]).T @ K
+
+
+def linear_update(W, K, V, eta, renorm_mode=RENORM_OFF):
+    W = _f64(W)
+    return renorm(W, W - linear_gradient(W, K, V, eta), renorm_mode)
+
+
+def linear_apply(W, Q):
+    return _f64(Q) @ _f64(W).T
+
+
+def linear_loss(W, K, V, eta):
+    return float(-np.sum(_f64(eta) * np.sum((_f64(K) @ _f64(W).T) * _f64(V), axis=1)))
+
+
+# --------------------------------------------------------------------------
+# State size ([notes], "Fast-weight state 大小与训练规模"): three matrices of
+# d x hidden each.
+# --------------------------------------------------------------------------
+def state_params(d, hidden, heads=1):
+    return 3 * d * hidden * heads
+
+
+# --------------------------------------------------------------------------
+# Error measures used by the parity tests.
+# --------------------------------------------------------------------------
+def rel_fro(x, ref):
+    """||x - ref||_F / ||ref||_F in fp64 (returns the absolute error if the
+    reference is exactly zero)."""
+    x, ref = _f64(x), _f64(ref)
+    den = np.sqrt(np.sum(ref * ref))
+    num = np.sqrt(np.sum((x - ref) ** 2))
+    return float(num / den) if den > 0 else float(num)
