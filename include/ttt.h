@@ -1,0 +1,155 @@
+/*
+ * recon_chunk_ttt_b200 — C ABI of the ZipMap global large-chunk TTT layer on
+ * B200 (sm_100a).
+ *
+ * The layer (kimjy99, "[논문리뷰] ZipMap: Linear-Time Stateful 3D
+ * Reconstruction via Test-Time Training", section 2 "Feature Backbone"):
+ *
+ *   f_W(x) = W2 [ SiLU(W1 x) ⊙ (W3 x) ]                          (Eq. 1)
+ *   L_i    = -f_W(k_i)^T v_i                                      (Eq. 2)
+ *   g      = ∇_W Σ_i η_i L_i     (over every token of the chunk)   (Eq. 3)
+ *   Ŵ      = ‖W‖ · (W - g) / ‖W - g‖   (L2 renormalisation, the update
+ *                                       equations after Eq. 3)
+ *   o_i    = f_Ŵ(q_i)            (apply, to image or ray-map queries)
+ *
+ * and, for streaming (section 3 "Streaming Reconstruction"), the same update
+ * with the tokens of one frame at a time, the state carried across calls.
+ * The renormalisation axis is row-wise (each row of W1, W3 of length d, each
+ * row of W2 of length hidden, rescaled to its pre-update norm); "frobenius"
+ * (one norm per matrix per head) and "off" are switches.  Newton–Schulz
+ * orthonormalisation of g is not applied (ns_steps must be 0).
+ *
+ * Conventions shared by every entry point
+ *  - All pointers except `cfg` are DEVICE pointers on the current CUDA device,
+ *    owned by the caller; the library allocates nothing and keeps no state
+ *    between calls apart from one device error word per device.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default
+ *    stream); arguments are validated on the host before anything is
+ *    enqueued, so an error status means nothing was launched.
+ *  - Layouts are dense, row-major, per head h = 0..H-1:
+ *        W1, W3 : float [H][hidden][d]      W2 : float [H][d][hidden]
+ *        K, V, Q: [n][H*d] token-major, bf16 (precision BF16_TC) or
+ *                 float (precision FP32_CHECK); head h is columns h*d..h*d+d-1
+ *        eta    : float [n][H]
+ *        O      : [m][H*d], bf16 (BF16_TC) or float (FP32_CHECK)
+ *        shadow : bf16 copies of Ŵ for the tensor-core apply, in the same
+ *                 layout as W1, W3, W2 (W1 block, then W3, then W2);
+ *                 ttt_shadow_bytes() bytes.
+ *  - Device pointers must be 16-byte aligned (tensor-memory-access rule).
+ *  - Supported shapes: (d, hidden) = (64, 128) or (256, 512), heads >= 1.
+ *  - n = 0 or eta = 0 gives Ŵ = W.  Outputs may alias the weight inputs
+ *    (in-place update); K, V, Q, eta and O must not alias outputs.
+ *  - Results are deterministic run to run (fixed-order reductions, no
+ *    atomics in any sum).
+ */
+#ifndef RECON_CHUNK_TTT_H
+#define RECON_CHUNK_TTT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* ttt_stream_t;
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum   */
+  TTT_ERR_UNSUPPORTED_SHAPE = 2, /* (d, hidden) not supported               */
+  TTT_ERR_ALIGNMENT = 3,         /* a pointer is not 16-byte aligned        */
+  TTT_ERR_WORKSPACE = 4,         /* workspace missing or too small          */
+  TTT_ERR_CUDA = 5,              /* a CUDA runtime call failed              */
+  TTT_ERR_DEVICE = 6             /* a kernel gave up a bounded wait         */
+} ttt_status;
+
+enum { TTT_MLP_SWIGLU = 0 };
+enum { TTT_RENORM_OFF = 0, TTT_RENORM_ROW = 1, TTT_RENORM_FROB = 2 };
+enum { TTT_PREC_BF16_TC = 0, TTT_PREC_FP32_CHECK = 1 };
+
+typedef struct {
+  int32_t heads;     /* H, number of independent fast-weight MLPs          */
+  int32_t d;         /* head dimension (64 or 256)                         */
+  int32_t hidden;    /* fast-weight hidden width (128 or 512)              */
+  int32_t mlp;       /* TTT_MLP_SWIGLU                                     */
+  int32_t renorm;    /* TTT_RENORM_*                                       */
+  int32_t ns_steps;  /* Newton–Schulz iterations: must be 0                */
+  int32_t precision; /* TTT_PREC_BF16_TC: bf16 tensor-core operands, fp32
+                        accumulation; TTT_PREC_FP32_CHECK: fp32 CUDA-core
+                        arithmetic throughout                              */
+} ttt_config;
+
+/* Human-readable name of a status code (static string). */
+const char* ttt_status_string(ttt_status s);
+
+/* Bytes of device workspace ttt_update / ttt_stream_step need for n tokens
+ * (0 if the config is invalid). */
+size_t ttt_update_workspace_bytes(const ttt_config* cfg, int64_t n_tokens);
+
+/* Bytes of the bf16 weight shadow (3 * H * d * hidden * 2). */
+size_t ttt_shadow_bytes(const ttt_config* cfg);
+
+/*
+ * One TTT update of all heads (Eq. 1–3 and the renormalisation above):
+ *   g = ∇_W Σ_{i<n} η_i (−f_W(k_i)^T v_i),  Ŵ = renorm(W − g).
+ * Inputs W1, W2, W3 (fp32), K, V, eta for n >= 0 tokens.  Writes Ŵ to
+ * W1_out, W2_out, W3_out (fp32, may equal the inputs) and, when `shadow` is
+ * not NULL, bf16 copies of Ŵ to `shadow` for ttt_apply.
+ * `workspace` must hold ttt_update_workspace_bytes(cfg, n) bytes (it may be
+ * NULL when that is 0); its contents need no initialisation.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, WORKSPACE, CUDA.
+ */
+ttt_status ttt_update(const ttt_config* cfg,
+                      const float* W1, const float* W2, const float* W3,
+                      const void* K, const void* V, const float* eta, int64_t n,
+                      float* W1_out, float* W2_out, float* W3_out, void* shadow,
+                      void* workspace, size_t workspace_bytes, ttt_stream_t stream);
+
+/*
+ * Apply (read) the fast weights to m >= 0 queries: O[i] = f_Ŵ(Q[i]) per head
+ * (section 2 of the review: o'_i = f_Ŵ(q_i); ray-map target queries use the
+ * same call).  BF16_TC reads `shadow` (bf16 Ŵ, from ttt_update or
+ * ttt_pack_shadow) and ignores W1..W3 (may be NULL); FP32_CHECK reads W1..W3
+ * and ignores `shadow`.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, CUDA.
+ */
+ttt_status ttt_apply(const ttt_config* cfg,
+                     const float* W1, const float* W2, const float* W3,
+                     const void* shadow, const void* Q, int64_t m, void* O,
+                     ttt_stream_t stream);
+
+/* Write bf16 copies of W1, W2, W3 into `shadow` (for ttt_apply on weights
+ * that did not come out of ttt_update). */
+ttt_status ttt_pack_shadow(const ttt_config* cfg,
+                           const float* W1, const float* W2, const float* W3,
+                           void* shadow, ttt_stream_t stream);
+
+/*
+ * One streaming step (section 3 of the review, the per-frame TTTUpdate):
+ * updates the state W1, W2, W3 IN PLACE with the n tokens of one frame, then
+ * applies the new state to that frame's m queries, writing O.  `shadow` is
+ * required for BF16_TC (it receives the bf16 copy of the new state) and may
+ * be NULL for FP32_CHECK.  Workspace as for ttt_update(cfg, n).
+ */
+ttt_status ttt_stream_step(const ttt_config* cfg,
+                           float* W1, float* W2, float* W3, void* shadow,
+                           const void* K, const void* V, const float* eta, int64_t n,
+                           const void* Q, int64_t m, void* O,
+                           void* workspace, size_t workspace_bytes, ttt_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear this device's error word.  A
+ * kernel that gives up a bounded wait (it never spins without a limit) sets
+ * the word and returns early; such a call's outputs are undefined.
+ * Returns TTT_OK, TTT_ERR_DEVICE (and *code = the kernel's reason, if code
+ * is not NULL) or TTT_ERR_CUDA.
+ */
+ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RECON_CHUNK_TTT_H */

@@ -1,0 +1,27 @@
+"""B200-native (sm_100a) ZipMap global large-chunk TTT layer.
+
+The layer runs in libttt.so (C ABI in include/ttt.h); ``recon_chunk_ttt_b200``
+exposes the same entry points through a thin ctypes binding:
+
+    ttt_update, ttt_apply, ttt_stream_step, ttt_pack_shadow,
+    ttt_update_workspace_bytes, ttt_shadow_bytes, ttt_check_device_error
+
+The binding (and torch) is imported on first use, so ``workloads`` can be
+imported on machines without CUDA.
+"""
+from __future__ import annotations
+
+_EXPORTS = {
+    "ttt_update", "ttt_apply", "ttt_stream_step", "ttt_pack_shadow",
+    "ttt_update_workspace_bytes", "ttt_shadow_bytes", "ttt_check_device_error",
+    "ttt_config", "make_config", "alloc_workspace", "alloc_shadow", "status_string",
+    "TTTError", "lib", "RENORM_OFF", "RENORM_ROW", "RENORM_FROB", "PREC_BF16_TC",
+    "PREC_FP32_CHECK", "LIB_PATH",
+}
+
+
+def __getattr__(name):
+    if name in _EXPORTS:
+        from . import _binding
+        return getattr(_binding, name)
+    raise AttributeError(name)

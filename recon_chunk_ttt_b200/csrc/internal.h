@@ -1,0 +1,62 @@
+// Internal host-side interface between the C-ABI layer (ttt_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ttt {
+
+// Problem description after validation.
+struct Problem {
+  int H, d, hid;
+  int64_t n;  // tokens (update) or queries (apply)
+  int renorm;
+};
+
+// Split-K plan of the token reduction: S contiguous token ranges of `chunk`
+// tokens (the last one shorter).  A function of (n, shape) only, so results
+// are bitwise reproducible.
+struct SplitPlan {
+  int S;
+  int64_t chunk;
+};
+
+// ---- fp32 CUDA-core check mode -------------------------------------------
+SplitPlan f32_split_plan(const Problem& p);
+size_t f32_workspace_bytes(const Problem& p);
+cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const float* W3,
+                       const float* K, const float* V, const float* eta, float* W1o, float* W2o,
+                       float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st);
+cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const float* W3,
+                      const float* Q, float* O, cudaStream_t st);
+
+// ---- shared: reduce split-K partials + renormalise -----------------------
+// Partials layout: [S][H][3][hid*d] floats; block 0 = P1 (G1, [hid][d]),
+// block 1 = P3 (G3, [hid][d]), block 2 = P2 (-G2, [d][hid]).
+// Writes W_out = renorm(W - G) in fp32 and, if shadow != nullptr, bf16.
+// `scratch` holds H*(2*hid+d)*2 doubles (Frobenius mode only).
+cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const float* W1,
+                          const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
+                          __nv_bfloat16_raw* shadow, float* scratch, cudaStream_t st);
+cudaError_t pack_shadow(int H, int d, int hid, const float* W1, const float* W2,
+                        const float* W3, __nv_bfloat16_raw* shadow, cudaStream_t st);
+
+// ---- bf16 tensor-core path (tcgen05) --------------------------------------
+SplitPlan tc_split_plan(const Problem& p);
+size_t tc_workspace_bytes(const Problem& p);
+cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const float* W3,
+                      const void* K, const void* V, const float* eta, float* W1o, float* W2o,
+                      float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st);
+cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,
+                     cudaStream_t st);
+
+// The per-device error word (defined in kernels_common.cu).
+int* device_error_ptr();                       // device address, nullptr on failure
+cudaError_t read_and_clear_device_error(int* value);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace ttt

@@ -1,0 +1,193 @@
+// Work shared by both precisions: the fixed-order reduction of the split-K
+// gradient partials, the update W' = W - g and the L2 renormalisation
+// (kimjy99 ZipMap review, section 2, the update equations after Eq. 3:
+// Ŵ = ‖W‖ (W - Δ)/‖W - Δ‖), plus the bf16 shadow packing.
+//
+// Renormalisation axis: row-wise by default (each row of W1, W3 of length d,
+// each row of W2 of length hidden, to its pre-update norm, no epsilon; a zero
+// updated row stays zero); Frobenius (whole matrix per head) or off on request.
+// This is HBM-bound CUDA-core work: one warp per row, a sum over the S
+// partials in increasing s, and a butterfly sum of squares, so the result is
+// the same bit pattern on every run.
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace ttt {
+
+namespace {
+
+__device__ int g_device_error = 0;
+
+constexpr int kMaxRowPerLane = 16;  // rows up to 512 elements
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ __nv_bfloat16_raw to_bf16_raw(float x) {
+  __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<__nv_bfloat16_raw*>(&b);
+}
+
+// Row decoding: per head, rows [0,hid) are W1, [hid,2hid) W3, [2hid,2hid+d) W2.
+struct RowRef {
+  int head, blk, row, len;  // blk: 0 = W1, 1 = W3, 2 = W2
+};
+__device__ __forceinline__ RowRef decode_row(int R, int d, int hid) {
+  const int per = 2 * hid + d;
+  RowRef r;
+  r.head = R / per;
+  int x = R % per;
+  if (x < hid) {
+    r.blk = 0; r.row = x; r.len = d;
+  } else if (x < 2 * hid) {
+    r.blk = 1; r.row = x - hid; r.len = d;
+  } else {
+    r.blk = 2; r.row = x - 2 * hid; r.len = hid;
+  }
+  return r;
+}
+
+__global__ void __launch_bounds__(256) reduce_renorm_kernel(
+    const float* __restrict__ partials, int S, int H, int d, int hid, int mode,
+    const float* W1, const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
+    __nv_bfloat16_raw* __restrict__ shadow, double* __restrict__ scratch) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= H * (2 * hid + d)) return;
+  const RowRef r = decode_row(warp, d, hid);
+  const size_t mat = (size_t)hid * d;
+  const float* W = r.blk == 0 ? W1 : r.blk == 1 ? W3 : W2;
+  float* Wo = r.blk == 0 ? W1o : r.blk == 1 ? W3o : W2o;
+  const size_t base = (size_t)r.head * mat + (size_t)r.row * r.len;
+  // P1, P3 are G1, G3 (subtract); P2 is -G2 (add).
+  const float sign = r.blk == 2 ? 1.f : -1.f;
+  const int pblk = r.blk;  // partial block index equals blk
+  const int per_lane = r.len / 32;
+  // The split sum, W' = W -/+ g and both norms are formed in fp64 so that the
+  // only rounding left on Ŵ - W is the final fp32 store.
+  double wn[kMaxRowPerLane];
+  double s_old = 0.0, s_new = 0.0;
+#pragma unroll
+  for (int k = 0; k < kMaxRowPerLane; ++k) {
+    if (k < per_lane) {
+      const int idx = lane + 32 * k;
+      const double w = (double)W[base + idx];
+      double g = 0.0;
+      for (int s = 0; s < S; ++s)
+        g += (double)partials[(((size_t)s * H + r.head) * 3 + pblk) * mat +
+                              (size_t)r.row * r.len + idx];
+      const double wp = w + (double)sign * g;
+      wn[k] = wp;
+      s_old = fma(w, w, s_old);
+      s_new = fma(wp, wp, s_new);
+    }
+  }
+  s_old = warp_sum(s_old);
+  s_new = warp_sum(s_new);
+  double scale = 1.0;
+  if (mode == 1) scale = s_new > 0.0 ? sqrt(s_old) / sqrt(s_new) : 1.0;
+  if (mode == 2 && lane == 0) {
+    scratch[2 * (size_t)warp] = s_old;
+    scratch[2 * (size_t)warp + 1] = s_new;
+  }
+  const size_t sh_off = (size_t)r.blk * H * mat;  // shadow blocks W1, W3, W2
+#pragma unroll
+  for (int k = 0; k < kMaxRowPerLane; ++k) {
+    if (k < per_lane) {
+      const int idx = lane + 32 * k;
+      const float v = (float)(wn[k] * scale);
+      Wo[base + idx] = v;
+      if (shadow != nullptr && mode != 2) shadow[sh_off + base + idx] = to_bf16_raw(v);
+    }
+  }
+}
+
+// Frobenius mode: one block per (head, matrix).  Sums the per-row squares in
+// row order, then rescales the matrix in place and writes the shadow.
+__global__ void __launch_bounds__(256) frob_scale_kernel(
+    int H, int d, int hid, const double* __restrict__ scratch, float* W1o, float* W2o,
+    float* W3o, __nv_bfloat16_raw* __restrict__ shadow) {
+  const int head = blockIdx.x / 3, blk = blockIdx.x % 3;
+  const int per = 2 * hid + d;
+  const int r0 = head * per + (blk == 0 ? 0 : blk == 1 ? hid : 2 * hid);
+  const int rows = blk == 2 ? d : hid;
+  __shared__ double sc;
+  if (threadIdx.x == 0) {
+    double so = 0.0, sn = 0.0;  // sequential, fixed order
+    for (int i = 0; i < rows; ++i) {
+      so += scratch[2 * (size_t)(r0 + i)];
+      sn += scratch[2 * (size_t)(r0 + i) + 1];
+    }
+    sc = sn > 0.0 ? sqrt(so) / sqrt(sn) : 1.0;
+  }
+  __syncthreads();
+  const size_t mat = (size_t)hid * d;
+  float* Wo = (blk == 0 ? W1o : blk == 1 ? W3o : W2o) + (size_t)head * mat;
+  __nv_bfloat16_raw* sh = shadow ? shadow + (size_t)blk * H * mat + (size_t)head * mat : nullptr;
+  const double s = sc;
+  for (size_t i = threadIdx.x; i < mat; i += blockDim.x) {
+    const float v = (float)((double)Wo[i] * s);
+    Wo[i] = v;
+    if (sh) sh[i] = to_bf16_raw(v);
+  }
+}
+
+__global__ void pack_shadow_kernel(size_t mat_total, const float* __restrict__ W1,
+                                   const float* __restrict__ W2, const float* __restrict__ W3,
+                                   __nv_bfloat16_raw* __restrict__ shadow) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < mat_total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    shadow[i] = to_bf16_raw(W1[i]);
+    shadow[mat_total + i] = to_bf16_raw(W3[i]);
+    shadow[2 * mat_total + i] = to_bf16_raw(W2[i]);
+  }
+}
+
+}  // namespace
+
+cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const float* W1,
+                          const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
+                          __nv_bfloat16_raw* shadow, float* scratch, cudaStream_t st) {
+  const int rows = p.H * (2 * p.hid + p.d);
+  const int blocks = (rows * 32 + 255) / 256;
+  reduce_renorm_kernel<<<blocks, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, p.renorm, W1, W2,
+                                              W3, W1o, W2o, W3o, shadow,
+                                              reinterpret_cast<double*>(scratch));
+  if (p.renorm == 2)
+    frob_scale_kernel<<<p.H * 3, 256, 0, st>>>(p.H, p.d, p.hid, reinterpret_cast<double*>(scratch),
+                                              W1o, W2o, W3o, shadow);
+  return cudaGetLastError();
+}
+
+int* device_error_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+cudaError_t read_and_clear_device_error(int* value) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *value = v;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
+cudaError_t pack_shadow(int H, int d, int hid, const float* W1, const float* W2,
+                        const float* W3, __nv_bfloat16_raw* shadow, cudaStream_t st) {
+  const size_t total = (size_t)H * hid * d;
+  int blocks = (int)((total + 255) / 256);
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  pack_shadow_kernel<<<blocks, 256, 0, st>>>(total, W1, W2, W3, shadow);
+  return cudaGetLastError();
+}
+
+}  // namespace ttt

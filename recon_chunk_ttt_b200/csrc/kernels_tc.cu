@@ -1,0 +1,953 @@
+// bf16 tensor-core path of the TTT update and apply on sm_100a: tcgen05 MMAs
+// with fp32 accumulators in tensor memory (TMEM), operands staged in shared
+// memory by TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast), warp
+// specialised (one TMA producer thread, one MMA issuer thread, epilogue
+// warps), every wait bounded.
+//
+// Update of one head (kimjy99 ZipMap review, section 2, Eq. 1-3):
+//   fb kernel   h1 = W1 k, h3 = W3 k (one N=128 MMA over [W1s; W3s]),
+//               du = -W2^T v (N=64 MMA), then in the epilogue
+//               η·u, η·dh1, η·dh3 (u = SiLU(h1) ⊙ h3, dh3 = du ⊙ SiLU(h1),
+//               dh1 = du ⊙ h3 ⊙ SiLU'(h1)) stored as bf16 [H][n][hid].
+//   grad kernel split-K token reduction on MN-major operands:
+//               P1 = Σ η dh1 k^T, P3 = Σ η dh3 k^T, P2 = Σ η u v^T (= -G2^T,
+//               stored transposed as [d][hid]); fixed token ranges.
+//   then the shared fixed-order reduce + renorm kernel.
+// Apply:        per 128-query tile, for each 64-wide hidden slice:
+//               F = Q [W1s; W3s]^T (TMEM), u = SiLU(h1) ⊙ h3 -> bf16 in shared
+//               memory, O += u W2s^T (TMEM); hidden activations never leave
+//               the SM.
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace ttt {
+namespace {
+
+constexpr int BM = 128;          // MMA M: tokens (fb, apply) or hidden rows (grad)
+constexpr int HS = 64;           // hidden slice per fb CTA / apply step
+constexpr int CH = 64;           // bf16 elements per 128-byte swizzle row
+constexpr int TK = 64;           // tokens per grad stage
+constexpr uint32_t KSTEP_BYTES = 32;  // 16 bf16 along K inside a K-major row
+
+// ----------------------------------------------------------------------------
+// Host: tensor maps
+// ----------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor of rank 2 or 3 with dims[0] contiguous; box inner dim is 64
+// elements (128 bytes) with the 128-byte swizzle.  Out-of-range rows read 0.
+bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* byte_strides, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = byte_strides[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Before a CTA exits, wait (bounded, ignoring the abort flag) until the last
+// loads issued into each of the `nstage` ring slots have landed, so no TMA
+// write can reach shared memory after the CTA is gone.  `count` is the number
+// of loads issued into the ring so far (slot i % nstage, phase (i/nstage)&1).
+__device__ __forceinline__ void drain_ring(uint64_t* full, int nstage, int64_t count, int* err) {
+  volatile int never = 0;
+  for (int64_t i = count - nstage < 0 ? 0 : count - nstage; i < count; ++i)
+    mbar_wait(&full[i % nstage], (uint32_t)((i / nstage) & 1), &never, err, kErrWaitFinal);
+}
+
+// σ(x) = (1 + tanh(x/2)) / 2 with the hardware tanh approximation.
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
+
+// ----------------------------------------------------------------------------
+// Weight prologue: bf16 copies of W1, W3 ([H][hid][d]) and of W2^T ([H][hid][d])
+// ----------------------------------------------------------------------------
+__global__ void convert_weights_kernel(int H, int d, int hid, const float* __restrict__ W1,
+                                       const float* __restrict__ W2, const float* __restrict__ W3,
+                                       __nv_bfloat16* __restrict__ b1, __nv_bfloat16* __restrict__ b3,
+                                       __nv_bfloat16* __restrict__ b2t) {
+  const size_t total = (size_t)H * hid * d;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    b1[i] = __float2bfloat16_rn(W1[i]);
+    b3[i] = __float2bfloat16_rn(W3[i]);
+    const size_t h = i / ((size_t)hid * d), r = i % ((size_t)hid * d);
+    const size_t j = r / d, c = r % d;
+    b2t[i] = __float2bfloat16_rn(W2[h * (size_t)hid * d + c * hid + j]);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// fb kernel: forward dual GEMM + backward GEMM + gated epilogue
+// ----------------------------------------------------------------------------
+template <int D>
+struct FB {
+  static constexpr int NCH = D / CH;
+  static constexpr int NSTAGE = 6;
+  static constexpr int STAGE = BM * CH * 2;              // 16 KB token chunk
+  static constexpr int W13_CH = 2 * HS * CH * 2;          // 16 KB: W1s rows then W3s rows
+  static constexpr int W2_CH = HS * CH * 2;               // 8 KB
+  static constexpr int OFF_W13 = 0;
+  static constexpr int OFF_W2 = OFF_W13 + NCH * W13_CH;
+  static constexpr int OFF_STAGE = OFF_W2 + NCH * W2_CH;
+  static constexpr int OFF_BAR = OFF_STAGE + NSTAGE * STAGE;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;       // + alignment slack
+  static constexpr int THREADS = 192;                     // producer, MMA, 4 epilogue warps
+  static constexpr uint32_t TMEM_COLS = 512;              // 2 x (F13 128 + DU 64), at 0 / 256
+};
+
+template <int D>
+__global__ void __launch_bounds__(FB<D>::THREADS, 1)
+    fb_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+              const __grid_constant__ CUtensorMap mW1, const __grid_constant__ CUtensorMap mW3,
+              const __grid_constant__ CUtensorMap mW2t, const float* __restrict__ eta, int64_t n,
+              int H, int hid, int64_t total_items, __nv_bfloat16* __restrict__ U,
+              __nv_bfloat16* __restrict__ DH1, __nv_bfloat16* __restrict__ DH3, int* err) {
+  using L = FB<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + L::NSTAGE;
+  uint64_t* wfull = empty + L::NSTAGE;
+  uint64_t* wempty = wfull + 1;
+  uint64_t* acc_full = wempty + 1;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nslices = hid / HS;
+  const int64_t ntiles = (n + BM - 1) / BM;
+  const int64_t it0 = total_items * blockIdx.x / gridDim.x;
+  const int64_t it1 = total_items * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(wfull, 1);
+    mbar_init(wempty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&mK);
+    tma_prefetch_desc(&mV);
+    int stage = 0;
+    uint32_t phase = 0, wphase = 0;
+    int cur_hs = -1;
+    int64_t issued = 0, wloads = 0;
+    bool ok = true;
+    for (int64_t it = it0; it < it1 && ok; ++it) {
+      const int hs = (int)(it / ntiles);
+      const int64_t tile = it % ntiles;
+      const int head = hs / nslices, slice = hs % nslices;
+      if (hs != cur_hs) {
+        if (cur_hs >= 0) {
+          if (!mbar_wait(wempty, wphase, abort_flag, err, kErrWaitEmpty)) { ok = false; break; }
+          wphase ^= 1;
+        }
+        mbar_arrive_expect_tx(wfull, L::NCH * (L::W13_CH + L::W2_CH));
+        const int row = head * hid + slice * HS;
+        for (int c = 0; c < L::NCH; ++c) {
+          uint8_t* w13 = smem + L::OFF_W13 + c * L::W13_CH;
+          tma_load_2d(w13, &mW1, wfull, c * CH, row);
+          tma_load_2d(w13 + HS * 128, &mW3, wfull, c * CH, row);
+          tma_load_2d(smem + L::OFF_W2 + c * L::W2_CH, &mW2t, wfull, c * CH, row);
+        }
+        ++wloads;
+        cur_hs = hs;
+      }
+      const int y = (int)(tile * BM);
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        const CUtensorMap* m = pass == 0 ? &mK : &mV;
+        for (int c = 0; c < L::NCH; ++c) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::STAGE);
+          tma_load_2d(smem + L::OFF_STAGE + stage * L::STAGE, m, &full[stage], head * D + c * CH,
+                      y);
+          ++issued;
+          if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    drain_ring(full, L::NSTAGE, issued, err);
+    drain_ring(wfull, 1, wloads, err);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idF = idesc_bf16_f32(BM, 2 * HS, false, false);
+    const uint32_t idU = idesc_bf16_f32(BM, HS, false, false);
+    int stage = 0;
+    uint32_t phase = 0, wphase = 0;
+    uint32_t aphase[2] = {0, 0};
+    int cur_hs = -1, buf = 0;
+    bool ok = true;
+    const uint32_t sbase = smem_u32(smem);
+    for (int64_t it = it0; it < it1 && ok; ++it) {
+      const int hs = (int)(it / ntiles);
+      if (hs != cur_hs) {
+        if (cur_hs >= 0) umma_commit(wempty);  // old weights free once prior MMAs finish
+        if (!mbar_wait(wfull, wphase, abort_flag, err, kErrWaitFull)) { ok = false; break; }
+        wphase ^= 1;
+        cur_hs = hs;
+      }
+      if (!mbar_wait(&acc_empty[buf], aphase[buf] ^ 1, abort_flag, err, kErrWaitAccFree)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t dF = tmem + buf * 256, dU = tmem + buf * 256 + 128;
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        for (int c = 0; c < L::NCH; ++c) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = sbase + L::OFF_STAGE + stage * L::STAGE;
+          const uint32_t b = pass == 0 ? sbase + L::OFF_W13 + c * L::W13_CH
+                                       : sbase + L::OFF_W2 + c * L::W2_CH;
+#pragma unroll
+          for (int kk = 0; kk < CH / 16; ++kk) {
+            const uint64_t da = sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024);
+            const uint64_t db = sdesc_sw128(b + kk * KSTEP_BYTES, 16, 1024);
+            umma_bf16(pass == 0 ? dF : dU, da, db, pass == 0 ? idF : idU, (c | kk) != 0);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
+        }
+      }
+      umma_commit(&acc_full[buf]);
+      aphase[buf] ^= 1;
+      buf ^= 1;
+    }
+    // Wait for every MMA issued by this thread before TMEM is released.
+    umma_commit(done);
+    volatile int never = 0;
+    mbar_wait(done, 0, &never, err, kErrWaitFinal);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    uint32_t aphase[2] = {0, 0};
+    int buf = 0;
+    for (int64_t it = it0; it < it1; ++it) {
+      const int hs = (int)(it / ntiles);
+      const int64_t tile = it % ntiles;
+      const int head = hs / nslices, slice = hs % nslices;
+      const bool got = mbar_wait(&acc_full[buf], aphase[buf], abort_flag, err, kErrWaitAcc);
+      __syncwarp();
+      if (!got) break;
+      aphase[buf] ^= 1;
+      tc_fence_after();
+      const int64_t tok = tile * BM + q * 32 + lane;
+      const bool live = tok < n;
+      const float ne = live ? -eta[tok * H + head] : 0.f;  // -η: du = -(W2^T v)
+      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256;
+      const size_t orow = ((size_t)head * n + (live ? tok : 0)) * hid + slice * HS;
+#pragma unroll
+      for (int half = 0; half < HS / 32; ++half) {
+        uint32_t r1[32], r3[32], rd[32];
+        tmem_ld_32x32(tl + half * 32, r1);
+        tmem_ld_32x32(tl + HS + half * 32, r3);
+        tmem_ld_32x32(tl + 128 + half * 32, rd);
+        tmem_ld_wait();
+        if (half == HS / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        uint32_t pu[16], p1[16], p3[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float o_u[2], o_1[2], o_3[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float h1 = __uint_as_float(r1[i + e]);
+            const float h3 = __uint_as_float(r3[i + e]);
+            const float edu = ne * __uint_as_float(rd[i + e]);  // η du
+            const float s = sigmoid_fast(h1);
+            const float a = h1 * s;                             // SiLU(h1)
+            const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
+            o_u[e] = -ne * (a * h3);
+            o_3[e] = edu * a;
+            o_1[e] = edu * h3 * dsl;
+          }
+          pu[i / 2] = pack_bf16x2(o_u[0], o_u[1]);
+          p1[i / 2] = pack_bf16x2(o_1[0], o_1[1]);
+          p3[i / 2] = pack_bf16x2(o_3[0], o_3[1]);
+        }
+        if (live) {
+          uint4* du_ = reinterpret_cast<uint4*>(U + orow + half * 32);
+          uint4* d1_ = reinterpret_cast<uint4*>(DH1 + orow + half * 32);
+          uint4* d3_ = reinterpret_cast<uint4*>(DH3 + orow + half * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            du_[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+            d1_[v] = make_uint4(p1[4 * v], p1[4 * v + 1], p1[4 * v + 2], p1[4 * v + 3]);
+            d3_[v] = make_uint4(p3[4 * v], p3[4 * v + 1], p3[4 * v + 2], p3[4 * v + 3]);
+          }
+        }
+      }
+      buf ^= 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// grad kernel: split-K token reduction with MN-major operands
+//   kind 0: acc0 = Σ_t DH1[t, tile]^T K[t, :], acc1 = Σ_t DH3[t, tile]^T K[t, :]
+//   kind 1: acc_a = Σ_t U[t, tile_a]^T V[t, :] for two hidden tiles (one if
+//           hid = 128)
+// Each CTA = (kind, head, hidden tile group, split s); split s owns tokens
+// [s*chunk, min(n, (s+1)*chunk)), chunk a multiple of TK.
+// ----------------------------------------------------------------------------
+template <int D>
+struct GR {
+  static constexpr int NSTAGE = 3;
+  static constexpr int A_TILE = BM * TK * 2;              // 16 KB: 2 boxes [64 tok x 64 hid]
+  static constexpr int B_TILE = D * TK * 2;               // D/64 boxes [64 tok x 64 d]
+  static constexpr int STAGE = 2 * A_TILE + B_TILE;
+  static constexpr int OFF_BAR = NSTAGE * STAGE;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 512;              // acc a at column a*256
+};
+
+template <int D>
+__global__ void __launch_bounds__(GR<D>::THREADS, 1)
+    grad_kernel(const __grid_constant__ CUtensorMap mDH1, const __grid_constant__ CUtensorMap mDH3,
+                const __grid_constant__ CUtensorMap mU, const __grid_constant__ CUtensorMap mK,
+                const __grid_constant__ CUtensorMap mV, int64_t n, int H, int hid, int64_t chunk,
+                int ctas_kind0, int ctas_kind1, float* __restrict__ partials, int* err) {
+  using L = GR<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + L::NSTAGE;
+  uint64_t* acc_full = empty + L::NSTAGE;
+  uint64_t* done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // Decode (split, kind, head, tile group).
+  const int per_split = ctas_kind0 + ctas_kind1;
+  const int s = blockIdx.x / per_split;
+  int r = blockIdx.x % per_split;
+  const int kind = r < ctas_kind0 ? 0 : 1;
+  if (kind == 1) r -= ctas_kind0;
+  const int groups_per_head = kind == 0 ? hid / BM : (hid / BM + 1) / 2;
+  const int head = r / groups_per_head, grp = r % groups_per_head;
+  const int j_first = kind == 0 ? grp * BM : grp * 2 * BM;
+  const int nacc = kind == 0 ? 2 : (j_first + BM < hid ? 2 : 1);
+  const int64_t ts = (int64_t)s * chunk;
+  const int64_t te = ts + chunk < n ? ts + chunk : n;
+  const int nsteps = te > ts ? (int)((te - ts + TK - 1) / TK) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    const uint32_t bytes = (uint32_t)(nacc * L::A_TILE + L::B_TILE);
+    for (int k = 0; k < nsteps; ++k) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) break;
+      uint8_t* st = smem + stage * L::STAGE;
+      mbar_arrive_expect_tx(&full[stage], bytes);
+      const int y = (int)(ts + (int64_t)k * TK);
+      for (int a = 0; a < nacc; ++a) {
+        const CUtensorMap* m = kind == 0 ? (a == 0 ? &mDH1 : &mDH3) : &mU;
+        const int j = kind == 0 ? j_first : j_first + a * BM;
+        tma_load_3d(st + a * L::A_TILE, m, &full[stage], j, y, head);
+        tma_load_3d(st + a * L::A_TILE + TK * 128, m, &full[stage], j + CH, y, head);
+      }
+      const CUtensorMap* mb = kind == 0 ? &mK : &mV;
+      for (int c = 0; c < D / CH; ++c)
+        tma_load_2d(st + 2 * L::A_TILE + c * TK * 128, mb, &full[stage], head * D + c * CH, y);
+      ++issued;
+      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
+    }
+    drain_ring(full, L::NSTAGE, issued, err);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(BM, D, true, true);
+    const uint32_t sbase = smem_u32(smem);
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int k = 0; k < nsteps; ++k) {
+      if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) break;
+      tc_fence_after();
+      const uint32_t st = sbase + stage * L::STAGE;
+#pragma unroll
+      for (int kk = 0; kk < TK / 16; ++kk) {
+        // 16 tokens = two 8-row groups of 1024 bytes.
+        const uint64_t db = sdesc_sw128(st + 2 * L::A_TILE + kk * 2048, TK * 128, 1024);
+        for (int a = 0; a < nacc; ++a) {
+          const uint64_t da = sdesc_sw128(st + a * L::A_TILE + kk * 2048, TK * 128, 1024);
+          umma_bf16(tmem + a * 256, da, db, idesc, (k | kk) != 0);
+        }
+      }
+      umma_commit(&empty[stage]);
+      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
+    }
+    umma_commit(acc_full);
+    umma_commit(done);
+    volatile int never = 0;
+    mbar_wait(done, 0, &never, err, kErrWaitFinal);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const bool have = nsteps > 0 && mbar_wait(acc_full, 0, abort_flag, err, kErrWaitAcc);
+    __syncwarp();
+    tc_fence_after();
+    const size_t mat = (size_t)hid * D;
+    for (int a = 0; a < nacc; ++a) {
+      const int blk = kind == 0 ? a : 2;  // P1, P3, P2
+      float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat;
+      const int j = (kind == 0 ? j_first : j_first + a * BM) + q * 32 + lane;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t rr[32];
+        if (have) {
+          tmem_ld_32x32(tmem + ((uint32_t)(q * 32) << 16) + a * 256 + c0, rr);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rr[i] = 0u;
+        }
+        if (kind == 0) {
+          float4* dst = reinterpret_cast<float4*>(P + (size_t)j * D + c0);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
+                                 __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) P[(size_t)(c0 + i) * hid + j] = __uint_as_float(rr[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// apply kernel: O = W2 [SiLU(W1 q) ⊙ W3 q], one (query tile, head) per CTA
+// ----------------------------------------------------------------------------
+template <int D>
+struct AP {
+  static constexpr int NCH = D / CH;
+  static constexpr int NSTAGE = 3;
+  static constexpr int STAGE = 32768;                    // 2 W13 chunks, or one W2 slice
+  static constexpr int W13_CH = 2 * HS * CH * 2;         // 16 KB
+  static constexpr int CH_PER_STAGE = NCH >= 2 ? 2 : 1;
+  static constexpr int OFF_Q = 0;                        // NCH x [128 x 128 B]
+  static constexpr int OFF_STAGE = OFF_Q + NCH * BM * 128;
+  static constexpr int OFF_U = OFF_STAGE + NSTAGE * STAGE;  // 2 x [128 x 128 B]
+  static constexpr int OFF_BAR = OFF_U + 2 * BM * 128;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 512;             // F[0] 0, F[1] 128, O at 256
+};
+
+template <int D>
+__global__ void __launch_bounds__(AP<D>::THREADS, 1)
+    apply_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW1,
+                 const __grid_constant__ CUtensorMap mW3, const __grid_constant__ CUtensorMap mW2,
+                 int64_t m, int H, int hid, __nv_bfloat16* __restrict__ O, int* err) {
+  using L = AP<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + L::NSTAGE;
+  uint64_t* q_full = empty + L::NSTAGE;
+  uint64_t* f_full = q_full + 1;
+  uint64_t* f_empty = f_full + 2;
+  uint64_t* u_full = f_empty + 2;
+  uint64_t* u_empty = u_full + 2;
+  uint64_t* o_full = u_empty + 2;
+  uint64_t* done = o_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t qt = blockIdx.x;
+  const int head = blockIdx.y;
+  const int nsl = hid / HS;
+  const int w13_stages = L::NCH / L::CH_PER_STAGE;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&f_full[b], 1);
+      mbar_init(&f_empty[b], 4);
+      mbar_init(&u_full[b], 4);
+      mbar_init(&u_empty[b], 1);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    mbar_arrive_expect_tx(q_full, L::NCH * BM * 128);
+    for (int c = 0; c < L::NCH; ++c)
+      tma_load_2d(smem + L::OFF_Q + c * BM * 128, &mQ, q_full, head * D + c * CH, (int)(qt * BM));
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    auto next = [&]() -> uint8_t* {
+      if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) return nullptr;
+      return smem + L::OFF_STAGE + stage * L::STAGE;
+    };
+    auto advance = [&]() {
+      ++issued;
+      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
+    };
+    auto load_w13 = [&](int js) {
+      for (int g = 0; g < w13_stages && ok; ++g) {
+        uint8_t* st = next();
+        if (!st) { ok = false; return; }
+        mbar_arrive_expect_tx(&full[stage], L::CH_PER_STAGE * L::W13_CH);
+        for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
+          const int c = g * L::CH_PER_STAGE + cc;
+          tma_load_2d(st + cc * L::W13_CH, &mW1, &full[stage], c * CH, head * hid + js * HS);
+          tma_load_2d(st + cc * L::W13_CH + HS * 128, &mW3, &full[stage], c * CH,
+                      head * hid + js * HS);
+        }
+        advance();
+      }
+    };
+    auto load_w2 = [&](int js) {
+      uint8_t* st = next();
+      if (!st) { ok = false; return; }
+      mbar_arrive_expect_tx(&full[stage], D * 128);
+      tma_load_2d(st, &mW2, &full[stage], js * HS, head * D);
+      advance();
+    };
+    for (int js = 0; js < nsl && ok; ++js) {
+      load_w13(js);
+      if (js >= 1 && ok) load_w2(js - 1);
+    }
+    if (ok) load_w2(nsl - 1);
+    drain_ring(full, L::NSTAGE, issued, err);
+    drain_ring(q_full, 1, 1, err);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idF = idesc_bf16_f32(BM, 2 * HS, false, false);
+    const uint32_t idO = idesc_bf16_f32(BM, D, false, false);
+    const uint32_t sbase = smem_u32(smem);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t fph[2] = {0, 0}, uph[2] = {0, 0};
+    bool ok = mbar_wait(q_full, 0, abort_flag, err, kErrWaitFull);
+    tc_fence_after();
+    auto take = [&]() -> bool {
+      if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) return false;
+      tc_fence_after();
+      return true;
+    };
+    auto release = [&]() {
+      umma_commit(&empty[stage]);
+      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
+    };
+    auto do_o = [&](int j) -> bool {
+      const int b = j & 1;
+      if (!mbar_wait(&u_full[b], uph[b], abort_flag, err, kErrWaitOperand)) return false;
+      uph[b] ^= 1;
+      tc_fence_after();
+      if (!take()) return false;
+      const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
+      const uint32_t ub = sbase + L::OFF_U + b * BM * 128;
+#pragma unroll
+      for (int kk = 0; kk < HS / 16; ++kk)
+        umma_bf16(tmem + 256, sdesc_sw128(ub + kk * KSTEP_BYTES, 16, 1024),
+                  sdesc_sw128(st + kk * KSTEP_BYTES, 16, 1024), idO, (j | kk) != 0);
+      release();
+      umma_commit(&u_empty[b]);
+      return true;
+    };
+    for (int js = 0; js < nsl && ok; ++js) {
+      const int b = js & 1;
+      if (!mbar_wait(&f_empty[b], fph[b] ^ 1, abort_flag, err, kErrWaitAccFree)) { ok = false; break; }
+      fph[b] ^= 1;
+      tc_fence_after();
+      for (int g = 0; g < w13_stages && ok; ++g) {
+        if (!take()) { ok = false; break; }
+        const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
+        for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
+          const int c = g * L::CH_PER_STAGE + cc;
+          const uint32_t qa = sbase + L::OFF_Q + c * BM * 128;
+#pragma unroll
+          for (int kk = 0; kk < CH / 16; ++kk)
+            umma_bf16(tmem + b * 128, sdesc_sw128(qa + kk * KSTEP_BYTES, 16, 1024),
+                      sdesc_sw128(st + cc * L::W13_CH + kk * KSTEP_BYTES, 16, 1024), idF,
+                      (c | kk) != 0);
+        }
+        release();
+      }
+      if (!ok) break;
+      umma_commit(&f_full[b]);
+      if (js >= 1 && !do_o(js - 1)) { ok = false; break; }
+    }
+    if (ok && do_o(nsl - 1)) umma_commit(o_full);
+    umma_commit(done);
+    volatile int never = 0;
+    mbar_wait(done, 0, &never, err, kErrWaitFinal);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int64_t qi = qt * BM + row;
+    uint32_t fph[2] = {0, 0}, uph[2] = {0, 0};
+    bool ok = true;
+    for (int js = 0; js < nsl && ok; ++js) {
+      const int b = js & 1;
+      const bool got = mbar_wait(&f_full[b], fph[b], abort_flag, err, kErrWaitAcc);
+      __syncwarp();
+      if (!got) { ok = false; break; }
+      fph[b] ^= 1;
+      tc_fence_after();
+      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + b * 128;
+      uint32_t pk[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r1[32], r3[32];
+        tmem_ld_32x32(tl + half * 32, r1);
+        tmem_ld_32x32(tl + HS + half * 32, r3);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float h1a = __uint_as_float(r1[i]), h1b = __uint_as_float(r1[i + 1]);
+          const float ua = h1a * sigmoid_fast(h1a) * __uint_as_float(r3[i]);
+          const float ub = h1b * sigmoid_fast(h1b) * __uint_as_float(r3[i + 1]);
+          pk[half * 16 + i / 2] = pack_bf16x2(ua, ub);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&f_empty[b]);
+      if (!mbar_wait(&u_empty[b], uph[b] ^ 1, abort_flag, err, kErrWaitOperand)) { ok = false; break; }
+      uph[b] ^= 1;
+      // K-major 128-byte-swizzled row: 16-byte chunk c of row r sits at
+      // chunk position c ^ (r % 8).
+      uint8_t* urow = smem + L::OFF_U + b * BM * 128 + (row / 8) * 1024 + (row % 8) * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(urow + ((c ^ (row % 8)) * 16)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&u_full[b]);
+    }
+    const bool got_o = ok && mbar_wait(o_full, 0, abort_flag, err, kErrWaitAcc);
+    __syncwarp();
+    if (got_o) {
+      tc_fence_after();
+      const uint32_t to = tmem + ((uint32_t)(q * 32) << 16) + 256;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld_32x32(to + c0, rr);
+        tmem_ld_wait();
+        if (qi < m) {
+          uint4* dst = reinterpret_cast<uint4*>(O + qi * (int64_t)H * D + (int64_t)head * D + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(
+                pack_bf16x2(__uint_as_float(rr[8 * v]), __uint_as_float(rr[8 * v + 1])),
+                pack_bf16x2(__uint_as_float(rr[8 * v + 2]), __uint_as_float(rr[8 * v + 3])),
+                pack_bf16x2(__uint_as_float(rr[8 * v + 4]), __uint_as_float(rr[8 * v + 5])),
+                pack_bf16x2(__uint_as_float(rr[8 * v + 6]), __uint_as_float(rr[8 * v + 7])));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+struct TcWs {
+  __nv_bfloat16 *b1, *b3, *b2t, *U, *DH1, *DH3;
+  float *partials, *scratch;
+};
+
+TcWs carve(const Problem& p, void* ws, int S) {
+  TcWs w;
+  char* c = static_cast<char*>(ws);
+  const size_t wsz = (size_t)p.H * p.hid * p.d;
+  w.b1 = reinterpret_cast<__nv_bfloat16*>(c);
+  w.b3 = w.b1 + wsz;
+  w.b2t = w.b3 + wsz;
+  c += align_up(3 * wsz * 2, 1024);
+  const size_t inter = (size_t)p.H * p.n * p.hid;
+  w.U = reinterpret_cast<__nv_bfloat16*>(c);
+  c += align_up(inter * 2, 1024);
+  w.DH1 = reinterpret_cast<__nv_bfloat16*>(c);
+  c += align_up(inter * 2, 1024);
+  w.DH3 = reinterpret_cast<__nv_bfloat16*>(c);
+  c += align_up(inter * 2, 1024);
+  w.partials = reinterpret_cast<float*>(c);
+  c += align_up((size_t)S * p.H * 3 * p.hid * p.d * 4, 1024);
+  w.scratch = reinterpret_cast<float*>(c);
+  return w;
+}
+
+int grad_ctas_per_split(const Problem& p) {
+  const int tiles = p.hid / BM;
+  return p.H * tiles + p.H * ((tiles + 1) / 2);
+}
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+template <int D>
+cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, const float* W3,
+                           const void* K, const void* V, const float* eta, float* W1o, float* W2o,
+                           float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st) {
+  const SplitPlan sp = tc_split_plan(p);
+  TcWs w = carve(p, ws, sp.S);
+  int* err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidDevice;
+  const size_t wsz = (size_t)p.H * p.hid * p.d;
+  if (p.n > 0) {
+    int cb = (int)((wsz + 255) / 256);
+    if (cb > 1184) cb = 1184;
+    convert_weights_kernel<<<cb, 256, 0, st>>>(p.H, p.d, p.hid, W1, W2, W3, w.b1, w.b3, w.b2t);
+    CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg;
+    const uint64_t ld = (uint64_t)p.H * D;
+    {
+      const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
+      const uint32_t box[2] = {CH, BM}, boxg[2] = {CH, TK};
+      if (!make_map(&mK, K, 2, dims, str, box) || !make_map(&mV, V, 2, dims, str, box) ||
+          !make_map(&mKg, K, 2, dims, str, boxg) || !make_map(&mVg, V, 2, dims, str, boxg))
+        return cudaErrorInvalidValue;
+    }
+    {
+      const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * p.hid}, str[1] = {(uint64_t)D * 2};
+      const uint32_t box[2] = {CH, HS};
+      if (!make_map(&mW1, w.b1, 2, dims, str, box) || !make_map(&mW3, w.b3, 2, dims, str, box) ||
+          !make_map(&mW2t, w.b2t, 2, dims, str, box))
+        return cudaErrorInvalidValue;
+    }
+    {
+      const uint64_t dims[3] = {(uint64_t)p.hid, (uint64_t)p.n, (uint64_t)p.H};
+      const uint64_t str[2] = {(uint64_t)p.hid * 2, (uint64_t)p.n * p.hid * 2};
+      const uint32_t box[3] = {CH, TK, 1};
+      if (!make_map(&mDH1, w.DH1, 3, dims, str, box) || !make_map(&mDH3, w.DH3, 3, dims, str, box) ||
+          !make_map(&mU, w.U, 3, dims, str, box))
+        return cudaErrorInvalidValue;
+    }
+    // fb: contiguous ranges of (head, slice, token tile) items per CTA.
+    const int64_t ntiles = (p.n + BM - 1) / BM;
+    const int64_t items = (int64_t)p.H * (p.hid / HS) * ntiles;
+    const int sms = num_sms();
+    const int grid_fb = (int)(items < sms ? items : sms);
+    cudaError_t e = cudaFuncSetAttribute(fb_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         FB<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
+        mK, mV, mW1, mW3, mW2t, eta, p.n, p.H, p.hid, items, w.U, w.DH1, w.DH3, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int tiles = p.hid / BM;
+    const int k0 = p.H * tiles, k1 = p.H * ((tiles + 1) / 2);
+    e = cudaFuncSetAttribute(grad_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GR<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    grad_kernel<D><<<sp.S * (k0 + k1), GR<D>::THREADS, GR<D>::SMEM, st>>>(
+        mDH1, mDH3, mU, mKg, mVg, p.n, p.H, p.hid, sp.chunk, k0, k1, w.partials, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else {
+    cudaMemsetAsync(w.partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * 4, st);
+  }
+  return reduce_renorm(p, sp.S, w.partials, W1, W2, W3, W1o, W2o, W3o, shadow, w.scratch, st);
+}
+
+template <int D>
+cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q,
+                          void* O, cudaStream_t st) {
+  if (p.n == 0) return cudaSuccess;
+  int* err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidDevice;
+  const size_t wsz = (size_t)p.H * p.hid * D;
+  const __nv_bfloat16_raw* s1 = shadow;
+  const __nv_bfloat16_raw* s3 = shadow + wsz;
+  const __nv_bfloat16_raw* s2 = shadow + 2 * wsz;
+  CUtensorMap mQ, mW1, mW3, mW2;
+  const uint64_t ld = (uint64_t)p.H * D;
+  {
+    const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
+    const uint32_t box[2] = {CH, BM};
+    if (!make_map(&mQ, Q, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * p.hid}, str[1] = {(uint64_t)D * 2};
+    const uint32_t box[2] = {CH, HS};
+    if (!make_map(&mW1, s1, 2, dims, str, box) || !make_map(&mW3, s3, 2, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)p.hid, (uint64_t)p.H * D}, str[1] = {(uint64_t)p.hid * 2};
+    const uint32_t box[2] = {CH, (uint32_t)D};
+    if (!make_map(&mW2, s2, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(apply_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, AP<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((p.n + BM - 1) / BM), p.H);
+  apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
+      mQ, mW1, mW3, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+SplitPlan tc_split_plan(const Problem& p) {
+  const int per = grad_ctas_per_split(p);
+  int S = 148 / per;
+  if (S < 1) S = 1;
+  const int64_t max_s = (p.n + TK - 1) / TK;
+  if (S > max_s) S = (int)(max_s < 1 ? 1 : max_s);
+  int64_t chunk = (p.n + S - 1) / S;
+  chunk = (chunk + TK - 1) / TK * TK;
+  if (chunk < TK) chunk = TK;
+  return {S, chunk};
+}
+
+size_t tc_workspace_bytes(const Problem& p) {
+  const SplitPlan sp = tc_split_plan(p);
+  const size_t wsz = (size_t)p.H * p.hid * p.d;
+  const size_t inter = (size_t)p.H * p.n * p.hid;
+  size_t b = align_up(3 * wsz * 2, 1024);
+  b += 3 * align_up(inter * 2, 1024);
+  b += align_up((size_t)sp.S * p.H * 3 * p.hid * p.d * 4, 1024);
+  b += align_up((size_t)p.H * (2 * p.hid + p.d) * 2 * 8, 1024);
+  return b;
+}
+
+cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const float* W3,
+                      const void* K, const void* V, const float* eta, float* W1o, float* W2o,
+                      float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st) {
+  if (p.d == 256) return tc_update_impl<256>(p, W1, W2, W3, K, V, eta, W1o, W2o, W3o, shadow, ws, st);
+  return tc_update_impl<64>(p, W1, W2, W3, K, V, eta, W1o, W2o, W3o, shadow, ws, st);
+}
+
+cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,
+                     cudaStream_t st) {
+  if (p.d == 256) return tc_apply_impl<256>(p, shadow, Q, O, st);
+  return tc_apply_impl<64>(p, shadow, Q, O, st);
+}
+
+}  // namespace ttt

@@ -1,0 +1,165 @@
+// C-ABI boundary (include/ttt.h): host-side validation, workspace planning and
+// dispatch to the fp32 check-mode or the bf16 tensor-core kernels.  Nothing
+// is enqueued unless every argument checks out.
+
+#include <cuda_runtime.h>
+
+#include "../../include/ttt.h"
+#include "common.cuh"
+#include "internal.h"
+
+using ttt::Problem;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ttt_status check_cfg(const ttt_config* cfg) {
+  if (cfg == nullptr) return TTT_ERR_INVALID_ARG;
+  if (cfg->heads < 1 || cfg->heads > 4096) return TTT_ERR_INVALID_ARG;
+  if (cfg->mlp != TTT_MLP_SWIGLU) return TTT_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->renorm < TTT_RENORM_OFF || cfg->renorm > TTT_RENORM_FROB) return TTT_ERR_INVALID_ARG;
+  if (cfg->precision != TTT_PREC_BF16_TC && cfg->precision != TTT_PREC_FP32_CHECK)
+    return TTT_ERR_INVALID_ARG;
+  if (cfg->ns_steps != 0) return TTT_ERR_UNSUPPORTED_SHAPE;
+  const bool ok = (cfg->d == 64 && cfg->hidden == 128) || (cfg->d == 256 && cfg->hidden == 512);
+  if (!ok) return TTT_ERR_UNSUPPORTED_SHAPE;
+  return TTT_OK;
+}
+
+Problem make_problem(const ttt_config* cfg, int64_t n) {
+  Problem p;
+  p.H = cfg->heads;
+  p.d = cfg->d;
+  p.hid = cfg->hidden;
+  p.n = n;
+  p.renorm = cfg->renorm;
+  return p;
+}
+
+// Token counts are limited so that every index fits the kernels' int64
+// arithmetic and the tensor-map coordinates (int32).
+constexpr int64_t kMaxTokens = (int64_t)1 << 30;
+
+ttt_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* ttt_status_string(ttt_status s) {
+  switch (s) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_INVALID_ARG: return "invalid argument";
+    case TTT_ERR_UNSUPPORTED_SHAPE: return "unsupported shape or option";
+    case TTT_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case TTT_ERR_WORKSPACE: return "workspace missing or too small";
+    case TTT_ERR_CUDA: return "CUDA runtime error";
+    case TTT_ERR_DEVICE: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+size_t ttt_update_workspace_bytes(const ttt_config* cfg, int64_t n_tokens) {
+  if (check_cfg(cfg) != TTT_OK || n_tokens < 0 || n_tokens > kMaxTokens) return 0;
+  const Problem p = make_problem(cfg, n_tokens);
+  return cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_workspace_bytes(p)
+                                               : ttt::tc_workspace_bytes(p);
+}
+
+size_t ttt_shadow_bytes(const ttt_config* cfg) {
+  if (check_cfg(cfg) != TTT_OK) return 0;
+  return (size_t)3 * cfg->heads * cfg->d * cfg->hidden * 2;
+}
+
+ttt_status ttt_update(const ttt_config* cfg, const float* W1, const float* W2, const float* W3,
+                      const void* K, const void* V, const float* eta, int64_t n, float* W1_out,
+                      float* W2_out, float* W3_out, void* shadow, void* workspace,
+                      size_t workspace_bytes, ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (n < 0 || n > kMaxTokens) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !W2 || !W3 || !W1_out || !W2_out || !W3_out) return TTT_ERR_INVALID_ARG;
+  if (n > 0 && (!K || !V || !eta)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {W1, W2, W3, K, V, eta, W1_out, W2_out, W3_out, shadow, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const Problem p = make_problem(cfg, n);
+  const size_t need = cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_workspace_bytes(p)
+                                                            : ttt::tc_workspace_bytes(p);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* sh = static_cast<__nv_bfloat16_raw*>(shadow);
+  if (cfg->precision == TTT_PREC_FP32_CHECK)
+    return cuda_status(ttt::f32_update(p, W1, W2, W3, static_cast<const float*>(K),
+                                       static_cast<const float*>(V), eta, W1_out, W2_out, W3_out,
+                                       sh, workspace, st));
+  return cuda_status(
+      ttt::tc_update(p, W1, W2, W3, K, V, eta, W1_out, W2_out, W3_out, sh, workspace, st));
+}
+
+ttt_status ttt_apply(const ttt_config* cfg, const float* W1, const float* W2, const float* W3,
+                     const void* shadow, const void* Q, int64_t m, void* O,
+                     ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (m < 0 || m > kMaxTokens) return TTT_ERR_INVALID_ARG;
+  if (m > 0 && (!Q || !O)) return TTT_ERR_INVALID_ARG;
+  if (cfg->precision == TTT_PREC_FP32_CHECK) {
+    if (!W1 || !W2 || !W3) return TTT_ERR_INVALID_ARG;
+  } else if (!shadow) {
+    return TTT_ERR_INVALID_ARG;
+  }
+  const void* ptrs[] = {W1, W2, W3, shadow, Q, O};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const Problem p = make_problem(cfg, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->precision == TTT_PREC_FP32_CHECK)
+    return cuda_status(ttt::f32_apply(p, W1, W2, W3, static_cast<const float*>(Q),
+                                      static_cast<float*>(O), st));
+  return cuda_status(
+      ttt::tc_apply(p, static_cast<const __nv_bfloat16_raw*>(shadow), Q, O, st));
+}
+
+ttt_status ttt_pack_shadow(const ttt_config* cfg, const float* W1, const float* W2,
+                           const float* W3, void* shadow, ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (!W1 || !W2 || !W3 || !shadow) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {W1, W2, W3, shadow};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return TTT_ERR_ALIGNMENT;
+  return cuda_status(ttt::pack_shadow(cfg->heads, cfg->d, cfg->hidden, W1, W2, W3,
+                                      static_cast<__nv_bfloat16_raw*>(shadow),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_stream_step(const ttt_config* cfg, float* W1, float* W2, float* W3, void* shadow,
+                           const void* K, const void* V, const float* eta, int64_t n,
+                           const void* Q, int64_t m, void* O, void* workspace,
+                           size_t workspace_bytes, ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (cfg->precision == TTT_PREC_BF16_TC && !shadow) return TTT_ERR_INVALID_ARG;
+  if (m < 0 || m > kMaxTokens) return TTT_ERR_INVALID_ARG;
+  if (m > 0 && (!Q || !O)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, O};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  s = ttt_update(cfg, W1, W2, W3, K, V, eta, n, W1, W2, W3, shadow, workspace, workspace_bytes,
+                 stream);
+  if (s != TTT_OK) return s;
+  return ttt_apply(cfg, W1, W2, W3, shadow, Q, m, O, stream);
+}
+
+ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TTT_ERR_CUDA;
+  int v = 0;
+  if (ttt::read_and_clear_device_error(&v) != cudaSuccess) return TTT_ERR_CUDA;
+  if (code) *code = v;
+  return v != 0 ? TTT_ERR_DEVICE : TTT_OK;
+}
+
+}  // extern "C"

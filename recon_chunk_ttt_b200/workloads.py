@@ -114,9 +114,15 @@ def draw_weights(rng: np.random.Generator, heads: int, d: int, hidden: int,
     return w1, w2, w3
 
 
+def bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) to the float32 values they encode."""
+    return (np.ascontiguousarray(bits).astype(np.uint32) << 16).view(np.float32)
+
+
 def _tokens(rng: np.random.Generator, n: int, heads: int, d: int,
-            normalise: bool, scale: float, bf16: bool, chunk: int = 65536):
-    out = np.empty((n, heads * d), dtype=np.float32)
+            normalise: bool, scale: float, bf16: bool, chunk: int = 65536,
+            bits: bool = False):
+    out = np.empty((n, heads * d), dtype=np.uint16 if (bits and bf16) else np.float32)
     for s in range(0, n, chunk):
         e = min(n, s + chunk)
         x = rng.standard_normal((e - s, heads * d), dtype=np.float32)
@@ -126,7 +132,10 @@ def _tokens(rng: np.random.Generator, n: int, heads: int, d: int,
             x = xh.reshape(e - s, heads * d).astype(np.float32)
         else:
             x = x * np.float32(scale)
-        out[s:e] = bf16_round(x) if bf16 else x
+        if bits and bf16:
+            out[s:e] = bf16_bits(bf16_round(x))
+        else:
+            out[s:e] = bf16_round(x) if bf16 else x
     return out
 
 
@@ -143,10 +152,12 @@ class LayerInputs:
 
 
 def make_inputs(w: Workload | str, n_tokens: int | None = None,
-                layer: int = 0) -> LayerInputs:
+                layer: int = 0, bits: bool = False) -> LayerInputs:
     """Draw one layer's inputs for a workload.  With n_tokens given, the same
     recipe and seed are used for a chunk of that many tokens (a different
-    draw from the first n_tokens of the full-size chunk)."""
+    draw from the first n_tokens of the full-size chunk).  With bits=True the
+    bf16 token arrays (K, V, Q, Qray) are returned as uint16 bit patterns,
+    half the host memory of float32 (same values)."""
     if isinstance(w, str):
         w = WORKLOADS[w]
     n = w.n_tokens if n_tokens is None else int(n_tokens)
@@ -161,9 +172,9 @@ def make_inputs(w: Workload | str, n_tokens: int | None = None,
         W1, W2, W3 = draw_weights(wrng, w.heads, w.d, w.hidden,
                                   1.0 / w.d, 1.0 / w.hidden)
     scale = 1.0 / np.sqrt(w.d)
-    K = _tokens(rng, n, w.heads, w.d, w.normalise, scale, w.bf16_inputs)
-    V = _tokens(rng, n, w.heads, w.d, w.normalise, scale, w.bf16_inputs)
-    Q = _tokens(rng, n, w.heads, w.d, w.normalise, scale, w.bf16_inputs)
+    K = _tokens(rng, n, w.heads, w.d, w.normalise, scale, w.bf16_inputs, bits=bits)
+    V = _tokens(rng, n, w.heads, w.d, w.normalise, scale, w.bf16_inputs, bits=bits)
+    Q = _tokens(rng, n, w.heads, w.d, w.normalise, scale, w.bf16_inputs, bits=bits)
     z = rng.standard_normal((n, w.heads))
     if w.name == "tiny":
         eta = (0.01 * _softplus(z)).astype(np.float32)
@@ -171,7 +182,8 @@ def make_inputs(w: Workload | str, n_tokens: int | None = None,
         eta = _softplus(z - 3.0).astype(np.float32)
     Qray = None
     if w.ray_views:
-        Qray = _tokens(rng, w.n_ray, w.heads, w.d, w.normalise, scale, w.bf16_inputs)
+        Qray = _tokens(rng, w.n_ray, w.heads, w.d, w.normalise, scale, w.bf16_inputs,
+                       bits=bits)
     return LayerInputs(W1, W2, W3, K, V, Q, eta, Qray)
 
 

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/ttt.h declares, and rejects bad arguments before
+anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttt.h")
+
+
+@pytest.fixture(scope="module")
+def B():
+    from recon_chunk_ttt_b200 import build
+    build.build()
+    from recon_chunk_ttt_b200 import _binding
+    return _binding
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttt_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("ttt_update", "ttt_apply", "ttt_stream_step", "ttt_update_workspace_bytes",
+              "ttt_status_string", "ttt_shadow_bytes", "ttt_pack_shadow",
+              "ttt_check_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(B):
+    L = B.lib()
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_status_strings(B):
+    assert B.status_string(0) == "ok"
+    assert "alignment" in B.status_string(B.TTT_ERR_ALIGNMENT) or \
+        "aligned" in B.status_string(B.TTT_ERR_ALIGNMENT)
+    assert B.status_string(99) == "unknown status"
+
+
+def _cfg(B, **kw):
+    base = dict(heads=4, d=256, hidden=512, renorm=B.RENORM_ROW, precision=B.PREC_BF16_TC)
+    base.update(kw)
+    return B.make_config(**base)
+
+
+def test_workspace_sizes(B):
+    cfg = _cfg(B)
+    n = 961800
+    ws = B.ttt_update_workspace_bytes(cfg, n)
+    inter = 3 * 4 * n * 512 * 2          # bf16 η·u, η·dh1, η·dh3
+    assert inter < ws < inter + 64 * 2**20
+    assert B.ttt_update_workspace_bytes(cfg, 0) > 0
+    f32 = B.ttt_update_workspace_bytes(_cfg(B, precision=B.PREC_FP32_CHECK), 1000)
+    assert f32 >= 3 * 4 * 1000 * 512 * 4
+    assert B.ttt_shadow_bytes(cfg) == 3 * 4 * 256 * 512 * 2
+    assert B.ttt_update_workspace_bytes(_cfg(B, d=100), 10) == 0
+    assert B.ttt_update_workspace_bytes(cfg, -1) == 0
+
+
+FAKE = 0x10000  # aligned, never dereferenced: validation fails first
+
+
+def _update(B, cfg, n=10, ws_bytes=1 << 40, **over):
+    args = dict(W1=FAKE, W2=FAKE, W3=FAKE, K=FAKE, V=FAKE, eta=FAKE, W1o=FAKE, W2o=FAKE,
+                W3o=FAKE, shadow=None, ws=FAKE)
+    args.update(over)
+    L = B.lib()
+    cp = ctypes.byref(cfg) if cfg is not None else None
+    return L.ttt_update(cp, args["W1"], args["W2"], args["W3"], args["K"], args["V"],
+                        args["eta"], n, args["W1o"], args["W2o"], args["W3o"], args["shadow"],
+                        args["ws"], ws_bytes, None)
+
+
+def test_update_rejects_bad_arguments(B):
+    assert _update(B, None) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B, d=128, hidden=256)) == B.TTT_ERR_UNSUPPORTED_SHAPE
+    assert _update(B, _cfg(B, ns_steps=1)) == B.TTT_ERR_UNSUPPORTED_SHAPE
+    assert _update(B, _cfg(B, renorm=7)) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B, precision=5)) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B, heads=0)) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B), n=-1) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B), W1=None) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B), K=None) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B), K=FAKE + 8) == B.TTT_ERR_ALIGNMENT
+    assert _update(B, _cfg(B), eta=FAKE + 4) == B.TTT_ERR_ALIGNMENT
+    assert _update(B, _cfg(B), ws=None) == B.TTT_ERR_WORKSPACE
+    assert _update(B, _cfg(B), ws_bytes=100) == B.TTT_ERR_WORKSPACE
+
+
+def test_apply_and_stream_reject_bad_arguments(B):
+    L = B.lib()
+    cfg = _cfg(B)
+    # bf16 apply needs the shadow
+    assert L.ttt_apply(ctypes.byref(cfg), None, None, None, None, FAKE, 5, FAKE,
+                       None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_apply(ctypes.byref(cfg), None, None, None, FAKE, FAKE + 2, 5, FAKE,
+                       None) == B.TTT_ERR_ALIGNMENT
+    assert L.ttt_apply(ctypes.byref(cfg), None, None, None, FAKE, FAKE, -3, FAKE,
+                       None) == B.TTT_ERR_INVALID_ARG
+    f32 = _cfg(B, precision=B.PREC_FP32_CHECK)
+    assert L.ttt_apply(ctypes.byref(f32), None, FAKE, FAKE, None, FAKE, 5, FAKE,
+                       None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_stream_step(ctypes.byref(cfg), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 5,
+                             FAKE, 5, FAKE, FAKE, 1 << 40, None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_pack_shadow(ctypes.byref(cfg), FAKE, FAKE, FAKE, None,
+                             None) == B.TTT_ERR_INVALID_ARG
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The package and the kernels never import or link the oracle."""
+    pkg = os.path.join(ROOT, "recon_chunk_ttt_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "ttt_oracle" not in txt, f
