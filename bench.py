@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the large-chunk TTT layer on B200: update + apply tokens/s per
+layer on the 700-frame scene (961,800 image tokens in one bidirectional chunk,
+4 heads x d=256, SwiGLU hidden 512, 16 ray-map target views = 21,984 ray
+queries, a 24-layer stack with independent seeded weights per layer).
+
+One step = for each of the 24 layers: ttt_update over all 961,800 tokens,
+ttt_apply to the 961,800 image queries and ttt_apply to the 21,984 ray
+queries.  value = 961,800 * 24 / step time (tokens/s per layer), summed over
+ranks for N > 1 (each rank reconstructs its own scene: weak scaling, no
+collective on the data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle (the reference arm of this build)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from recon_chunk_ttt_b200 import workloads as wl  # noqa: E402
+
+METRIC = "TTT update+apply tokens/s per layer @700 frames"
+UNIT = "tokens/s"
+GEMM_UNIT = lambda d, h: 2 * d * h  # noqa: E731  flops of one d x h matrix-vector product
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="scene700")
+    ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_config(w: wl.Workload, layers: int) -> dict:
+    return {
+        "workload": (f"{w.name}: {w.frames} frames x {w.p} tokens = {w.n_tokens} tokens in one "
+                     f"chunk, {w.heads} heads x d={w.d}, SwiGLU hidden {w.hidden}, {layers} "
+                     f"layers, {w.n_ray} ray queries"),
+        "tokens": w.n_tokens, "ray_queries": w.n_ray, "layers": layers, "heads": w.heads,
+        "d": w.d, "hidden": w.hidden, "renorm": "row",
+        "l2": "inputs larger than L2 (K, V, Q bf16 = %.1f GB)" % (3 * w.n_tokens * w.heads * w.d
+                                                                  * 2 / 1e9),
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ttt_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        under = [s for s in sm if s > 500] or sm
+        return {"sm_mhz": statistics.median(under) if under else None,
+                "sm_max_mhz": max(mx) if mx else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w: wl.Workload, frames: int, seed_layer: int = 0):
+    """Time the fp64 oracle's update + apply on `frames` frames of the
+    workload (one layer).  Returns (tokens, seconds)."""
+    import oracle as O
+    x = wl.make_inputs(w, n_tokens=frames * w.p, layer=seed_layer)
+    t0 = time.perf_counter()
+    Wh = O.ttt_update(x.W1, x.W2, x.W3, x.K, x.V, x.eta, O.RENORM_ROW)
+    O.ttt_apply(*Wh, x.Q)
+    return frames * w.p, time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w: wl.Workload, seconds: float) -> dict:
+    tok, dt = oracle_sample(w, 1)
+    frames = max(1, min(w.frames, int(seconds / max(dt, 1e-3))))
+    tok, dt = oracle_sample(w, frames)
+    return {"value": tok / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle, one layer of {w.name}: update + image apply on "
+                       f"{frames} frames ({tok} tokens, {w.heads} heads) in {dt:.1f} s")}
+
+
+def run_reference(args, w: wl.Workload, world: int, rank: int):
+    if rank != 0:
+        return
+    layers = args.layers or w.layers
+    # size one step at about 5 s of CPU work
+    tok, dt = oracle_sample(w, 1)
+    frames = max(1, min(w.frames, int(5.0 / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(w, frames)
+    times = []
+    for _ in range(args.steps):
+        tok, dt = oracle_sample(w, frames)
+        times.append(dt)
+    t = sum(times) / len(times)
+    value = tok / t
+    sample = (f"fp64 numpy oracle, one layer of {w.name}: update + image apply on {frames} "
+              f"frames ({tok} tokens, {w.heads} heads) per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, layers),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
+    import torch
+    import recon_chunk_ttt_b200 as R
+    from recon_chunk_ttt_b200 import build as B
+
+    B.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    layers = args.layers or w.layers
+    H, d, hid = w.heads, w.d, w.hidden
+    T, M = w.n_tokens, w.n_ray
+    cfg = R.make_config(H, d, hid, renorm=R.RENORM_ROW, precision=R.PREC_BF16_TC)
+
+    x = wl.make_inputs(w, bits=True)
+    to_bf = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)  # noqa: E731
+    hK, hV, hQ = to_bf(x.K), to_bf(x.V), to_bf(x.Q)
+    hQr = to_bf(x.Qray) if x.Qray is not None else torch.zeros((0, H * d), dtype=torch.bfloat16)
+    heta = torch.from_numpy(x.eta)
+    hW = []
+    for layer in range(layers):
+        xl = x if layer == 0 else None
+        if xl is None:
+            rngw = np.random.default_rng([w.seed, layer])
+            W1, W2, W3 = wl.draw_weights(rngw, H, d, hid, 1.0 / d, 1.0 / hid)
+        else:
+            W1, W2, W3 = xl.W1, xl.W2, xl.W3
+        hW.append(tuple(torch.from_numpy(a) for a in (W1, W2, W3)))
+    del x
+
+    K, V, Q, Qr = (t.to(dev) for t in (hK, hV, hQ, hQr))
+    eta = heta.to(dev)
+    Win = [tuple(t.to(dev) for t in ws) for ws in hW]
+    Wout = [tuple(torch.empty_like(t) for t in ws) for ws in Win]
+    shadow = R.alloc_shadow(cfg, dev)
+    ws_buf = R.alloc_workspace(cfg, T, dev)
+    O = torch.empty((T, H * d), dtype=torch.bfloat16, device=dev)
+    Or = torch.empty((M, H * d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(o_hook=None):
+        for layer in range(layers):
+            W1, W2, W3 = Win[layer]
+            a, b, c = Wout[layer]
+            R.ttt_update(cfg, W1, W2, W3, K, V, eta, a, b, c, shadow=shadow, workspace=ws_buf,
+                         stream=stream)
+            R.ttt_apply(cfg, Q, O, shadow=shadow, stream=stream)
+            if M:
+                R.ttt_apply(cfg, Qr, Or, shadow=shadow, stream=stream)
+            if o_hook is not None:
+                o_hook(layer)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    R.ttt_check_device_error()
+
+    # -------------------------------------------------- timed region
+    R.ttt_trace_enable(True)
+    R.ttt_trace_read(reset=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    R.ttt_trace_enable(False)
+    trace = R.ttt_trace_read(reset=True)
+    R.ttt_check_device_error()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms)
+    value = world * T * layers / (ms / 1e3)
+
+    # -------------------------------------------------- roofline
+    pk, pk_kind = peaks()
+    unit = GEMM_UNIT(d, hid)
+    kflops = {  # algorithmic flops of all launches of each kernel in the timed region
+        "tc_fwd_bwd": 3 * unit * T * H * layers * args.steps,
+        "tc_grad": 3 * unit * T * H * layers * args.steps,
+        "tc_apply": 3 * unit * (T + M) * H * layers * args.steps,
+    }
+    per_kernel = {k: {"launches": v[0], "ms_total": v[1], "ms_avg": v[1] / max(v[0], 1)}
+                  for k, v in trace.items()}
+    dom = max((k for k in kflops if k in trace), key=lambda k: trace[k][1])
+    launches = trace[dom][0]
+    achieved = kflops[dom] / (trace[dom][1] / 1e3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            tj = json.load(f)
+        ent = tj.get(dom)
+        if ent and ent.get("source_sha") == kernel_source_sha():
+            traffic = ent["bytes_per_token_head"] * T * H * (1 if dom != "tc_apply" else
+                                                             (T + M) / (2 * T))
+    upd_ms = (trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1] +
+              trace.get("tc_convert_weights", (0, 0))[1] + trace.get("reduce_renorm", (0, 0))[1])
+    upd_flops = 6 * unit * T * H * layers * args.steps
+    gemm_upd_ms = trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1]
+    roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_kind": f"bf16_tflops_sustained ({pk_kind})", "traffic": traffic,
+            "flops_per_launch": kflops[dom] / max(launches, 1)}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal q/k/v, L2-normalised per head; no dataset)",
+            "config": workload_config(w, layers), "roofline": roof,
+            "update_gemm_tensor_frac": {
+                "value": upd_flops / (gemm_upd_ms / 1e3) / 1e12 / peak if gemm_upd_ms else None,
+                "of": "bf16_tflops_sustained",
+                "burst_frac": (upd_flops / (gemm_upd_ms / 1e3) / 1e12 / pk["bf16_tflops"]
+                               if gemm_upd_ms else None),
+                "update_ms_per_layer": upd_ms / (layers * args.steps)},
+            "kernels": per_kernel, "clocks": clk,
+            "gpu_launches": int(sum(v[0] for v in trace.values()))}
+
+    # -------------------------------------------------- e2e through host buffers
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta,
+                          Win, Wout, shadow, ws_buf, O, Or, layers, T, M, world, barrier,
+                          max_over_ranks)
+    # -------------------------------------------------- CPU baseline
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta, Win, Wout,
+        shadow, ws_buf, O, Or, layers, T, M, world, barrier, max_over_ranks):
+    """The same step through the public API with the inputs in pinned host
+    memory: every step copies K, V, Q, ray Q, eta and the 24 layers' weights
+    host -> device, runs the stack, and copies every layer's outputs (image
+    and ray O) and updated weights device -> host (on a second stream,
+    overlapped with the next layer)."""
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    pK, pV, pQ, pQr, peta = (pin(t) for t in (hK, hV, hQ, hQr, heta))
+    pW = [tuple(pin(t) for t in ws) for ws in hW]
+    oO = [torch.empty(O.shape, dtype=O.dtype, pin_memory=True) for _ in range(2)]
+    oOr = [torch.empty(Or.shape, dtype=Or.dtype, pin_memory=True) for _ in range(2)]
+    oW = [tuple(torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ws) for ws in Win]
+    st = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
+    h2d = sum(t.numel() * t.element_size() for t in (pK, pV, pQ, pQr, peta)) + \
+        sum(t.numel() * t.element_size() for ws in pW for t in ws)
+    d2h = layers * (O.numel() * O.element_size() + Or.numel() * Or.element_size()) + \
+        sum(t.numel() * t.element_size() for ws in Win for t in ws)
+    # Outputs of layer l go to host buffer l % 2 on the side stream; the
+    # device O/Or buffers are double-buffered too so compute never overwrites
+    # an output still being copied.
+    Ob = [O, torch.empty_like(O)]
+    Orb = [Or, torch.empty_like(Or)]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def one():
+        for src, dst in ((pK, K), (pV, V), (pQ, Q), (pQr, Qr), (peta, eta)):
+            dst.copy_(src, non_blocking=True)
+        for ws_h, ws_d in zip(pW, Win):
+            for a, b in zip(ws_h, ws_d):
+                b.copy_(a, non_blocking=True)
+        for layer in range(layers):
+            b = layer % 2
+            st.wait_event(done[b]) if layer >= 2 else None
+            W1, W2, W3 = Win[layer]
+            a1, a2, a3 = Wout[layer]
+            R.ttt_update(cfg, W1, W2, W3, K, V, eta, a1, a2, a3, shadow=shadow,
+                         workspace=ws_buf, stream=st)
+            R.ttt_apply(cfg, Q, Ob[b], shadow=shadow, stream=st)
+            if M:
+                R.ttt_apply(cfg, Qr, Orb[b], shadow=shadow, stream=st)
+            ev = torch.cuda.Event()
+            ev.record(st)
+            side.wait_event(ev)
+            with torch.cuda.stream(side):
+                oO[b].copy_(Ob[b], non_blocking=True)
+                oOr[b].copy_(Orb[b], non_blocking=True)
+                for t_h, t_d in zip(oW[layer], Wout[layer]):
+                    t_h.copy_(t_d, non_blocking=True)
+            done[b].record(side)
+        st.wait_stream(side)
+
+    one()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.e2e_steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
+    return {"value": world * T * layers / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": args.e2e_steps}
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "recon_chunk_ttt_b200", "csrc"))):
+        with open(os.path.join(ROOT, "recon_chunk_ttt_b200", "csrc", f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+    else:
+        run_ours(args, w, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

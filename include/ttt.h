@@ -21,8 +21,9 @@
  *
  * Conventions shared by every entry point
  *  - All pointers except `cfg` are DEVICE pointers on the current CUDA device,
- *    owned by the caller; the library allocates nothing and keeps no state
- *    between calls apart from one device error word per device.
+ *    owned by the caller; the library allocates no device memory and keeps no
+ *    state between calls apart from one device error word per device and the
+ *    optional tracing totals (ttt_trace_enable).
  *  - Every call is asynchronous on `stream` (NULL = the legacy default
  *    stream); arguments are validated on the host before anything is
  *    enqueued, so an error status means nothing was launched.
@@ -147,6 +148,25 @@ ttt_status ttt_stream_step(const ttt_config* cfg,
  * is not NULL) or TTT_ERR_CUDA.
  */
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
+
+/*
+ * Tracing.  With tracing on, every kernel launch of the library is bracketed
+ * by two CUDA events on the caller's stream (host-side state: an event pool
+ * and per-kernel totals, guarded by a mutex).  ttt_trace_read synchronises
+ * the recorded events, adds their elapsed times to per-kernel totals and
+ * copies up to `capacity` entries (name, launches, total milliseconds) into
+ * `entries`; *count receives the number of kernel names seen.  reset != 0
+ * clears the totals after reading.  Off by default.
+ */
+typedef struct {
+  char name[32];
+  int64_t launches;
+  double total_ms;
+} ttt_trace_entry;
+
+ttt_status ttt_trace_enable(int32_t on);
+ttt_status ttt_trace_read(ttt_trace_entry* entries, int32_t capacity, int32_t* count,
+                          int32_t reset);
 
 #ifdef __cplusplus
 }

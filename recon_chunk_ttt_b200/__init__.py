@@ -4,7 +4,8 @@ The layer runs in libttt.so (C ABI in include/ttt.h); ``recon_chunk_ttt_b200``
 exposes the same entry points through a thin ctypes binding:
 
     ttt_update, ttt_apply, ttt_stream_step, ttt_pack_shadow,
-    ttt_update_workspace_bytes, ttt_shadow_bytes, ttt_check_device_error
+    ttt_update_workspace_bytes, ttt_shadow_bytes, ttt_check_device_error,
+    ttt_trace_enable, ttt_trace_read
 
 The binding (and torch) is imported on first use, so ``workloads`` can be
 imported on machines without CUDA.
@@ -16,7 +17,7 @@ _EXPORTS = {
     "ttt_update_workspace_bytes", "ttt_shadow_bytes", "ttt_check_device_error",
     "ttt_config", "make_config", "alloc_workspace", "alloc_shadow", "status_string",
     "TTTError", "lib", "RENORM_OFF", "RENORM_ROW", "RENORM_FROB", "PREC_BF16_TC",
-    "PREC_FP32_CHECK", "LIB_PATH",
+    "PREC_FP32_CHECK", "LIB_PATH", "ttt_trace_enable", "ttt_trace_read",
 }
 
 

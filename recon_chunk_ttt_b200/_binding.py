@@ -35,6 +35,11 @@ def make_config(heads: int, d: int, hidden: int, renorm: int = RENORM_ROW,
     return ttt_config(heads, d, hidden, mlp, renorm, ns_steps, precision)
 
 
+class ttt_trace_entry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double)]
+
+
 class TTTError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -73,6 +78,11 @@ def lib() -> ctypes.CDLL:
         L.ttt_stream_step.restype = ctypes.c_int
         L.ttt_check_device_error.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
         L.ttt_check_device_error.restype = ctypes.c_int
+        L.ttt_trace_enable.argtypes = [ctypes.c_int32]
+        L.ttt_trace_enable.restype = ctypes.c_int
+        L.ttt_trace_read.argtypes = [ctypes.POINTER(ttt_trace_entry), ctypes.c_int32,
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+        L.ttt_trace_read.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -182,3 +192,19 @@ def ttt_check_device_error(stream=None) -> int:
     if st != TTT_OK:
         raise TTTError(st, f"device error word = {code.value}")
     return code.value
+
+
+def ttt_trace_enable(on: bool = True) -> None:
+    """Bracket every kernel launch of the library with CUDA events."""
+    _check(lib().ttt_trace_enable(1 if on else 0), "ttt_trace_enable")
+
+
+def ttt_trace_read(reset: bool = True) -> dict:
+    """{kernel name: (launches, total device ms)} since the last reset."""
+    cap = 64
+    arr = (ttt_trace_entry * cap)()
+    cnt = ctypes.c_int32(0)
+    _check(lib().ttt_trace_read(arr, cap, ctypes.byref(cnt), 1 if reset else 0),
+           "ttt_trace_read")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms))
+            for i in range(min(cnt.value, cap))}

@@ -57,6 +57,22 @@ cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const vo
 int* device_error_ptr();                       // device address, nullptr on failure
 cudaError_t read_and_clear_device_error(int* value);
 
+// Tracing (trace.cu): a scope records CUDA events around the launches it
+// encloses when tracing is enabled through ttt_trace_enable().
+bool trace_on();
+class TraceScope {
+ public:
+  TraceScope(const char* name, cudaStream_t st);
+  ~TraceScope();
+  TraceScope(const TraceScope&) = delete;
+  TraceScope& operator=(const TraceScope&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t st_;
+  void* a_;
+};
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace ttt

@@ -154,6 +154,7 @@ cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const 
                           __nv_bfloat16_raw* shadow, float* scratch, cudaStream_t st) {
   const int rows = p.H * (2 * p.hid + p.d);
   const int blocks = (rows * 32 + 255) / 256;
+  TraceScope ts("reduce_renorm", st);
   reduce_renorm_kernel<<<blocks, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, p.renorm, W1, W2,
                                               W3, W1o, W2o, W3o, shadow,
                                               reinterpret_cast<double*>(scratch));
@@ -186,6 +187,7 @@ cudaError_t pack_shadow(int H, int d, int hid, const float* W1, const float* W2,
   const size_t total = (size_t)H * hid * d;
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 8) blocks = 148 * 8;
+  TraceScope ts("pack_shadow", st);
   pack_shadow_kernel<<<blocks, 256, 0, st>>>(total, W1, W2, W3, shadow);
   return cudaGetLastError();
 }

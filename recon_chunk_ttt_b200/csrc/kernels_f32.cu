@@ -284,11 +284,17 @@ cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const
   float* scratch = reinterpret_cast<float*>(w);
   if (p.n > 0) {
     dim3 g1((unsigned)((p.n + kT - 1) / kT), p.hid / kJ, p.H);
-    f32_fwd_bwd_kernel<<<g1, 256, 0, st>>>(K, V, eta, W1, W2, W3, p.n, p.H, p.d, p.hid, U, DH1,
-                                          DH3);
+    {
+      TraceScope ts("f32_fwd_bwd", st);
+      f32_fwd_bwd_kernel<<<g1, 256, 0, st>>>(K, V, eta, W1, W2, W3, p.n, p.H, p.d, p.hid, U, DH1,
+                                            DH3);
+    }
     dim3 g2((p.hid / kJ) * (p.d / kJ), 3 * p.H, sp.S);
-    f32_grad_kernel<<<g2, 256, 0, st>>>(U, DH1, DH3, K, V, p.n, p.H, p.d, p.hid, sp.chunk,
-                                       partials);
+    {
+      TraceScope ts("f32_grad", st);
+      f32_grad_kernel<<<g2, 256, 0, st>>>(U, DH1, DH3, K, V, p.n, p.H, p.d, p.hid, sp.chunk,
+                                         partials);
+    }
   } else {
     cudaMemsetAsync(partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * sizeof(float), st);
   }
@@ -305,6 +311,7 @@ cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 g((unsigned)((p.n + kQ - 1) / kQ), p.H);
+  TraceScope ts("f32_apply", st);
   f32_apply_kernel<<<g, 256, smem, st>>>(Q, W1, W2, W3, p.n, p.H, p.d, p.hid, O);
   return cudaGetLastError();
 }

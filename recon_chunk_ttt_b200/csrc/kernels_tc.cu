@@ -823,7 +823,10 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   if (p.n > 0) {
     int cb = (int)((wsz + 255) / 256);
     if (cb > 1184) cb = 1184;
-    convert_weights_kernel<<<cb, 256, 0, st>>>(p.H, p.d, p.hid, W1, W2, W3, w.b1, w.b3, w.b2t);
+    {
+      TraceScope ts("tc_convert_weights", st);
+      convert_weights_kernel<<<cb, 256, 0, st>>>(p.H, p.d, p.hid, W1, W2, W3, w.b1, w.b3, w.b2t);
+    }
     CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg;
     const uint64_t ld = (uint64_t)p.H * D;
     {
@@ -856,8 +859,11 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     cudaError_t e = cudaFuncSetAttribute(fb_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          FB<D>::SMEM);
     if (e != cudaSuccess) return e;
-    fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
-        mK, mV, mW1, mW3, mW2t, eta, p.n, p.H, p.hid, items, w.U, w.DH1, w.DH3, err);
+    {
+      TraceScope ts("tc_fwd_bwd", st);
+      fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
+          mK, mV, mW1, mW3, mW2t, eta, p.n, p.H, p.hid, items, w.U, w.DH1, w.DH3, err);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int tiles = p.hid / BM;
@@ -865,8 +871,11 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     e = cudaFuncSetAttribute(grad_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GR<D>::SMEM);
     if (e != cudaSuccess) return e;
-    grad_kernel<D><<<sp.S * (k0 + k1), GR<D>::THREADS, GR<D>::SMEM, st>>>(
-        mDH1, mDH3, mU, mKg, mVg, p.n, p.H, p.hid, sp.chunk, k0, k1, w.partials, err);
+    {
+      TraceScope ts("tc_grad", st);
+      grad_kernel<D><<<sp.S * (k0 + k1), GR<D>::THREADS, GR<D>::SMEM, st>>>(
+          mDH1, mDH3, mU, mKg, mVg, p.n, p.H, p.hid, sp.chunk, k0, k1, w.partials, err);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   } else {
@@ -907,8 +916,11 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, AP<D>::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.n + BM - 1) / BM), p.H);
-  apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
-      mQ, mW1, mW3, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
+  {
+    TraceScope ts("tc_apply", st);
+    apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
+        mQ, mW1, mW3, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
+  }
   return cudaGetLastError();
 }
 

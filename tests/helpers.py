@@ -68,9 +68,17 @@ def oracle_update_apply(x: wl.LayerInputs, precision: int, renorm: int):
     return Wh, O.ttt_apply(*Wh, xo.Q)
 
 
+def as_output_type(W_ref):
+    """The oracle's Ŵ rounded to the library's output type (fp32).  Ŵ - W taken
+    from an fp32 Ŵ cannot be finer than ulp(W); comparing with the rounded
+    reference removes that floor (which dominates when the update is tiny,
+    e.g. one token) and leaves the kernels' own error."""
+    return np.asarray(W_ref, dtype=np.float32).astype(np.float64)
+
+
 def rel_errors(gpu, ref, x):
     """Relative Frobenius errors on Ŵ - W (per matrix) and on O."""
     W = (x.W1, x.W2, x.W3)
-    errs = [O.rel_fro(g - w, r - w) for g, r, w in zip(gpu[:3], ref[0], W)]
+    errs = [O.rel_fro(g - w, as_output_type(r) - w) for g, r, w in zip(gpu[:3], ref[0], W)]
     errs.append(O.rel_fro(gpu[3], ref[1]))
     return errs

@@ -9,8 +9,8 @@ import pytest
 import oracle as O
 from recon_chunk_ttt_b200 import workloads as wl
 
-from helpers import (TOL_F32, TOL_TC, gpu_inputs, oracle_update_apply, rel_errors,
-                     run_update_apply, to_dev)
+from helpers import (TOL_F32, TOL_TC, as_output_type, gpu_inputs, oracle_update_apply,
+                     rel_errors, run_update_apply, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -161,7 +161,8 @@ def test_stream_first_frames_vs_oracle(precision, tol):
     xo = oracle_inputs(x, precision)
     Ws, ref_out = O.ttt_stream(xo.W1, xo.W2, xo.W3, xo.K, xo.V, xo.eta, xo.Q, p)
     gpu = [t.cpu().double().numpy() for t in (W1, W2, W3)]
-    errs = [O.rel_fro(g_ - w_, r - w_) for g_, r, w_ in zip(gpu, Ws, (x.W1, x.W2, x.W3))]
+    errs = [O.rel_fro(g_ - w_, as_output_type(r) - w_)
+            for g_, r, w_ in zip(gpu, Ws, (x.W1, x.W2, x.W3))]
     errs.append(O.rel_fro(out.float().cpu().double().numpy(), ref_out))
     assert max(errs) <= tol, errs
 
