@@ -52,16 +52,26 @@ def test_scale100_bf16():
 
 
 # ------------------------------------------------------- ragged / edge sizes
+def _eta_scale(n, precision):
+    """With a handful of tokens the update is ~1e-4 of W, below what an fp32 Ŵ
+    resolves at 1e-5 relative on Ŵ - W (a one-ulp difference in W - g already
+    exceeds it); the fp32 check of those sizes uses larger write strengths so
+    the update is large enough to be measured.  The bf16 path keeps eta as is."""
+    return max(1.0, 2000.0 / n) if precision == R.PREC_FP32_CHECK else 1.0
+
+
 @pytest.mark.parametrize("n", [1, 63, 127, 129, 1000, 4097])
 @pytest.mark.parametrize("precision,tol", PRECS)
 def test_ragged_d256(n, precision, tol):
-    _check(wl.random_layer(100 + n, n, 2, 256, 512), precision, tol)
+    x = wl.random_layer(100 + n, n, 2, 256, 512, eta_scale=_eta_scale(n, precision))
+    _check(x, precision, tol)
 
 
 @pytest.mark.parametrize("n,H", [(1, 3), (65, 3), (300, 2), (1001, 1)])
 @pytest.mark.parametrize("precision,tol", PRECS)
 def test_ragged_d64(n, H, precision, tol):
-    _check(wl.random_layer(200 + n, n, H, 64, 128), precision, tol)
+    x = wl.random_layer(200 + n, n, H, 64, 128, eta_scale=_eta_scale(n, precision))
+    _check(x, precision, tol)
 
 
 @pytest.mark.parametrize("renorm", [0, 2])
@@ -113,12 +123,10 @@ def test_token_permutation(precision, tol):
 @pytest.mark.parametrize("precision", [R.PREC_BF16_TC, R.PREC_FP32_CHECK])
 def test_zero_eta_padding(precision):
     x = wl.random_layer(12, 1000, 2, 256, 512)
-    rng = np.random.default_rng(1)
     pad = wl.random_layer(13, 300, 2, 256, 512)
     xp = wl.LayerInputs(x.W1, x.W2, x.W3, np.concatenate([x.K, pad.K]),
                         np.concatenate([x.V, pad.V]), x.Q,
                         np.concatenate([x.eta, np.zeros_like(pad.eta)]), None)
-    del rng
     a = run_update_apply(x, precision, R.RENORM_ROW)
     b = run_update_apply(xp, precision, R.RENORM_ROW)
     errs = [O.rel_fro(u - w, v - w) for u, v, w in zip(a[:3], b[:3], (x.W1, x.W2, x.W3))]
