@@ -125,16 +125,36 @@ struct FB {
   static constexpr int OFF_STAGE = OFF_W2 + NCH * W2_CH;
   static constexpr int OFF_BAR = OFF_STAGE + NSTAGE * STAGE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;       // + alignment slack
-  static constexpr int THREADS = 192;                     // producer, MMA, 4 epilogue warps
+  static constexpr int EPI_WARPS = 8;                     // 2 per TMEM lane quadrant
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;     // producer, MMA, epilogue
   static constexpr uint32_t TMEM_COLS = 512;              // 2 x (F13 128 + DU 64), at 0 / 256
 };
+
+// Work items are (head*nslices + slice, token tile) pairs.  With reps > 0 the
+// grid is groups*reps CTAs: CTA b owns group b / reps and the token tiles
+// [r*ntiles/reps, (r+1)*ntiles/reps), r = b % reps, so the hidden slices of one
+// head walk the same k/v tiles in lockstep and share them through L2.  With
+// reps == 0 (more groups than CTAs) each CTA takes a contiguous range of the
+// flattened item space.
+__device__ __forceinline__ void fb_item_range(int64_t ntiles, int groups, int reps,
+                                              int64_t& it0, int64_t& it1) {
+  if (reps > 0) {
+    const int64_t g = blockIdx.x / reps, r = blockIdx.x % reps;
+    it0 = g * ntiles + r * ntiles / reps;
+    it1 = g * ntiles + (r + 1) * ntiles / reps;
+  } else {
+    const int64_t total = (int64_t)groups * ntiles;
+    it0 = total * blockIdx.x / gridDim.x;
+    it1 = total * (blockIdx.x + 1) / gridDim.x;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(FB<D>::THREADS, 1)
     fb_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
               const __grid_constant__ CUtensorMap mW1, const __grid_constant__ CUtensorMap mW3,
               const __grid_constant__ CUtensorMap mW2t, const float* __restrict__ eta, int64_t n,
-              int H, int hid, int64_t total_items, __nv_bfloat16* __restrict__ U,
+              int H, int hid, int reps, __nv_bfloat16* __restrict__ U,
               __nv_bfloat16* __restrict__ DH1, __nv_bfloat16* __restrict__ DH3, int* err) {
   using L = FB<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -152,8 +172,8 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nslices = hid / HS;
   const int64_t ntiles = (n + BM - 1) / BM;
-  const int64_t it0 = total_items * blockIdx.x / gridDim.x;
-  const int64_t it1 = total_items * (blockIdx.x + 1) / gridDim.x;
+  int64_t it0, it1;
+  fb_item_range(ntiles, H * nslices, reps, it0, it1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::NSTAGE; ++s) {
@@ -164,7 +184,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
     mbar_init(wempty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], L::EPI_WARPS);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -232,7 +252,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
     const uint32_t idU = idesc_bf16_f32(BM, HS, false, false);
     int stage = 0;
     uint32_t phase = 0, wphase = 0;
-    uint32_t aphase[2] = {0, 0};
+    uint32_t abits = 0;  // bit b: phase parity of accumulator buffer b
     int cur_hs = -1, buf = 0;
     bool ok = true;
     const uint32_t sbase = smem_u32(smem);
@@ -244,7 +264,8 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
         wphase ^= 1;
         cur_hs = hs;
       }
-      if (!mbar_wait(&acc_empty[buf], aphase[buf] ^ 1, abort_flag, err, kErrWaitAccFree)) {
+      if (!mbar_wait(&acc_empty[buf], ((abits >> buf) & 1) ^ 1, abort_flag, err,
+                     kErrWaitAccFree)) {
         ok = false;
         break;
       }
@@ -271,7 +292,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
         }
       }
       umma_commit(&acc_full[buf]);
-      aphase[buf] ^= 1;
+      abits ^= 1u << buf;
       buf ^= 1;
     }
     // Wait for every MMA issued by this thread before TMEM is released.
@@ -280,65 +301,64 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
     mbar_wait(done, 0, &never, err, kErrWaitFinal);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant of this warp
-    uint32_t aphase[2] = {0, 0};
+    // Two warps per TMEM lane quadrant; warp half `ch` takes hidden columns
+    // [32*ch, 32*ch+32) of the slice.
+    const int q = warp & 3;
+    const int ch = (warp - 2) / 4;
+    uint32_t abits = 0;
     int buf = 0;
     for (int64_t it = it0; it < it1; ++it) {
       const int hs = (int)(it / ntiles);
       const int64_t tile = it % ntiles;
       const int head = hs / nslices, slice = hs % nslices;
-      const bool got = mbar_wait(&acc_full[buf], aphase[buf], abort_flag, err, kErrWaitAcc);
+      const bool got =
+          mbar_wait(&acc_full[buf], (abits >> buf) & 1, abort_flag, err, kErrWaitAcc);
       __syncwarp();
       if (!got) break;
-      aphase[buf] ^= 1;
+      abits ^= 1u << buf;
       tc_fence_after();
       const int64_t tok = tile * BM + q * 32 + lane;
       const bool live = tok < n;
       const float ne = live ? -eta[tok * H + head] : 0.f;  // -η: du = -(W2^T v)
-      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256;
-      const size_t orow = ((size_t)head * n + (live ? tok : 0)) * hid + slice * HS;
+      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256 + ch * 32;
+      uint32_t r1[32], r3[32], rd[32];
+      tmem_ld_32x32(tl, r1);
+      tmem_ld_32x32(tl + HS, r3);
+      tmem_ld_32x32(tl + 128, rd);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      uint32_t pu[16], p1[16], p3[16];
 #pragma unroll
-      for (int half = 0; half < HS / 32; ++half) {
-        uint32_t r1[32], r3[32], rd[32];
-        tmem_ld_32x32(tl + half * 32, r1);
-        tmem_ld_32x32(tl + HS + half * 32, r3);
-        tmem_ld_32x32(tl + 128 + half * 32, rd);
-        tmem_ld_wait();
-        if (half == HS / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      for (int i = 0; i < 32; i += 2) {
+        float o_u[2], o_1[2], o_3[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float h1 = __uint_as_float(r1[i + e]);
+          const float h3 = __uint_as_float(r3[i + e]);
+          const float edu = ne * __uint_as_float(rd[i + e]);  // η du
+          const float s = sigmoid_fast(h1);
+          const float a = h1 * s;                             // SiLU(h1)
+          const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
+          o_u[e] = -ne * (a * h3);
+          o_3[e] = edu * a;
+          o_1[e] = edu * h3 * dsl;
         }
-        uint32_t pu[16], p1[16], p3[16];
+        pu[i / 2] = pack_bf16x2(o_u[0], o_u[1]);
+        p1[i / 2] = pack_bf16x2(o_1[0], o_1[1]);
+        p3[i / 2] = pack_bf16x2(o_3[0], o_3[1]);
+      }
+      if (live) {
+        const size_t orow = ((size_t)head * n + tok) * hid + slice * HS + ch * 32;
+        uint4* du_ = reinterpret_cast<uint4*>(U + orow);
+        uint4* d1_ = reinterpret_cast<uint4*>(DH1 + orow);
+        uint4* d3_ = reinterpret_cast<uint4*>(DH3 + orow);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float o_u[2], o_1[2], o_3[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float h1 = __uint_as_float(r1[i + e]);
-            const float h3 = __uint_as_float(r3[i + e]);
-            const float edu = ne * __uint_as_float(rd[i + e]);  // η du
-            const float s = sigmoid_fast(h1);
-            const float a = h1 * s;                             // SiLU(h1)
-            const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
-            o_u[e] = -ne * (a * h3);
-            o_3[e] = edu * a;
-            o_1[e] = edu * h3 * dsl;
-          }
-          pu[i / 2] = pack_bf16x2(o_u[0], o_u[1]);
-          p1[i / 2] = pack_bf16x2(o_1[0], o_1[1]);
-          p3[i / 2] = pack_bf16x2(o_3[0], o_3[1]);
-        }
-        if (live) {
-          uint4* du_ = reinterpret_cast<uint4*>(U + orow + half * 32);
-          uint4* d1_ = reinterpret_cast<uint4*>(DH1 + orow + half * 32);
-          uint4* d3_ = reinterpret_cast<uint4*>(DH3 + orow + half * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            du_[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
-            d1_[v] = make_uint4(p1[4 * v], p1[4 * v + 1], p1[4 * v + 2], p1[4 * v + 3]);
-            d3_[v] = make_uint4(p3[4 * v], p3[4 * v + 1], p3[4 * v + 2], p3[4 * v + 3]);
-          }
+        for (int v = 0; v < 4; ++v) {
+          du_[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+          d1_[v] = make_uint4(p1[4 * v], p1[4 * v + 1], p1[4 * v + 2], p1[4 * v + 3]);
+          d3_[v] = make_uint4(p3[4 * v], p3[4 * v + 1], p3[4 * v + 2], p3[4 * v + 3]);
         }
       }
       buf ^= 1;
@@ -530,10 +550,18 @@ struct AP {
   static constexpr int OFF_U = OFF_STAGE + NSTAGE * STAGE;  // 2 x [128 x 128 B]
   static constexpr int OFF_BAR = OFF_U + 2 * BM * 128;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int EPI_WARPS = 8;                    // 2 per TMEM lane quadrant
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr uint32_t TMEM_COLS = 512;             // F[0] 0, F[1] 128, O at 256
 };
 
+// Persistent: CTA b takes (query tile, head) items b, b + grid, ...  Per item
+// and 64-wide hidden slice js: F(js) = Q [W1s; W3s]^T into TMEM buffer js&1,
+// the epilogue turns it into u = SiLU(h1) ⊙ h3 (bf16, shared memory), and
+// O += u W2s^T.  The MMA issuer runs F(js+1) before O(js) so the epilogue of
+// slice js overlaps an MMA; the q chunks are released one by one during the
+// last slice so the next item's q streams in early; O is drained while the
+// next item's first F MMAs run.
 template <int D>
 __global__ void __launch_bounds__(AP<D>::THREADS, 1)
     apply_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW1,
@@ -544,35 +572,41 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* empty = full + L::NSTAGE;
-  uint64_t* q_full = empty + L::NSTAGE;
-  uint64_t* f_full = q_full + 1;
+  uint64_t* q_full = empty + L::NSTAGE;  // one per d-chunk
+  uint64_t* q_empty = q_full + L::NCH;
+  uint64_t* f_full = q_empty + L::NCH;
   uint64_t* f_empty = f_full + 2;
   uint64_t* u_full = f_empty + 2;
   uint64_t* u_empty = u_full + 2;
   uint64_t* o_full = u_empty + 2;
-  uint64_t* done = o_full + 1;
+  uint64_t* o_empty = o_full + 1;
+  uint64_t* done = o_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t qt = blockIdx.x;
-  const int head = blockIdx.y;
   const int nsl = hid / HS;
   const int w13_stages = L::NCH / L::CH_PER_STAGE;
+  const int64_t nqt = (m + BM - 1) / BM;
+  const int64_t items = nqt * H;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NSTAGE; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(q_full, 1);
+    for (int c = 0; c < L::NCH; ++c) {
+      mbar_init(&q_full[c], 1);
+      mbar_init(&q_empty[c], 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&f_full[b], 1);
-      mbar_init(&f_empty[b], 4);
-      mbar_init(&u_full[b], 4);
+      mbar_init(&f_empty[b], L::EPI_WARPS);
+      mbar_init(&u_full[b], L::EPI_WARPS);
       mbar_init(&u_empty[b], 1);
     }
     mbar_init(o_full, 1);
+    mbar_init(o_empty, L::EPI_WARPS);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -588,12 +622,10 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    mbar_arrive_expect_tx(q_full, L::NCH * BM * 128);
-    for (int c = 0; c < L::NCH; ++c)
-      tma_load_2d(smem + L::OFF_Q + c * BM * 128, &mQ, q_full, head * D + c * CH, (int)(qt * BM));
+    tma_prefetch_desc(&mQ);
     int stage = 0;
     uint32_t phase = 0;
-    int64_t issued = 0;
+    int64_t issued = 0, qloads = 0;
     bool ok = true;
     auto next = [&]() -> uint8_t* {
       if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) return nullptr;
@@ -603,34 +635,48 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       ++issued;
       if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
     };
-    auto load_w13 = [&](int js) {
-      for (int g = 0; g < w13_stages && ok; ++g) {
+    for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
+      const int64_t qt = it / H;
+      const int head = (int)(it % H);
+      for (int c = 0; c < L::NCH && ok; ++c) {
+        if (!mbar_wait(&q_empty[c], (uint32_t)(i & 1) ^ 1, abort_flag, err, kErrWaitEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[c], BM * 128);
+        tma_load_2d(smem + L::OFF_Q + c * BM * 128, &mQ, &q_full[c], head * D + c * CH,
+                    (int)(qt * BM));
+      }
+      ++qloads;
+      auto load_w13 = [&](int js) {
+        for (int g = 0; g < w13_stages && ok; ++g) {
+          uint8_t* st = next();
+          if (!st) { ok = false; return; }
+          mbar_arrive_expect_tx(&full[stage], L::CH_PER_STAGE * L::W13_CH);
+          for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
+            const int c = g * L::CH_PER_STAGE + cc;
+            tma_load_2d(st + cc * L::W13_CH, &mW1, &full[stage], c * CH, head * hid + js * HS);
+            tma_load_2d(st + cc * L::W13_CH + HS * 128, &mW3, &full[stage], c * CH,
+                        head * hid + js * HS);
+          }
+          advance();
+        }
+      };
+      auto load_w2 = [&](int js) {
         uint8_t* st = next();
         if (!st) { ok = false; return; }
-        mbar_arrive_expect_tx(&full[stage], L::CH_PER_STAGE * L::W13_CH);
-        for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
-          const int c = g * L::CH_PER_STAGE + cc;
-          tma_load_2d(st + cc * L::W13_CH, &mW1, &full[stage], c * CH, head * hid + js * HS);
-          tma_load_2d(st + cc * L::W13_CH + HS * 128, &mW3, &full[stage], c * CH,
-                      head * hid + js * HS);
-        }
+        mbar_arrive_expect_tx(&full[stage], D * 128);
+        tma_load_2d(st, &mW2, &full[stage], js * HS, head * D);
         advance();
+      };
+      for (int js = 0; js < nsl && ok; ++js) {
+        load_w13(js);
+        if (js >= 1 && ok) load_w2(js - 1);
       }
-    };
-    auto load_w2 = [&](int js) {
-      uint8_t* st = next();
-      if (!st) { ok = false; return; }
-      mbar_arrive_expect_tx(&full[stage], D * 128);
-      tma_load_2d(st, &mW2, &full[stage], js * HS, head * D);
-      advance();
-    };
-    for (int js = 0; js < nsl && ok; ++js) {
-      load_w13(js);
-      if (js >= 1 && ok) load_w2(js - 1);
+      if (ok) load_w2(nsl - 1);
     }
-    if (ok) load_w2(nsl - 1);
     drain_ring(full, L::NSTAGE, issued, err);
-    drain_ring(q_full, 1, 1, err);
+    for (int c = 0; c < L::NCH; ++c) drain_ring(&q_full[c], 1, qloads, err);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idF = idesc_bf16_f32(BM, 2 * HS, false, false);
@@ -638,9 +684,7 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
     const uint32_t sbase = smem_u32(smem);
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t fph[2] = {0, 0}, uph[2] = {0, 0};
-    bool ok = mbar_wait(q_full, 0, abort_flag, err, kErrWaitFull);
-    tc_fence_after();
+    bool ok = true;
     auto take = [&]() -> bool {
       if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) return false;
       tc_fence_after();
@@ -650,10 +694,14 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       umma_commit(&empty[stage]);
       if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
     };
-    auto do_o = [&](int j) -> bool {
-      const int b = j & 1;
-      if (!mbar_wait(&u_full[b], uph[b], abort_flag, err, kErrWaitOperand)) return false;
-      uph[b] ^= 1;
+    // g = global slice counter: buffer g&1, its (g>>1)-th use.
+    auto do_o = [&](int64_t g, int j, int64_t item_i) -> bool {
+      const int b = (int)(g & 1);
+      const uint32_t par = (uint32_t)((g >> 1) & 1);
+      if (!mbar_wait(&u_full[b], par, abort_flag, err, kErrWaitOperand)) return false;
+      if (j == 0 &&
+          !mbar_wait(o_empty, (uint32_t)(item_i & 1) ^ 1, abort_flag, err, kErrWaitAccFree))
+        return false;
       tc_fence_after();
       if (!take()) return false;
       const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
@@ -666,85 +714,105 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       umma_commit(&u_empty[b]);
       return true;
     };
-    for (int js = 0; js < nsl && ok; ++js) {
-      const int b = js & 1;
-      if (!mbar_wait(&f_empty[b], fph[b] ^ 1, abort_flag, err, kErrWaitAccFree)) { ok = false; break; }
-      fph[b] ^= 1;
-      tc_fence_after();
-      for (int g = 0; g < w13_stages && ok; ++g) {
-        if (!take()) { ok = false; break; }
-        const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
-        for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
-          const int c = g * L::CH_PER_STAGE + cc;
-          const uint32_t qa = sbase + L::OFF_Q + c * BM * 128;
-#pragma unroll
-          for (int kk = 0; kk < CH / 16; ++kk)
-            umma_bf16(tmem + b * 128, sdesc_sw128(qa + kk * KSTEP_BYTES, 16, 1024),
-                      sdesc_sw128(st + cc * L::W13_CH + kk * KSTEP_BYTES, 16, 1024), idF,
-                      (c | kk) != 0);
+    for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
+      for (int js = 0; js < nsl && ok; ++js) {
+        const int64_t g = i * nsl + js;
+        const int b = (int)(g & 1);
+        if (!mbar_wait(&f_empty[b], (uint32_t)((g >> 1) & 1) ^ 1, abort_flag, err,
+                       kErrWaitAccFree)) {
+          ok = false;
+          break;
         }
-        release();
+        tc_fence_after();
+        for (int gs = 0; gs < w13_stages && ok; ++gs) {
+          if (!take()) { ok = false; break; }
+          const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
+          for (int cc = 0; cc < L::CH_PER_STAGE && ok; ++cc) {
+            const int c = gs * L::CH_PER_STAGE + cc;
+            if (js == 0) {
+              if (!mbar_wait(&q_full[c], (uint32_t)(i & 1), abort_flag, err, kErrWaitFull)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            const uint32_t qa = sbase + L::OFF_Q + c * BM * 128;
+#pragma unroll
+            for (int kk = 0; kk < CH / 16; ++kk)
+              umma_bf16(tmem + b * 128, sdesc_sw128(qa + kk * KSTEP_BYTES, 16, 1024),
+                        sdesc_sw128(st + cc * L::W13_CH + kk * KSTEP_BYTES, 16, 1024), idF,
+                        (c | kk) != 0);
+            if (js == nsl - 1) umma_commit(&q_empty[c]);  // q chunk c no longer needed
+          }
+          release();
+        }
+        if (!ok) break;
+        umma_commit(&f_full[b]);
+        if (js >= 1 && !do_o(g - 1, js - 1, i)) { ok = false; break; }
       }
       if (!ok) break;
-      umma_commit(&f_full[b]);
-      if (js >= 1 && !do_o(js - 1)) { ok = false; break; }
+      if (!do_o(i * nsl + nsl - 1, nsl - 1, i)) break;
+      umma_commit(o_full);
     }
-    if (ok && do_o(nsl - 1)) umma_commit(o_full);
     umma_commit(done);
     volatile int never = 0;
     mbar_wait(done, 0, &never, err, kErrWaitFinal);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
+    const int ch = (warp - 2) / 4;  // hidden columns [32ch, 32ch+32) of a slice
     const int row = q * 32 + lane;
-    const int64_t qi = qt * BM + row;
-    uint32_t fph[2] = {0, 0}, uph[2] = {0, 0};
     bool ok = true;
-    for (int js = 0; js < nsl && ok; ++js) {
-      const int b = js & 1;
-      const bool got = mbar_wait(&f_full[b], fph[b], abort_flag, err, kErrWaitAcc);
-      __syncwarp();
-      if (!got) { ok = false; break; }
-      fph[b] ^= 1;
-      tc_fence_after();
-      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + b * 128;
-      uint32_t pk[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+    for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
+      const int64_t qt = it / H;
+      const int head = (int)(it % H);
+      const int64_t qi = qt * BM + row;
+      for (int js = 0; js < nsl && ok; ++js) {
+        const int64_t g = i * nsl + js;
+        const int b = (int)(g & 1);
+        const uint32_t par = (uint32_t)((g >> 1) & 1);
+        const bool got = mbar_wait(&f_full[b], par, abort_flag, err, kErrWaitAcc);
+        __syncwarp();
+        if (!got) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + b * 128 + ch * 32;
         uint32_t r1[32], r3[32];
-        tmem_ld_32x32(tl + half * 32, r1);
-        tmem_ld_32x32(tl + HS + half * 32, r3);
+        tmem_ld_32x32(tl, r1);
+        tmem_ld_32x32(tl + HS, r3);
         tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&f_empty[b]);
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float h1a = __uint_as_float(r1[i]), h1b = __uint_as_float(r1[i + 1]);
-          const float ua = h1a * sigmoid_fast(h1a) * __uint_as_float(r3[i]);
-          const float ub = h1b * sigmoid_fast(h1b) * __uint_as_float(r3[i + 1]);
-          pk[half * 16 + i / 2] = pack_bf16x2(ua, ub);
+        for (int k = 0; k < 32; k += 2) {
+          const float h1a = __uint_as_float(r1[k]), h1b = __uint_as_float(r1[k + 1]);
+          const float ua = h1a * sigmoid_fast(h1a) * __uint_as_float(r3[k]);
+          const float ub = h1b * sigmoid_fast(h1b) * __uint_as_float(r3[k + 1]);
+          pk[k / 2] = pack_bf16x2(ua, ub);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&f_empty[b]);
-      if (!mbar_wait(&u_empty[b], uph[b] ^ 1, abort_flag, err, kErrWaitOperand)) { ok = false; break; }
-      uph[b] ^= 1;
-      // K-major 128-byte-swizzled row: 16-byte chunk c of row r sits at
-      // chunk position c ^ (r % 8).
-      uint8_t* urow = smem + L::OFF_U + b * BM * 128 + (row / 8) * 1024 + (row % 8) * 128;
+        if (!mbar_wait(&u_empty[b], par ^ 1, abort_flag, err, kErrWaitOperand)) {
+          ok = false;
+          break;
+        }
+        // K-major 128-byte-swizzled row: 16-byte chunk c of row r sits at
+        // chunk position c ^ (r % 8).
+        uint8_t* urow = smem + L::OFF_U + b * BM * 128 + (row / 8) * 1024 + (row % 8) * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(urow + ((c ^ (row % 8)) * 16)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(urow + (((ch * 4 + c) ^ (row % 8)) * 16)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&u_full[b]);
+      }
+      if (!ok) break;
+      const bool got_o = mbar_wait(o_full, (uint32_t)(i & 1), abort_flag, err, kErrWaitAcc);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&u_full[b]);
-    }
-    const bool got_o = ok && mbar_wait(o_full, 0, abort_flag, err, kErrWaitAcc);
-    __syncwarp();
-    if (got_o) {
+      if (!got_o) break;
       tc_fence_after();
       const uint32_t to = tmem + ((uint32_t)(q * 32) << 16) + 256;
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = ch * (D / 2); c0 < (ch + 1) * (D / 2); c0 += 32) {
         uint32_t rr[32];
         tmem_ld_32x32(to + c0, rr);
         tmem_ld_wait();
@@ -759,6 +827,9 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
                 pack_bf16x2(__uint_as_float(rr[8 * v + 6]), __uint_as_float(rr[8 * v + 7])));
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
     }
   }
   tc_fence_before();
@@ -851,18 +922,18 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
           !make_map(&mU, w.U, 3, dims, str, box))
         return cudaErrorInvalidValue;
     }
-    // fb: contiguous ranges of (head, slice, token tile) items per CTA.
-    const int64_t ntiles = (p.n + BM - 1) / BM;
-    const int64_t items = (int64_t)p.H * (p.hid / HS) * ntiles;
+    // fb: (head, slice) groups x token-range replicas, see fb_item_range.
     const int sms = num_sms();
-    const int grid_fb = (int)(items < sms ? items : sms);
+    const int groups = p.H * (p.hid / HS);
+    const int reps = groups <= sms ? sms / groups : 0;
+    const int grid_fb = reps > 0 ? groups * reps : sms;
     cudaError_t e = cudaFuncSetAttribute(fb_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          FB<D>::SMEM);
     if (e != cudaSuccess) return e;
     {
       TraceScope ts("tc_fwd_bwd", st);
       fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
-          mK, mV, mW1, mW3, mW2t, eta, p.n, p.H, p.hid, items, w.U, w.DH1, w.DH3, err);
+          mK, mV, mW1, mW3, mW2t, eta, p.n, p.H, p.hid, reps, w.U, w.DH1, w.DH3, err);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -915,7 +986,9 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
   cudaError_t e = cudaFuncSetAttribute(apply_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, AP<D>::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((p.n + BM - 1) / BM), p.H);
+  const int64_t items = (p.n + BM - 1) / BM * p.H;
+  const int sms = num_sms();
+  const unsigned grid = (unsigned)(items < sms ? items : sms);
   {
     TraceScope ts("tc_apply", st);
     apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
