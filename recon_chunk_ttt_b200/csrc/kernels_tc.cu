@@ -116,14 +116,16 @@ __global__ void convert_weights_kernel(int H, int d, int hid, const float* __res
 template <int D>
 struct FB {
   static constexpr int NCH = D / CH;
-  static constexpr int NSTAGE = 6;
+  static constexpr int NSTAGE = 4;
   static constexpr int STAGE = BM * CH * 2;              // 16 KB token chunk
   static constexpr int W13_CH = 2 * HS * CH * 2;          // 16 KB: W1s rows then W3s rows
   static constexpr int W2_CH = HS * CH * 2;               // 8 KB
+  static constexpr int OUT_TILE = BM * HS * 2;            // 16 KB: one output [128 x 64] bf16
   static constexpr int OFF_W13 = 0;
   static constexpr int OFF_W2 = OFF_W13 + NCH * W13_CH;
   static constexpr int OFF_STAGE = OFF_W2 + NCH * W2_CH;
-  static constexpr int OFF_BAR = OFF_STAGE + NSTAGE * STAGE;
+  static constexpr int OFF_OUT = OFF_STAGE + NSTAGE * STAGE;  // η·u, η·dh1, η·dh3 staging
+  static constexpr int OFF_BAR = OFF_OUT + 3 * OUT_TILE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;       // + alignment slack
   static constexpr int EPI_WARPS = 8;                     // 2 per TMEM lane quadrant
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;     // producer, MMA, epilogue
@@ -153,9 +155,9 @@ template <int D>
 __global__ void __launch_bounds__(FB<D>::THREADS, 1)
     fb_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
               const __grid_constant__ CUtensorMap mW1, const __grid_constant__ CUtensorMap mW3,
-              const __grid_constant__ CUtensorMap mW2t, const float* __restrict__ eta, int64_t n,
-              int H, int hid, int reps, __nv_bfloat16* __restrict__ U,
-              __nv_bfloat16* __restrict__ DH1, __nv_bfloat16* __restrict__ DH3, int* err) {
+              const __grid_constant__ CUtensorMap mW2t, const __grid_constant__ CUtensorMap mUs,
+              const __grid_constant__ CUtensorMap mD1s, const __grid_constant__ CUtensorMap mD3s,
+              const float* __restrict__ eta, int64_t n, int H, int hid, int reps, int* err) {
   using L = FB<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -302,67 +304,88 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // Two warps per TMEM lane quadrant; warp half `ch` takes hidden columns
-    // [32*ch, 32*ch+32) of the slice.
+    // [32*ch, 32*ch+32) of the slice.  Outputs are staged in shared memory in
+    // the 128-byte-swizzled box layout and written by TMA bulk stores.
     const int q = warp & 3;
     const int ch = (warp - 2) / 4;
+    const int row = q * 32 + lane;
+    const bool leader = warp == 2 && lane == 0;
+    uint8_t* stage_out = smem + L::OFF_OUT;
+    uint8_t* my_row = stage_out + (row / 8) * 1024 + (row % 8) * 128;
     uint32_t abits = 0;
     int buf = 0;
     for (int64_t it = it0; it < it1; ++it) {
       const int hs = (int)(it / ntiles);
       const int64_t tile = it % ntiles;
       const int head = hs / nslices, slice = hs % nslices;
+      const int64_t tok = tile * BM + row;
+      const bool live = tok < n;
+      const float ne = live ? -__ldg(&eta[tok * H + head]) : 0.f;  // -η: du = -(W2^T v)
       const bool got =
           mbar_wait(&acc_full[buf], (abits >> buf) & 1, abort_flag, err, kErrWaitAcc);
       __syncwarp();
-      if (!got) break;
+      // The previous tile's stores must have finished reading the staging box;
+      // the barrier also makes every epilogue warp leave together on a failure.
+      if (leader) bulk_wait_group_read0();
+      if (named_bar_any(1, 32 * L::EPI_WARPS, !got)) break;
       abits ^= 1u << buf;
       tc_fence_after();
-      const int64_t tok = tile * BM + q * 32 + lane;
-      const bool live = tok < n;
-      const float ne = live ? -eta[tok * H + head] : 0.f;  // -η: du = -(W2^T v)
       const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256 + ch * 32;
-      uint32_t r1[32], r3[32], rd[32];
-      tmem_ld_32x32(tl, r1);
-      tmem_ld_32x32(tl + HS, r3);
-      tmem_ld_32x32(tl + 128, rd);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      uint32_t pu[16], p1[16], p3[16];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float o_u[2], o_1[2], o_3[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float h1 = __uint_as_float(r1[i + e]);
-          const float h3 = __uint_as_float(r3[i + e]);
-          const float edu = ne * __uint_as_float(rd[i + e]);  // η du
-          const float s = sigmoid_fast(h1);
-          const float a = h1 * s;                             // SiLU(h1)
-          const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
-          o_u[e] = -ne * (a * h3);
-          o_3[e] = edu * a;
-          o_1[e] = edu * h3 * dsl;
+      for (int sub = 0; sub < 2; ++sub) {  // 16 hidden columns at a time
+        uint32_t r1[16], r3[16], rd[16];
+        tmem_ld_16x(tl + sub * 16, r1);
+        tmem_ld_16x(tl + HS + sub * 16, r3);
+        tmem_ld_16x(tl + 128 + sub * 16, rd);
+        tmem_ld_wait();
+        if (sub == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
-        pu[i / 2] = pack_bf16x2(o_u[0], o_u[1]);
-        p1[i / 2] = pack_bf16x2(o_1[0], o_1[1]);
-        p3[i / 2] = pack_bf16x2(o_3[0], o_3[1]);
+        uint32_t pu[8], p1[8], p3[8];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          float o_u[2], o_1[2], o_3[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float h1 = __uint_as_float(r1[i + e]);
+            const float h3 = __uint_as_float(r3[i + e]);
+            const float edu = ne * __uint_as_float(rd[i + e]);  // η du
+            const float s = sigmoid_fast(h1);
+            const float a = h1 * s;                             // SiLU(h1)
+            const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
+            o_u[e] = -ne * (a * h3);
+            o_3[e] = edu * a;
+            o_1[e] = edu * h3 * dsl;
+          }
+          pu[i / 2] = pack_bf16x2(o_u[0], o_u[1]);
+          p1[i / 2] = pack_bf16x2(o_1[0], o_1[1]);
+          p3[i / 2] = pack_bf16x2(o_3[0], o_3[1]);
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int off = ((ch * 4 + sub * 2 + c) ^ (row % 8)) * 16;
+          *reinterpret_cast<uint4*>(my_row + off) =
+              make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
+          *reinterpret_cast<uint4*>(my_row + L::OUT_TILE + off) =
+              make_uint4(p1[4 * c], p1[4 * c + 1], p1[4 * c + 2], p1[4 * c + 3]);
+          *reinterpret_cast<uint4*>(my_row + 2 * L::OUT_TILE + off) =
+              make_uint4(p3[4 * c], p3[4 * c + 1], p3[4 * c + 2], p3[4 * c + 3]);
+        }
       }
-      if (live) {
-        const size_t orow = ((size_t)head * n + tok) * hid + slice * HS + ch * 32;
-        uint4* du_ = reinterpret_cast<uint4*>(U + orow);
-        uint4* d1_ = reinterpret_cast<uint4*>(DH1 + orow);
-        uint4* d3_ = reinterpret_cast<uint4*>(DH3 + orow);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          du_[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
-          d1_[v] = make_uint4(p1[4 * v], p1[4 * v + 1], p1[4 * v + 2], p1[4 * v + 3]);
-          d3_[v] = make_uint4(p3[4 * v], p3[4 * v + 1], p3[4 * v + 2], p3[4 * v + 3]);
-        }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 32 * L::EPI_WARPS);
+      if (leader) {
+        const int x = slice * HS, y = (int)(tile * BM);
+        tma_store_3d(&mUs, stage_out, x, y, head);
+        tma_store_3d(&mD1s, stage_out + L::OUT_TILE, x, y, head);
+        tma_store_3d(&mD3s, stage_out + 2 * L::OUT_TILE, x, y, head);
+        bulk_commit_group();
       }
       buf ^= 1;
     }
+    if (leader) bulk_wait_group0();
   }
   tc_fence_before();
   __syncthreads();
@@ -541,7 +564,7 @@ __global__ void __launch_bounds__(GR<D>::THREADS, 1)
 template <int D>
 struct AP {
   static constexpr int NCH = D / CH;
-  static constexpr int NSTAGE = 3;
+  static constexpr int NSTAGE = 4;
   static constexpr int STAGE = 32768;                    // 2 W13 chunks, or one W2 slice
   static constexpr int W13_CH = 2 * HS * CH * 2;         // 16 KB
   static constexpr int CH_PER_STAGE = NCH >= 2 ? 2 : 1;
@@ -898,7 +921,7 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
       TraceScope ts("tc_convert_weights", st);
       convert_weights_kernel<<<cb, 256, 0, st>>>(p.H, p.d, p.hid, W1, W2, W3, w.b1, w.b3, w.b2t);
     }
-    CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg;
+    CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg, mUs, mD1s, mD3s;
     const uint64_t ld = (uint64_t)p.H * D;
     {
       const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
@@ -917,9 +940,10 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     {
       const uint64_t dims[3] = {(uint64_t)p.hid, (uint64_t)p.n, (uint64_t)p.H};
       const uint64_t str[2] = {(uint64_t)p.hid * 2, (uint64_t)p.n * p.hid * 2};
-      const uint32_t box[3] = {CH, TK, 1};
+      const uint32_t box[3] = {CH, TK, 1}, boxs[3] = {CH, BM, 1};
       if (!make_map(&mDH1, w.DH1, 3, dims, str, box) || !make_map(&mDH3, w.DH3, 3, dims, str, box) ||
-          !make_map(&mU, w.U, 3, dims, str, box))
+          !make_map(&mU, w.U, 3, dims, str, box) || !make_map(&mUs, w.U, 3, dims, str, boxs) ||
+          !make_map(&mD1s, w.DH1, 3, dims, str, boxs) || !make_map(&mD3s, w.DH3, 3, dims, str, boxs))
         return cudaErrorInvalidValue;
     }
     // fb: (head, slice) groups x token-range replicas, see fb_item_range.
@@ -933,7 +957,7 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     {
       TraceScope ts("tc_fwd_bwd", st);
       fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
-          mK, mV, mW1, mW3, mW2t, eta, p.n, p.H, p.hid, reps, w.U, w.DH1, w.DH3, err);
+          mK, mV, mW1, mW3, mW2t, mUs, mD1s, mD3s, eta, p.n, p.H, p.hid, reps, err);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
