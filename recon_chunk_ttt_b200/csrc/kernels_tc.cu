@@ -116,7 +116,7 @@ __global__ void convert_weights_kernel(int H, int d, int hid, const float* __res
 template <int D>
 struct FB {
   static constexpr int NCH = D / CH;
-  static constexpr int NSTAGE = 4;
+  static constexpr int NSTAGE = 6;
   static constexpr int STAGE = BM * CH * 2;              // 16 KB token chunk
   static constexpr int W13_CH = 2 * HS * CH * 2;          // 16 KB: W1s rows then W3s rows
   static constexpr int W2_CH = HS * CH * 2;               // 8 KB
@@ -124,8 +124,8 @@ struct FB {
   static constexpr int OFF_W13 = 0;
   static constexpr int OFF_W2 = OFF_W13 + NCH * W13_CH;
   static constexpr int OFF_STAGE = OFF_W2 + NCH * W2_CH;
-  static constexpr int OFF_OUT = OFF_STAGE + NSTAGE * STAGE;  // η·u, η·dh1, η·dh3 staging
-  static constexpr int OFF_BAR = OFF_OUT + 3 * OUT_TILE;
+  static constexpr int OFF_OUT = OFF_STAGE + NSTAGE * STAGE;  // 2 rotating output boxes
+  static constexpr int OFF_BAR = OFF_OUT + 2 * OUT_TILE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;       // + alignment slack
   static constexpr int EPI_WARPS = 8;                     // 2 per TMEM lane quadrant
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;     // producer, MMA, epilogue
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
     const int row = q * 32 + lane;
     const bool leader = warp == 2 && lane == 0;
     uint8_t* stage_out = smem + L::OFF_OUT;
-    uint8_t* my_row = stage_out + (row / 8) * 1024 + (row % 8) * 128;
+    uint32_t out_k = 0;  // stores issued so far (selects the staging buffer)
     uint32_t abits = 0;
     int buf = 0;
     for (int64_t it = it0; it < it1; ++it) {
@@ -324,64 +324,59 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
       const bool got =
           mbar_wait(&acc_full[buf], (abits >> buf) & 1, abort_flag, err, kErrWaitAcc);
       __syncwarp();
-      // The previous tile's stores must have finished reading the staging box;
-      // the barrier also makes every epilogue warp leave together on a failure.
-      if (leader) bulk_wait_group_read0();
       if (named_bar_any(1, 32 * L::EPI_WARPS, !got)) break;
       abits ^= 1u << buf;
       tc_fence_after();
       const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256 + ch * 32;
+      uint32_t r1[32], r3[32], rd[32];
+      tmem_ld_32x32(tl, r1);
+      tmem_ld_32x32(tl + HS, r3);
+      tmem_ld_32x32(tl + 128, rd);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      uint32_t pk[3][16];  // η·u, η·dh1, η·dh3 as packed bf16 pairs
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {  // 16 hidden columns at a time
-        uint32_t r1[16], r3[16], rd[16];
-        tmem_ld_16x(tl + sub * 16, r1);
-        tmem_ld_16x(tl + HS + sub * 16, r3);
-        tmem_ld_16x(tl + 128 + sub * 16, rd);
-        tmem_ld_wait();
-        if (sub == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      for (int i = 0; i < 32; i += 2) {
+        float o_u[2], o_1[2], o_3[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float h1 = __uint_as_float(r1[i + e]);
+          const float h3 = __uint_as_float(r3[i + e]);
+          const float edu = ne * __uint_as_float(rd[i + e]);  // η du
+          const float s = sigmoid_fast(h1);
+          const float a = h1 * s;                             // SiLU(h1)
+          const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
+          o_u[e] = -ne * (a * h3);
+          o_3[e] = edu * a;
+          o_1[e] = edu * h3 * dsl;
         }
-        uint32_t pu[8], p1[8], p3[8];
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          float o_u[2], o_1[2], o_3[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float h1 = __uint_as_float(r1[i + e]);
-            const float h3 = __uint_as_float(r3[i + e]);
-            const float edu = ne * __uint_as_float(rd[i + e]);  // η du
-            const float s = sigmoid_fast(h1);
-            const float a = h1 * s;                             // SiLU(h1)
-            const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
-            o_u[e] = -ne * (a * h3);
-            o_3[e] = edu * a;
-            o_1[e] = edu * h3 * dsl;
-          }
-          pu[i / 2] = pack_bf16x2(o_u[0], o_u[1]);
-          p1[i / 2] = pack_bf16x2(o_1[0], o_1[1]);
-          p3[i / 2] = pack_bf16x2(o_3[0], o_3[1]);
-        }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int off = ((ch * 4 + sub * 2 + c) ^ (row % 8)) * 16;
-          *reinterpret_cast<uint4*>(my_row + off) =
-              make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
-          *reinterpret_cast<uint4*>(my_row + L::OUT_TILE + off) =
-              make_uint4(p1[4 * c], p1[4 * c + 1], p1[4 * c + 2], p1[4 * c + 3]);
-          *reinterpret_cast<uint4*>(my_row + 2 * L::OUT_TILE + off) =
-              make_uint4(p3[4 * c], p3[4 * c + 1], p3[4 * c + 2], p3[4 * c + 3]);
-        }
+        pk[0][i / 2] = pack_bf16x2(o_u[0], o_u[1]);
+        pk[1][i / 2] = pack_bf16x2(o_1[0], o_1[1]);
+        pk[2][i / 2] = pack_bf16x2(o_3[0], o_3[1]);
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 32 * L::EPI_WARPS);
-      if (leader) {
-        const int x = slice * HS, y = (int)(tile * BM);
-        tma_store_3d(&mUs, stage_out, x, y, head);
-        tma_store_3d(&mD1s, stage_out + L::OUT_TILE, x, y, head);
-        tma_store_3d(&mD3s, stage_out + 2 * L::OUT_TILE, x, y, head);
-        bulk_commit_group();
+      // Three [128 x 64] boxes go out through two rotating staging buffers;
+      // before refilling one, the store issued from it two stores ago must
+      // have finished reading it.
+      const int x = slice * HS, y = (int)(tile * BM);
+#pragma unroll
+      for (int o = 0; o < 3; ++o) {
+        uint8_t* box = stage_out + (out_k & 1) * L::OUT_TILE;
+        if (leader) bulk_wait_group_read1();
+        named_bar_sync(1, 32 * L::EPI_WARPS);
+        uint8_t* r = box + (row / 8) * 1024 + (row % 8) * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(r + (((ch * 4 + c) ^ (row % 8)) * 16)) =
+              make_uint4(pk[o][4 * c], pk[o][4 * c + 1], pk[o][4 * c + 2], pk[o][4 * c + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 32 * L::EPI_WARPS);
+        if (leader) {
+          tma_store_3d(o == 0 ? &mUs : o == 1 ? &mD1s : &mD3s, box, x, y, head);
+          bulk_commit_group();
+        }
+        ++out_k;
       }
       buf ^= 1;
     }
@@ -581,10 +576,10 @@ struct AP {
 // Persistent: CTA b takes (query tile, head) items b, b + grid, ...  Per item
 // and 64-wide hidden slice js: F(js) = Q [W1s; W3s]^T into TMEM buffer js&1,
 // the epilogue turns it into u = SiLU(h1) ⊙ h3 (bf16, shared memory), and
-// O += u W2s^T.  The MMA issuer runs F(js+1) before O(js) so the epilogue of
-// slice js overlaps an MMA; the q chunks are released one by one during the
+// O += u W2s^T.  The q chunks are released one by one during the
 // last slice so the next item's q streams in early; O is drained while the
-// next item's first F MMAs run.
+// next item's first F MMAs run.  The issue order is F(0), F(1), F(2), O(0),
+// F(3), O(1), ... so u(js) has two F MMAs' time to be produced.
 template <int D>
 __global__ void __launch_bounds__(AP<D>::THREADS, 1)
     apply_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW1,
@@ -694,9 +689,9 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       };
       for (int js = 0; js < nsl && ok; ++js) {
         load_w13(js);
-        if (js >= 1 && ok) load_w2(js - 1);
+        if (js >= 2 && ok) load_w2(js - 2);
       }
-      if (ok) load_w2(nsl - 1);
+      for (int j = nsl >= 2 ? nsl - 2 : 0; j < nsl && ok; ++j) load_w2(j);
     }
     drain_ring(full, L::NSTAGE, issued, err);
     for (int c = 0; c < L::NCH; ++c) drain_ring(&q_full[c], 1, qloads, err);
@@ -771,10 +766,15 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
         }
         if (!ok) break;
         umma_commit(&f_full[b]);
-        if (js >= 1 && !do_o(g - 1, js - 1, i)) { ok = false; break; }
+        // O lags F by two slices, so the epilogue of slice js has the time of
+        // two F MMAs to produce u before the tensor pipe needs it.
+        if (js >= 2 && !do_o(g - 2, js - 2, i)) { ok = false; break; }
       }
       if (!ok) break;
-      if (!do_o(i * nsl + nsl - 1, nsl - 1, i)) break;
+      bool tail_ok = true;
+      for (int j = nsl >= 2 ? nsl - 2 : 0; j < nsl && tail_ok; ++j)
+        tail_ok = do_o(i * nsl + j, j, i);
+      if (!tail_ok) break;
       umma_commit(o_full);
     }
     umma_commit(done);
