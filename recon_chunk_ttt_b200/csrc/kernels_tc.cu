@@ -865,336 +865,6 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
 }
 
 // ----------------------------------------------------------------------------
-// apply2 kernel: the apply on CTA pairs with 2-SM MMAs.  A pair takes 256
-// queries of one head (128 per CTA) and each CTA keeps only its half of every
-// weight slice: the W1s rows (rank 0) or the W3s rows (rank 1) of F, and half
-// of the d rows of W2s for O, so each SM streams half the weight bytes of the
-// one-CTA version for the same MMA work.  Schedule as in apply_kernel: F(js)
-// into TMEM buffer js&1, the epilogue writes u = SiLU(h1) ⊙ h3 (bf16) into its
-// own shared memory, O += u W2s^T two slices behind F.
-// ----------------------------------------------------------------------------
-template <int D>
-struct AP2 {
-  static constexpr int NCH = D / CH;
-  static constexpr int NSTAGE = 6;
-  static constexpr int STAGE = 16384;
-  static constexpr int W13_HALF = HS * CH * 2;             // 8 KB: 64 rows x 128 B per d-chunk
-  static constexpr int CH_PER_STAGE = NCH >= 2 ? 2 : 1;
-  static constexpr int W2_HALF = (D / 2) * 128;            // [D/2 d-rows x 64 hidden]
-  static constexpr int OFF_Q = 0;                          // NCH x [128 x 128 B]
-  static constexpr int OFF_STAGE = OFF_Q + NCH * BM * 128;
-  static constexpr int OFF_U = OFF_STAGE + NSTAGE * STAGE; // 2 x [128 x 128 B]
-  static constexpr int OFF_BAR = OFF_U + 2 * BM * 128;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr int EPI_WARPS = 8;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr uint32_t TMEM_COLS = 512;               // F[0] 0, F[1] 128, O at 256
-};
-
-template <int D>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP2<D>::THREADS, 1)
-    apply2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW1,
-                  const __grid_constant__ CUtensorMap mW3, const __grid_constant__ CUtensorMap mW2,
-                  int64_t m, int H, int hid, __nv_bfloat16* __restrict__ O, int* err) {
-  using L = AP2<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* empty = full + L::NSTAGE;
-  uint64_t* q_full = empty + L::NSTAGE;
-  uint64_t* q_empty = q_full + L::NCH;
-  uint64_t* f_full = q_empty + L::NCH;
-  uint64_t* f_empty = f_full + 2;
-  uint64_t* u_full = f_empty + 2;
-  uint64_t* u_empty = u_full + 2;
-  uint64_t* o_full = u_empty + 2;
-  uint64_t* o_empty = o_full + 1;
-  uint64_t* done = o_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_rank();
-  const bool leader_cta = rank == 0;
-  const int nsl = hid / HS;
-  const int w13_stages = L::NCH / L::CH_PER_STAGE;
-  const int64_t npt = (m + 2 * BM - 1) / (2 * BM);  // 256-query pair tiles
-  const int64_t items = npt * H;
-  const int64_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < L::NSTAGE; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    for (int c = 0; c < L::NCH; ++c) {
-      mbar_init(&q_full[c], 1);
-      mbar_init(&q_empty[c], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&f_full[b], 1);
-      mbar_init(&f_empty[b], 2 * L::EPI_WARPS);
-      mbar_init(&u_full[b], 2 * L::EPI_WARPS);
-      mbar_init(&u_empty[b], 1);
-    }
-    mbar_init(o_full, 1);
-    mbar_init(o_empty, 2 * L::EPI_WARPS);
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    // Both CTAs load their halves; completion bytes of both count on the
-    // leader's barriers, and only the leader posts the expected byte count.
-    tma_prefetch_desc(&mQ);
-    int stage = 0;
-    uint32_t phase = 0;
-    int64_t issued = 0, qloads = 0;
-    bool ok = true;
-    auto next = [&]() -> uint8_t* {
-      if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) return nullptr;
-      return smem + L::OFF_STAGE + stage * L::STAGE;
-    };
-    auto advance = [&]() {
-      ++issued;
-      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
-    };
-    for (int64_t it = pair, i = 0; it < items && ok; it += npairs, ++i) {
-      const int64_t pt = it / H;
-      const int head = (int)(it % H);
-      const int row0 = (int)(pt * 2 * BM + rank * BM);
-      for (int c = 0; c < L::NCH && ok; ++c) {
-        if (!mbar_wait(&q_empty[c], (uint32_t)(i & 1) ^ 1, abort_flag, err, kErrWaitEmpty)) {
-          ok = false;
-          break;
-        }
-        if (leader_cta) mbar_arrive_expect_tx(&q_full[c], 2 * BM * 128);
-        tma_load_2d_pair(smem + L::OFF_Q + c * BM * 128, &mQ, map_to_rank(&q_full[c], 0),
-                         head * D + c * CH, row0);
-      }
-      ++qloads;
-      auto load_w13 = [&](int js) {
-        for (int g = 0; g < w13_stages && ok; ++g) {
-          uint8_t* st = next();
-          if (!st) { ok = false; return; }
-          if (leader_cta) mbar_arrive_expect_tx(&full[stage], 2 * L::CH_PER_STAGE * L::W13_HALF);
-          const uint32_t lb = map_to_rank(&full[stage], 0);
-          for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
-            const int c = g * L::CH_PER_STAGE + cc;
-            tma_load_2d_pair(st + cc * L::W13_HALF, rank == 0 ? &mW1 : &mW3, lb, c * CH,
-                             head * hid + js * HS);
-          }
-          advance();
-        }
-      };
-      auto load_w2 = [&](int js) {
-        uint8_t* st = next();
-        if (!st) { ok = false; return; }
-        if (leader_cta) mbar_arrive_expect_tx(&full[stage], 2 * L::W2_HALF);
-        tma_load_2d_pair(st, &mW2, map_to_rank(&full[stage], 0), js * HS,
-                         head * D + (int)rank * (D / 2));
-        advance();
-      };
-      for (int js = 0; js < nsl && ok; ++js) {
-        load_w13(js);
-        if (js >= 2 && ok) load_w2(js - 2);
-      }
-      for (int j = nsl >= 2 ? nsl - 2 : 0; j < nsl && ok; ++j) load_w2(j);
-    }
-    if (leader_cta) {
-      drain_ring(full, L::NSTAGE, issued, err);
-      for (int c = 0; c < L::NCH; ++c) drain_ring(&q_full[c], 1, qloads, err);
-    } else {
-      // The peer's loads complete on the leader's barriers; the leader's MMA
-      // releases each stage in both CTAs once consumed, which implies the
-      // peer's bytes have landed.
-      volatile int never = 0;
-      for (int64_t k = issued - L::NSTAGE < 0 ? 0 : issued - L::NSTAGE; k < issued; ++k)
-        mbar_wait(&empty[k % L::NSTAGE], (uint32_t)((k / L::NSTAGE) & 1), &never, err,
-                  kErrWaitFinal);
-    }
-  } else if (warp == 1 && lane == 0 && leader_cta) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idF = idesc_bf16_f32(2 * BM, 2 * HS, false, false);
-    const uint32_t idO = idesc_bf16_f32(2 * BM, D, false, false);
-    const uint32_t sbase = smem_u32(smem);
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    auto take = [&]() -> bool {
-      if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) return false;
-      tc_fence_after();
-      return true;
-    };
-    auto release = [&]() {
-      umma_commit_pair(&empty[stage]);
-      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
-    };
-    auto do_o = [&](int64_t g, int j, int64_t item_i) -> bool {
-      const int b = (int)(g & 1);
-      const uint32_t par = (uint32_t)((g >> 1) & 1);
-      if (!mbar_wait(&u_full[b], par, abort_flag, err, kErrWaitOperand)) return false;
-      if (j == 0 &&
-          !mbar_wait(o_empty, (uint32_t)(item_i & 1) ^ 1, abort_flag, err, kErrWaitAccFree))
-        return false;
-      tc_fence_after();
-      if (!take()) return false;
-      const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
-      const uint32_t ub = sbase + L::OFF_U + b * BM * 128;
-#pragma unroll
-      for (int kk = 0; kk < HS / 16; ++kk)
-        umma_bf16_pair(tmem + 256, sdesc_sw128(ub + kk * KSTEP_BYTES, 16, 1024),
-                       sdesc_sw128(st + kk * KSTEP_BYTES, 16, 1024), idO, (j | kk) != 0);
-      release();
-      umma_commit_pair(&u_empty[b]);
-      return true;
-    };
-    for (int64_t it = pair, i = 0; it < items && ok; it += npairs, ++i) {
-      for (int js = 0; js < nsl && ok; ++js) {
-        const int64_t g = i * nsl + js;
-        const int b = (int)(g & 1);
-        if (!mbar_wait(&f_empty[b], (uint32_t)((g >> 1) & 1) ^ 1, abort_flag, err,
-                       kErrWaitAccFree)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int gs = 0; gs < w13_stages && ok; ++gs) {
-          if (!take()) { ok = false; break; }
-          const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
-          for (int cc = 0; cc < L::CH_PER_STAGE && ok; ++cc) {
-            const int c = gs * L::CH_PER_STAGE + cc;
-            if (js == 0) {
-              if (!mbar_wait(&q_full[c], (uint32_t)(i & 1), abort_flag, err, kErrWaitFull)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            const uint32_t qa = sbase + L::OFF_Q + c * BM * 128;
-#pragma unroll
-            for (int kk = 0; kk < CH / 16; ++kk)
-              umma_bf16_pair(tmem + b * 128, sdesc_sw128(qa + kk * KSTEP_BYTES, 16, 1024),
-                             sdesc_sw128(st + cc * L::W13_HALF + kk * KSTEP_BYTES, 16, 1024),
-                             idF, (c | kk) != 0);
-            if (js == nsl - 1) umma_commit_pair(&q_empty[c]);
-          }
-          release();
-        }
-        if (!ok) break;
-        umma_commit_pair(&f_full[b]);
-        if (js >= 2 && !do_o(g - 2, js - 2, i)) { ok = false; break; }
-      }
-      if (!ok) break;
-      bool tail_ok = true;
-      for (int j = nsl >= 2 ? nsl - 2 : 0; j < nsl && tail_ok; ++j)
-        tail_ok = do_o(i * nsl + j, j, i);
-      if (!tail_ok) break;
-      umma_commit_pair(o_full);
-    }
-    umma_commit_pair(done);
-    volatile int never = 0;
-    mbar_wait(done, 0, &never, err, kErrWaitFinal);
-  } else if (warp >= 2) {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const int ch = (warp - 2) / 4;  // hidden columns [32ch, 32ch+32) of a slice
-    const int row = q * 32 + lane;
-    const uint32_t l_f_empty[2] = {map_to_rank(&f_empty[0], 0), map_to_rank(&f_empty[1], 0)};
-    const uint32_t l_u_full[2] = {map_to_rank(&u_full[0], 0), map_to_rank(&u_full[1], 0)};
-    const uint32_t l_o_empty = map_to_rank(o_empty, 0);
-    bool ok = true;
-    for (int64_t it = pair, i = 0; it < items && ok; it += npairs, ++i) {
-      const int64_t pt = it / H;
-      const int head = (int)(it % H);
-      const int64_t qi = pt * 2 * BM + rank * BM + row;
-      for (int js = 0; js < nsl && ok; ++js) {
-        const int64_t g = i * nsl + js;
-        const int b = (int)(g & 1);
-        const uint32_t par = (uint32_t)((g >> 1) & 1);
-        const bool got = mbar_wait(&f_full[b], par, abort_flag, err, kErrWaitAcc);
-        __syncwarp();
-        if (!got) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + b * 128 + ch * 32;
-        uint32_t r1[32], r3[32];
-        tmem_ld_32x32(tl, r1);
-        tmem_ld_32x32(tl + HS, r3);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(b ? l_f_empty[1] : l_f_empty[0]);
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float h1a = __uint_as_float(r1[k]), h1b = __uint_as_float(r1[k + 1]);
-          const float ua = h1a * sigmoid_fast(h1a) * __uint_as_float(r3[k]);
-          const float ub = h1b * sigmoid_fast(h1b) * __uint_as_float(r3[k + 1]);
-          pk[k / 2] = pack_bf16x2(ua, ub);
-        }
-        if (!mbar_wait(&u_empty[b], par ^ 1, abort_flag, err, kErrWaitOperand)) {
-          ok = false;
-          break;
-        }
-        uint8_t* urow = smem + L::OFF_U + b * BM * 128 + (row / 8) * 1024 + (row % 8) * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(urow + (((ch * 4 + c) ^ (row % 8)) * 16)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(b ? l_u_full[1] : l_u_full[0]);
-      }
-      if (!ok) break;
-      const bool got_o = mbar_wait(o_full, (uint32_t)(i & 1), abort_flag, err, kErrWaitAcc);
-      __syncwarp();
-      if (!got_o) break;
-      tc_fence_after();
-      const uint32_t to = tmem + ((uint32_t)(q * 32) << 16) + 256;
-      for (int c0 = ch * (D / 2); c0 < (ch + 1) * (D / 2); c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld_32x32(to + c0, rr);
-        tmem_ld_wait();
-        if (qi < m) {
-          uint4* dst = reinterpret_cast<uint4*>(O + qi * (int64_t)H * D + (int64_t)head * D + c0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(
-                pack_bf16x2(__uint_as_float(rr[8 * v]), __uint_as_float(rr[8 * v + 1])),
-                pack_bf16x2(__uint_as_float(rr[8 * v + 2]), __uint_as_float(rr[8 * v + 3])),
-                pack_bf16x2(__uint_as_float(rr[8 * v + 4]), __uint_as_float(rr[8 * v + 5])),
-                pack_bf16x2(__uint_as_float(rr[8 * v + 6]), __uint_as_float(rr[8 * v + 7])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(l_o_empty);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync_all();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc_pair(tmem, L::TMEM_COLS);
-  }
-}
-
-// ----------------------------------------------------------------------------
 // Host side
 // ----------------------------------------------------------------------------
 struct TcWs {
@@ -1226,29 +896,6 @@ TcWs carve(const Problem& p, void* ws, int S) {
 int grad_ctas_per_split(const Problem& p) {
   const int tiles = p.hid / BM;
   return p.H * tiles + p.H * ((tiles + 1) / 2);
-}
-
-// Clusters of two CTAs of `kernel` that can be resident at once (a cluster
-// must sit inside one GPC, so this can be below SMs / 2).
-template <typename Kern>
-int max_active_pairs(Kern kernel, int threads, int smem) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(threads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = 2;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, (void*)kernel, &cfg) != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    return 1;
-  }
-  return n;
 }
 
 int num_sms() {
@@ -1357,18 +1004,18 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
   }
   {
     const uint64_t dims[2] = {(uint64_t)p.hid, (uint64_t)p.H * D}, str[1] = {(uint64_t)p.hid * 2};
-    const uint32_t box[2] = {CH, (uint32_t)(D / 2)};  // each CTA of a pair loads half the d rows
+    const uint32_t box[2] = {CH, (uint32_t)D};
     if (!make_map(&mW2, s2, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(apply2_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, AP2<D>::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(apply_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, AP<D>::SMEM);
   if (e != cudaSuccess) return e;
-  const int64_t items = (p.n + 2 * BM - 1) / (2 * BM) * p.H;
-  const int pairs_max = max_active_pairs(apply2_kernel<D>, AP2<D>::THREADS, AP2<D>::SMEM);
-  const unsigned grid = 2u * (unsigned)(items < pairs_max ? items : pairs_max);
+  const int64_t items = (p.n + BM - 1) / BM * p.H;
+  const int sms = num_sms();
+  const unsigned grid = (unsigned)(items < sms ? items : sms);
   {
     TraceScope ts("tc_apply", st);
-    apply2_kernel<D><<<grid, AP2<D>::THREADS, AP2<D>::SMEM, st>>>(
+    apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
         mQ, mW1, mW3, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
   }
   return cudaGetLastError();
