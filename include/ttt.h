@@ -150,6 +150,30 @@ ttt_status ttt_stream_step(const ttt_config* cfg,
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
 
 /*
+ * Allocation-free streaming step (the pages have no counterpart: this is a
+ * deployment aid).  Same arguments and result as ttt_stream_step() minus the
+ * workspace: the scratch is a fixed TTT_STATIC_SCRATCH_BYTES device array
+ * inside the library, for callers that cannot allocate device memory when a
+ * frame arrives (fixed memory budgets, allocator owned by another runtime, no
+ * cudaMalloc after start-up).  The call allocates nothing.
+ *  - Returns TTT_ERR_WORKSPACE, before launching anything, when
+ *    ttt_update_workspace_bytes(cfg, n) exceeds TTT_STATIC_SCRATCH_BYTES
+ *    (with 4 heads of d = 256, hidden 512 that is about 2,100 tokens per call;
+ *    one 518 x 518 frame is 1,374).
+ *  - Every GPU that loads the library may hold the array until exit.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents (nothing in it has to start at zero); calls that can overlap on
+ *    the GPU race on it and must be serialised by the caller.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ */
+#define TTT_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+ttt_status ttt_stream_step_static(const ttt_config* cfg,
+                                  float* W1, float* W2, float* W3, void* shadow,
+                                  const void* K, const void* V, const float* eta, int64_t n,
+                                  const void* Q, int64_t m, void* O, ttt_stream_t stream);
+
+/*
  * Tracing.  With tracing on, every kernel launch of the library is bracketed
  * by two CUDA events on the caller's stream (host-side state: an event pool
  * and per-kernel totals, guarded by a mutex).  ttt_trace_read synchronises
