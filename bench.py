@@ -126,11 +126,45 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- distributed
-def dist_setup(args):
+def dist_setup(args=None):
+    """(world size, rank, local rank) from the torchrun environment."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """Max of a per-rank value over all ranks (identity for one rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world: int, tokens: int, layers: int, ms: float) -> float:
+    """Whole-job tokens/s per layer: every rank processes its own scene of
+    `tokens` tokens through `layers` layers in `ms` (the slowest rank's
+    time)."""
+    return world * tokens * layers / (ms / 1e3)
+
+
+def roofline_entry(name: str, flops: float, bytes_: float, ms: float, pk: dict) -> dict:
+    """Achieved rate of one kernel against the resource that bounds it: the
+    larger of flops / bf16 peak and bytes / HBM peak."""
+    t_tensor = flops / (pk["bf16_tflops_sustained"] * 1e12)
+    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tensor:
+        ach = bytes_ / (ms / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "peak_kind": "hbm_gbs"}
+    ach = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
+            "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"],
+            "peak_kind": "bf16_tflops_sustained"}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -214,13 +248,8 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
             import torch.distributed as dist
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v: float) -> float:
+        return max_over_ranks(v, world, dev)
 
     layers = args.layers or w.layers
     H, d, hid = w.heads, w.d, w.hidden
@@ -288,41 +317,46 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     R.ttt_trace_enable(False)
     trace = R.ttt_trace_read(reset=True)
     R.ttt_check_device_error()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms)
-    value = world * T * layers / (ms / 1e3)
+    ms = rank_max(e0.elapsed_time(e1) / args.steps)
+    value = aggregate_value(world, T, layers, ms)
 
     # -------------------------------------------------- roofline
     pk, pk_kind = peaks()
     unit = GEMM_UNIT(d, hid)
-    kflops = {  # algorithmic flops of all launches of each kernel in the timed region
-        "tc_fwd_bwd": 3 * unit * T * H * layers * args.steps,
-        "tc_grad": 3 * unit * T * H * layers * args.steps,
-        "tc_apply": 3 * unit * (T + M) * H * layers * args.steps,
+    reps = layers * args.steps
+    # algorithmic flops and bytes of all launches of each kernel in the timed region
+    work = {
+        "tc_fwd_bwd": (3 * unit * T * H * reps, (2 * d * 2 + 4 + 3 * hid * 2) * T * H * reps),
+        "tc_grad": (3 * unit * T * H * reps, (3 * hid * 2 + 2 * d * 2) * T * H * reps),
+        "tc_apply": (3 * unit * (T + M) * H * reps, 2 * d * 2 * (T + M) * H * reps),
     }
     per_kernel = {k: {"launches": v[0], "ms_total": v[1], "ms_avg": v[1] / max(v[0], 1)}
                   for k, v in trace.items()}
-    dom = max((k for k in kflops if k in trace), key=lambda k: trace[k][1])
+    for k, (fl, by) in work.items():
+        if k in trace:
+            per_kernel[k]["roofline"] = roofline_entry(k, fl, by, trace[k][1], pk)
+    dom = max((k for k in work if k in trace), key=lambda k: trace[k][1])
     launches = trace[dom][0]
-    achieved = kflops[dom] / (trace[dom][1] / 1e3) / 1e12
-    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    traffic = None
+    roof = dict(roofline_entry(dom, work[dom][0], work[dom][1], trace[dom][1], pk))
+    roof["peak_kind"] += f" ({pk_kind})"
+    roof["kernel"] = dom
+    per_launch = roof["achieved"] * (1e12 if roof["unit"] == "TFLOP/s" else 1e9) * (
+        trace[dom][1] / 1e3) / max(launches, 1)
+    roof["algorithmic_per_launch"] = per_launch
+    roof["traffic"] = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         with open(tp) as f:
             tj = json.load(f)
         ent = tj.get(dom)
         if ent and ent.get("source_sha") == kernel_source_sha():
-            traffic = ent["bytes_per_token_head"] * T * H * (1 if dom != "tc_apply" else
-                                                             (T + M) / (2 * T))
-    upd_ms = (trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1] +
-              trace.get("tc_convert_weights", (0, 0))[1] + trace.get("reduce_renorm", (0, 0))[1])
-    upd_flops = 6 * unit * T * H * layers * args.steps
+            units_per_launch = (T + M) * H / 2 if dom == "tc_apply" else T * H
+            roof["traffic"] = ent["bytes_per_unit"] * units_per_launch
     gemm_upd_ms = trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1]
-    roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s", "frac": achieved / peak,
-            "peak_kind": f"bf16_tflops_sustained ({pk_kind})", "traffic": traffic,
-            "flops_per_launch": kflops[dom] / max(launches, 1)}
+    upd_ms = gemm_upd_ms + trace.get("tc_convert_weights", (0, 0))[1] + \
+        trace.get("reduce_renorm", (0, 0))[1]
+    upd_flops = 6 * unit * T * H * reps
+    peak = pk["bf16_tflops_sustained"]
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -341,7 +375,7 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     if not args.no_e2e:
         line["e2e"] = e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta,
                           Win, Wout, shadow, ws_buf, O, Or, layers, T, M, world, barrier,
-                          max_over_ranks)
+                          rank_max)
     # -------------------------------------------------- CPU baseline
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -416,7 +450,7 @@ def e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta, W
     torch.cuda.synchronize(dev)
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
-    return {"value": world * T * layers / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+    return {"value": aggregate_value(world, T, layers, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": args.e2e_steps}
 

@@ -208,3 +208,23 @@ def ttt_trace_read(reset: bool = True) -> dict:
            "ttt_trace_read")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms))
             for i in range(min(cnt.value, cap))}
+
+
+def ttt_stream_step_static(cfg: ttt_config, W1, W2, W3, shadow, K, V, eta, Q, O=None,
+                           stream=None):
+    """ttt_stream_step without a workspace argument: the library's fixed
+    device scratch is used, so the call allocates nothing on the device (O is
+    allocated here only when not given)."""
+    L = lib()
+    if not hasattr(L.ttt_stream_step_static, "_typed"):
+        L.ttt_stream_step_static.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64,
+                                             _P, _P]
+        L.ttt_stream_step_static.restype = ctypes.c_int
+        L.ttt_stream_step_static._typed = True
+    n, m = int(K.shape[0]), int(Q.shape[0])
+    if O is None:
+        O = torch.empty((m, cfg.heads * cfg.d), dtype=_token_dtype(cfg), device=Q.device)
+    _check(L.ttt_stream_step_static(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W3),
+                                    _ptr(shadow), _ptr(K), _ptr(V), _ptr(eta), n, _ptr(Q), m,
+                                    _ptr(O), _stream(stream)), "ttt_stream_step_static")
+    return O
