@@ -48,14 +48,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor of rank 2 or 3 with dims[0] contiguous; box inner dim is 64
+// bf16 tensor of rank 2..5 with dims[0] contiguous; box inner dim is 64
 // elements (128 bytes) with the 128-byte swizzle.  Out-of-range rows read 0.
+// The outer dimensions may be listed in any stride order: a "chunk" dimension
+// of stride 128 bytes placed after the row dimension makes one box land as
+// consecutive [rows x 128 B] blocks, the layout the MMA descriptors expect.
 bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
               const uint64_t* byte_strides, const uint32_t* box) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t gd[3], gs[2];
-  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5] = {1, 1, 1, 1, 1};
   for (int i = 0; i < rank; ++i) {
     gd[i] = dims[i];
     bx[i] = box[i];
@@ -116,8 +119,10 @@ __global__ void convert_weights_kernel(int H, int d, int hid, const float* __res
 template <int D>
 struct FB {
   static constexpr int NCH = D / CH;
-  static constexpr int NSTAGE = 6;
-  static constexpr int STAGE = BM * CH * 2;              // 16 KB token chunk
+  static constexpr int CPS = NCH >= 2 ? 2 : 1;            // d-chunks per stage (one TMA box)
+  static constexpr int NSTAGE = 6 / CPS;
+  static constexpr int CHUNK = BM * CH * 2;               // 16 KB: 128 tokens x 64 d
+  static constexpr int STAGE = CPS * CHUNK;
   static constexpr int W13_CH = 2 * HS * CH * 2;          // 16 KB: W1s rows then W3s rows
   static constexpr int W2_CH = HS * CH * 2;               // 8 KB
   static constexpr int OUT_TILE = BM * HS * 2;            // 16 KB: one output [128 x 64] bf16
@@ -233,14 +238,15 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
       const int y = (int)(tile * BM);
       for (int pass = 0; pass < 2 && ok; ++pass) {
         const CUtensorMap* m = pass == 0 ? &mK : &mV;
-        for (int c = 0; c < L::NCH; ++c) {
+        for (int g = 0; g < L::NCH / L::CPS; ++g) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[stage], L::STAGE);
-          tma_load_2d(smem + L::OFF_STAGE + stage * L::STAGE, m, &full[stage], head * D + c * CH,
-                      y);
+          // one box = CPS chunks of [128 tokens x 64 d]
+          tma_load_3d(smem + L::OFF_STAGE + stage * L::STAGE, m, &full[stage], 0, y,
+                      head * L::NCH + g * L::CPS);
           ++issued;
           if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
         }
@@ -274,20 +280,23 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
       tc_fence_after();
       const uint32_t dF = tmem + buf * 256, dU = tmem + buf * 256 + 128;
       for (int pass = 0; pass < 2 && ok; ++pass) {
-        for (int c = 0; c < L::NCH; ++c) {
+        for (int g = 0; g < L::NCH / L::CPS; ++g) {
           if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a = sbase + L::OFF_STAGE + stage * L::STAGE;
-          const uint32_t b = pass == 0 ? sbase + L::OFF_W13 + c * L::W13_CH
-                                       : sbase + L::OFF_W2 + c * L::W2_CH;
+          for (int cc = 0; cc < L::CPS; ++cc) {
+            const int c = g * L::CPS + cc;
+            const uint32_t a = sbase + L::OFF_STAGE + stage * L::STAGE + cc * L::CHUNK;
+            const uint32_t b = pass == 0 ? sbase + L::OFF_W13 + c * L::W13_CH
+                                         : sbase + L::OFF_W2 + c * L::W2_CH;
 #pragma unroll
-          for (int kk = 0; kk < CH / 16; ++kk) {
-            const uint64_t da = sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024);
-            const uint64_t db = sdesc_sw128(b + kk * KSTEP_BYTES, 16, 1024);
-            umma_bf16(pass == 0 ? dF : dU, da, db, pass == 0 ? idF : idU, (c | kk) != 0);
+            for (int kk = 0; kk < CH / 16; ++kk) {
+              const uint64_t da = sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024);
+              const uint64_t db = sdesc_sw128(b + kk * KSTEP_BYTES, 16, 1024);
+              umma_bf16(pass == 0 ? dF : dU, da, db, pass == 0 ? idF : idU, (c | kk) != 0);
+            }
           }
           umma_commit(&empty[stage]);
           if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
@@ -475,12 +484,11 @@ __global__ void __launch_bounds__(GR<D>::THREADS, 1)
       for (int a = 0; a < nacc; ++a) {
         const CUtensorMap* m = kind == 0 ? (a == 0 ? &mDH1 : &mDH3) : &mU;
         const int j = kind == 0 ? j_first : j_first + a * BM;
-        tma_load_3d(st + a * L::A_TILE, m, &full[stage], j, y, head);
-        tma_load_3d(st + a * L::A_TILE + TK * 128, m, &full[stage], j + CH, y, head);
+        // one box: 2 hidden chunks x [64 tokens x 64 hidden]
+        tma_load_4d(st + a * L::A_TILE, m, &full[stage], 0, y, j / CH, head);
       }
-      const CUtensorMap* mb = kind == 0 ? &mK : &mV;
-      for (int c = 0; c < D / CH; ++c)
-        tma_load_2d(st + 2 * L::A_TILE + c * TK * 128, mb, &full[stage], head * D + c * CH, y);
+      // one box: D/64 d-chunks x [64 tokens x 64 d]
+      tma_load_3d(st + 2 * L::A_TILE, kind == 0 ? &mK : &mV, &full[stage], 0, y, head * (D / CH));
       ++issued;
       if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
     }
@@ -582,8 +590,8 @@ struct AP {
 // F(3), O(1), ... so u(js) has two F MMAs' time to be produced.
 template <int D>
 __global__ void __launch_bounds__(AP<D>::THREADS, 1)
-    apply_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW1,
-                 const __grid_constant__ CUtensorMap mW3, const __grid_constant__ CUtensorMap mW2,
+    apply_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW13,
+                 const __grid_constant__ CUtensorMap mW2,
                  int64_t m, int H, int hid, __nv_bfloat16* __restrict__ O, int* err) {
   using L = AP<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -671,12 +679,8 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
           uint8_t* st = next();
           if (!st) { ok = false; return; }
           mbar_arrive_expect_tx(&full[stage], L::CH_PER_STAGE * L::W13_CH);
-          for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
-            const int c = g * L::CH_PER_STAGE + cc;
-            tma_load_2d(st + cc * L::W13_CH, &mW1, &full[stage], c * CH, head * hid + js * HS);
-            tma_load_2d(st + cc * L::W13_CH + HS * 128, &mW3, &full[stage], c * CH,
-                        head * hid + js * HS);
-          }
+          // one box: CH_PER_STAGE d-chunks x {W1s, W3s} x 64 rows
+          tma_load_4d(st, &mW13, &full[stage], 0, head * hid + js * HS, 0, g * L::CH_PER_STAGE);
           advance();
         }
       };
@@ -924,10 +928,14 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg, mUs, mD1s, mD3s;
     const uint64_t ld = (uint64_t)p.H * D;
     {
-      const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
-      const uint32_t box[2] = {CH, BM}, boxg[2] = {CH, TK};
-      if (!make_map(&mK, K, 2, dims, str, box) || !make_map(&mV, V, 2, dims, str, box) ||
-          !make_map(&mKg, K, 2, dims, str, boxg) || !make_map(&mVg, V, 2, dims, str, boxg))
+      // {64 d, tokens, d-chunks of all heads}: fb boxes are FB::CPS chunks of 128
+      // tokens, grad boxes all D/64 chunks of one head for 64 tokens.
+      const uint64_t dims3[3] = {(uint64_t)CH, (uint64_t)p.n, ld / CH};
+      const uint64_t str3[2] = {ld * 2, CH * 2};
+      const uint32_t box3[3] = {CH, BM, (uint32_t)FB<D>::CPS};
+      const uint32_t boxg[3] = {CH, TK, (uint32_t)(D / CH)};
+      if (!make_map(&mK, K, 3, dims3, str3, box3) || !make_map(&mV, V, 3, dims3, str3, box3) ||
+          !make_map(&mKg, K, 3, dims3, str3, boxg) || !make_map(&mVg, V, 3, dims3, str3, boxg))
         return cudaErrorInvalidValue;
     }
     {
@@ -938,11 +946,18 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
         return cudaErrorInvalidValue;
     }
     {
+      // stores (fb): {hidden, tokens, heads}, box [128 tokens x 64 hidden]
       const uint64_t dims[3] = {(uint64_t)p.hid, (uint64_t)p.n, (uint64_t)p.H};
       const uint64_t str[2] = {(uint64_t)p.hid * 2, (uint64_t)p.n * p.hid * 2};
-      const uint32_t box[3] = {CH, TK, 1}, boxs[3] = {CH, BM, 1};
-      if (!make_map(&mDH1, w.DH1, 3, dims, str, box) || !make_map(&mDH3, w.DH3, 3, dims, str, box) ||
-          !make_map(&mU, w.U, 3, dims, str, box) || !make_map(&mUs, w.U, 3, dims, str, boxs) ||
+      const uint32_t boxs[3] = {CH, BM, 1};
+      // loads (grad): {64 hidden, tokens, hidden chunks, heads}, box = 2 chunks x 64 tokens
+      const uint64_t dims4[4] = {(uint64_t)CH, (uint64_t)p.n, (uint64_t)(p.hid / CH),
+                                 (uint64_t)p.H};
+      const uint64_t str4[3] = {(uint64_t)p.hid * 2, CH * 2, (uint64_t)p.n * p.hid * 2};
+      const uint32_t box4[4] = {CH, TK, 2, 1};
+      if (!make_map(&mDH1, w.DH1, 4, dims4, str4, box4) ||
+          !make_map(&mDH3, w.DH3, 4, dims4, str4, box4) ||
+          !make_map(&mU, w.U, 4, dims4, str4, box4) || !make_map(&mUs, w.U, 3, dims, str, boxs) ||
           !make_map(&mD1s, w.DH1, 3, dims, str, boxs) || !make_map(&mD3s, w.DH3, 3, dims, str, boxs))
         return cudaErrorInvalidValue;
     }
@@ -989,7 +1004,7 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
   const __nv_bfloat16_raw* s1 = shadow;
   const __nv_bfloat16_raw* s3 = shadow + wsz;
   const __nv_bfloat16_raw* s2 = shadow + 2 * wsz;
-  CUtensorMap mQ, mW1, mW3, mW2;
+  CUtensorMap mQ, mW13, mW2;
   const uint64_t ld = (uint64_t)p.H * D;
   {
     const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
@@ -997,10 +1012,12 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
     if (!make_map(&mQ, Q, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * p.hid}, str[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {CH, HS};
-    if (!make_map(&mW1, s1, 2, dims, str, box) || !make_map(&mW3, s3, 2, dims, str, box))
-      return cudaErrorInvalidValue;
+    // {64 d, hidden rows of all heads, matrix (W1 | W3), d-chunks}: one box holds,
+    // per d-chunk, the 64 rows of W1s followed by the 64 rows of W3s.
+    const uint64_t dims[4] = {(uint64_t)CH, (uint64_t)p.H * p.hid, 2, (uint64_t)(D / CH)};
+    const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)(s3 - s1) * 2, CH * 2};
+    const uint32_t box[4] = {CH, HS, 2, (uint32_t)AP<D>::CH_PER_STAGE};
+    if (!make_map(&mW13, s1, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t dims[2] = {(uint64_t)p.hid, (uint64_t)p.H * D}, str[1] = {(uint64_t)p.hid * 2};
@@ -1016,7 +1033,7 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
   {
     TraceScope ts("tc_apply", st);
     apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
-        mQ, mW1, mW3, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
+        mQ, mW13, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
   }
   return cudaGetLastError();
 }
