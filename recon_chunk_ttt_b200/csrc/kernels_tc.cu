@@ -120,15 +120,15 @@ template <int D>
 struct FB {
   static constexpr int NCH = D / CH;
   static constexpr int CPS = NCH >= 2 ? 2 : 1;            // d-chunks per stage (one TMA box)
-  static constexpr int NSTAGE = 8 / CPS;
+  static constexpr int NSTAGE = 6 / CPS;
   static constexpr int CHUNK = BM * CH * 2;               // 16 KB: 128 tokens x 64 d
   static constexpr int STAGE = CPS * CHUNK;
-  static constexpr int W13_CH = HS * CH * 2;              // 8 KB: this CTA's 64 rows (W1s or W3s)
-  static constexpr int W2_CH = (HS / 2) * CH * 2;         // 4 KB: this CTA's 32 rows of W2s^T
+  static constexpr int W13_CH = 2 * HS * CH * 2;          // 16 KB: W1s rows then W3s rows
+  static constexpr int W2_CH = HS * CH * 2;               // 8 KB
   static constexpr int OUT_TILE = BM * HS * 2;            // 16 KB: one output [128 x 64] bf16
   static constexpr int OFF_W13 = 0;
   static constexpr int OFF_W2 = OFF_W13 + NCH * W13_CH;
-  static constexpr int OFF_STAGE = (OFF_W2 + NCH * W2_CH + 1023) / 1024 * 1024;
+  static constexpr int OFF_STAGE = OFF_W2 + NCH * W2_CH;
   static constexpr int OFF_OUT = OFF_STAGE + NSTAGE * STAGE;  // 2 rotating output boxes
   static constexpr int OFF_BAR = OFF_OUT + 2 * OUT_TILE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;       // + alignment slack
@@ -137,37 +137,27 @@ struct FB {
   static constexpr uint32_t TMEM_COLS = 512;              // 2 x (F13 128 + DU 64), at 0 / 256
 };
 
-// Work items are (head*nslices + slice, 256-token pair tile).  With reps > 0
-// the grid is groups*reps CTA pairs: pair p owns group p / reps and the pair
-// tiles [r*ntiles/reps, (r+1)*ntiles/reps), r = p % reps, so the hidden slices
-// of one head walk the same k/v tiles in lockstep and share them through L2.
-// With reps == 0 (more groups than pairs) each pair takes a contiguous range
-// of the flattened item space.
-__device__ __forceinline__ void fb_item_range(int64_t ntiles, int groups, int reps, int64_t pair,
-                                              int64_t npairs, int64_t& it0, int64_t& it1) {
+// Work items are (head*nslices + slice, token tile) pairs.  With reps > 0 the
+// grid is groups*reps CTAs: CTA b owns group b / reps and the token tiles
+// [r*ntiles/reps, (r+1)*ntiles/reps), r = b % reps, so the hidden slices of one
+// head walk the same k/v tiles in lockstep and share them through L2.  With
+// reps == 0 (more groups than CTAs) each CTA takes a contiguous range of the
+// flattened item space.
+__device__ __forceinline__ void fb_item_range(int64_t ntiles, int groups, int reps,
+                                              int64_t& it0, int64_t& it1) {
   if (reps > 0) {
-    const int64_t g = pair / reps, r = pair % reps;
+    const int64_t g = blockIdx.x / reps, r = blockIdx.x % reps;
     it0 = g * ntiles + r * ntiles / reps;
     it1 = g * ntiles + (r + 1) * ntiles / reps;
   } else {
     const int64_t total = (int64_t)groups * ntiles;
-    it0 = total * pair / npairs;
-    it1 = total * (pair + 1) / npairs;
+    it0 = total * blockIdx.x / gridDim.x;
+    it1 = total * (blockIdx.x + 1) / gridDim.x;
   }
 }
 
-// Forward dual GEMM + backward GEMM + gated epilogue on CTA pairs (2-SM MMAs).
-// A pair takes 256 tokens (128 per CTA) of one (head, 64-wide hidden slice):
-//   F  = K [W1s; W3s]^T  (M = 256, N = 128; CTA 0 holds the W1s rows, CTA 1
-//                         the W3s rows of B)
-//   DU = V W2s           (M = 256, N = 64; each CTA holds 32 of the rows of
-//                         W2s^T)
-// into double-buffered TMEM; each CTA's 8 epilogue warps turn its own 128
-// rows into η·u, η·dh1, η·dh3 (bf16) and store them with TMA.  The leader CTA
-// (rank 0) issues every MMA; both CTAs load their own operands, whose bytes
-// count on the leader's barriers.
 template <int D>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
+__global__ void __launch_bounds__(FB<D>::THREADS, 1)
     fb_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
               const __grid_constant__ CUtensorMap mW1, const __grid_constant__ CUtensorMap mW3,
               const __grid_constant__ CUtensorMap mW2t, const __grid_constant__ CUtensorMap mUs,
@@ -187,12 +177,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_rank();
-  const bool leader_cta = rank == 0;
   const int nslices = hid / HS;
-  const int64_t ntiles = (n + 2 * BM - 1) / (2 * BM);
+  const int64_t ntiles = (n + BM - 1) / BM;
   int64_t it0, it1;
-  fb_item_range(ntiles, H * nslices, reps, blockIdx.x / 2, gridDim.x / 2, it0, it1);
+  fb_item_range(ntiles, H * nslices, reps, it0, it1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::NSTAGE; ++s) {
@@ -203,20 +191,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
     mbar_init(wempty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2 * L::EPI_WARPS);
+      mbar_init(&acc_empty[b], L::EPI_WARPS);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
-    tmem_relinquish_pair();
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  __syncwarp();
-  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -238,16 +224,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
           if (!mbar_wait(wempty, wphase, abort_flag, err, kErrWaitEmpty)) { ok = false; break; }
           wphase ^= 1;
         }
-        if (leader_cta) mbar_arrive_expect_tx(wfull, 2 * L::NCH * (L::W13_CH + L::W2_CH));
-        const uint32_t lb = map_to_rank(wfull, 0);
+        mbar_arrive_expect_tx(wfull, L::NCH * (L::W13_CH + L::W2_CH));
         const int row = head * hid + slice * HS;
-        // this CTA's half of B: W1s (rank 0) or W3s (rank 1), 32 rows of W2s^T
-        tma_load_3d_pair(smem + L::OFF_W13, rank == 0 ? &mW1 : &mW3, lb, 0, row, 0);
-        tma_load_3d_pair(smem + L::OFF_W2, &mW2t, lb, 0, row + (int)rank * (HS / 2), 0);
+        for (int c = 0; c < L::NCH; ++c) {
+          uint8_t* w13 = smem + L::OFF_W13 + c * L::W13_CH;
+          tma_load_2d(w13, &mW1, wfull, c * CH, row);
+          tma_load_2d(w13 + HS * 128, &mW3, wfull, c * CH, row);
+          tma_load_2d(smem + L::OFF_W2 + c * L::W2_CH, &mW2t, wfull, c * CH, row);
+        }
         ++wloads;
         cur_hs = hs;
       }
-      const int y = (int)(tile * 2 * BM + rank * BM);
+      const int y = (int)(tile * BM);
       for (int pass = 0; pass < 2 && ok; ++pass) {
         const CUtensorMap* m = pass == 0 ? &mK : &mV;
         for (int g = 0; g < L::NCH / L::CPS; ++g) {
@@ -255,28 +243,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
             ok = false;
             break;
           }
-          if (leader_cta) mbar_arrive_expect_tx(&full[stage], 2 * L::STAGE);
-          // one box = CPS chunks of [128 tokens x 64 d] of this CTA's tokens
-          tma_load_3d_pair(smem + L::OFF_STAGE + stage * L::STAGE, m, map_to_rank(&full[stage], 0),
-                           0, y, head * L::NCH + g * L::CPS);
+          mbar_arrive_expect_tx(&full[stage], L::STAGE);
+          // one box = CPS chunks of [128 tokens x 64 d]
+          tma_load_3d(smem + L::OFF_STAGE + stage * L::STAGE, m, &full[stage], 0, y,
+                      head * L::NCH + g * L::CPS);
           ++issued;
           if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
         }
       }
     }
-    if (leader_cta) {
-      drain_ring(full, L::NSTAGE, issued, err);
-      drain_ring(wfull, 1, wloads, err);
-    } else {
-      // The leader's final commit fires once every MMA, hence every read of
-      // this CTA's loaded data, has completed.
-      volatile int never = 0;
-      mbar_wait(done, 0, &never, err, kErrWaitFinal);
-    }
-  } else if (warp == 1 && lane == 0 && leader_cta) {
+    drain_ring(full, L::NSTAGE, issued, err);
+    drain_ring(wfull, 1, wloads, err);
+  } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idF = idesc_bf16_f32(2 * BM, 2 * HS, false, false);
-    const uint32_t idU = idesc_bf16_f32(2 * BM, HS, false, false);
+    const uint32_t idF = idesc_bf16_f32(BM, 2 * HS, false, false);
+    const uint32_t idU = idesc_bf16_f32(BM, HS, false, false);
     int stage = 0;
     uint32_t phase = 0, wphase = 0;
     uint32_t abits = 0;  // bit b: phase parity of accumulator buffer b
@@ -286,7 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
     for (int64_t it = it0; it < it1 && ok; ++it) {
       const int hs = (int)(it / ntiles);
       if (hs != cur_hs) {
-        if (cur_hs >= 0) umma_commit_pair(wempty);  // old weights free once prior MMAs finish
+        if (cur_hs >= 0) umma_commit(wempty);  // old weights free once prior MMAs finish
         if (!mbar_wait(wfull, wphase, abort_flag, err, kErrWaitFull)) { ok = false; break; }
         wphase ^= 1;
         cur_hs = hs;
@@ -314,20 +295,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
             for (int kk = 0; kk < CH / 16; ++kk) {
               const uint64_t da = sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024);
               const uint64_t db = sdesc_sw128(b + kk * KSTEP_BYTES, 16, 1024);
-              umma_bf16_pair(pass == 0 ? dF : dU, da, db, pass == 0 ? idF : idU, (c | kk) != 0);
+              umma_bf16(pass == 0 ? dF : dU, da, db, pass == 0 ? idF : idU, (c | kk) != 0);
             }
           }
-          umma_commit_pair(&empty[stage]);
+          umma_commit(&empty[stage]);
           if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
         }
       }
-      umma_commit_pair(&acc_full[buf]);
+      umma_commit(&acc_full[buf]);
       abits ^= 1u << buf;
       buf ^= 1;
     }
-    // Every MMA issued must complete before TMEM is released; `done` also
-    // tells the peer CTA that all of its loaded data has been consumed.
-    umma_commit_pair(done);
+    // Wait for every MMA issued by this thread before TMEM is released.
+    umma_commit(done);
     volatile int never = 0;
     mbar_wait(done, 0, &never, err, kErrWaitFinal);
   } else if (warp >= 2) {
@@ -339,8 +319,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
     const int ch = (warp - 2) / 4;
     const int row = q * 32 + lane;
     const bool leader = warp == 2 && lane == 0;
-    const uint32_t l_acc_empty0 = map_to_rank(&acc_empty[0], 0);
-    const uint32_t l_acc_empty1 = map_to_rank(&acc_empty[1], 0);
     uint8_t* stage_out = smem + L::OFF_OUT;
     uint32_t out_k = 0;  // stores issued so far (selects the staging buffer)
     uint32_t abits = 0;
@@ -349,13 +327,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
       const int hs = (int)(it / ntiles);
       const int64_t tile = it % ntiles;
       const int head = hs / nslices, slice = hs % nslices;
-      const int64_t tok = tile * 2 * BM + rank * BM + row;
+      const int64_t tok = tile * BM + row;
       const bool live = tok < n;
       const float ne = live ? -__ldg(&eta[tok * H + head]) : 0.f;  // -η: du = -(W2^T v)
       const bool got =
           mbar_wait(&acc_full[buf], (abits >> buf) & 1, abort_flag, err, kErrWaitAcc);
       __syncwarp();
-      // The barrier also makes every epilogue warp leave together on a failure.
       if (named_bar_any(1, 32 * L::EPI_WARPS, !got)) break;
       abits ^= 1u << buf;
       tc_fence_after();
@@ -367,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(buf ? l_acc_empty1 : l_acc_empty0);
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
       uint32_t pk[3][16];  // η·u, η·dh1, η·dh3 as packed bf16 pairs
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
@@ -391,7 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
       // Three [128 x 64] boxes go out through two rotating staging buffers;
       // before refilling one, the store issued from it two stores ago must
       // have finished reading it.
-      const int x = slice * HS, y = (int)(tile * 2 * BM + rank * BM);
+      const int x = slice * HS, y = (int)(tile * BM);
 #pragma unroll
       for (int o = 0; o < 3; ++o) {
         uint8_t* box = stage_out + (out_k & 1) * L::OUT_TILE;
@@ -405,8 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
         fence_proxy_async_smem();
         named_bar_sync(1, 32 * L::EPI_WARPS);
         if (leader) {
-          if (y < n)  // the second CTA's rows of the last pair tile may all lie past n
-            tma_store_3d(o == 0 ? &mUs : o == 1 ? &mD1s : &mD3s, box, x, y, head);
+          tma_store_3d(o == 0 ? &mUs : o == 1 ? &mD1s : &mD3s, box, x, y, head);
           bulk_commit_group();
         }
         ++out_k;
@@ -417,12 +393,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FB<D>::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  __syncwarp();
-  cluster_sync_all();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc_pair(tmem, L::TMEM_COLS);
+    tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
 
@@ -928,34 +902,6 @@ int grad_ctas_per_split(const Problem& p) {
   return p.H * tiles + p.H * ((tiles + 1) / 2);
 }
 
-// Clusters of two CTAs of `kernel` that can be resident at once (a cluster
-// must sit inside one GPC, so this can be below SMs / 2).
-template <typename Kern>
-int max_active_pairs(Kern kernel, int threads, int smem) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return 1;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(threads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = 2;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, (void*)kernel, &cfg) != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    return 1;
-  }
-  return n;
-}
-
 int num_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -993,14 +939,10 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
         return cudaErrorInvalidValue;
     }
     {
-      // {64 d, hidden rows of all heads, d-chunks}: one box = all d-chunks of
-      // 64 rows (W1s / W3s) or 32 rows (half of W2s^T).
-      const uint64_t dims[3] = {(uint64_t)CH, (uint64_t)p.H * p.hid, (uint64_t)(D / CH)};
-      const uint64_t str[2] = {(uint64_t)D * 2, CH * 2};
-      const uint32_t box13[3] = {CH, HS, (uint32_t)(D / CH)};
-      const uint32_t box2[3] = {CH, HS / 2, (uint32_t)(D / CH)};
-      if (!make_map(&mW1, w.b1, 3, dims, str, box13) || !make_map(&mW3, w.b3, 3, dims, str, box13) ||
-          !make_map(&mW2t, w.b2t, 3, dims, str, box2))
+      const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * p.hid}, str[1] = {(uint64_t)D * 2};
+      const uint32_t box[2] = {CH, HS};
+      if (!make_map(&mW1, w.b1, 2, dims, str, box) || !make_map(&mW3, w.b3, 2, dims, str, box) ||
+          !make_map(&mW2t, w.b2t, 2, dims, str, box))
         return cudaErrorInvalidValue;
     }
     {
@@ -1019,17 +961,17 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
           !make_map(&mD1s, w.DH1, 3, dims, str, boxs) || !make_map(&mD3s, w.DH3, 3, dims, str, boxs))
         return cudaErrorInvalidValue;
     }
-    // fb: CTA pairs; (head, slice) groups x token-range replicas (fb_item_range).
+    // fb: (head, slice) groups x token-range replicas, see fb_item_range.
+    const int sms = num_sms();
     const int groups = p.H * (p.hid / HS);
-    const int max_pairs = max_active_pairs(fb_kernel<D>, FB<D>::THREADS, FB<D>::SMEM);
-    const int reps = groups <= max_pairs ? max_pairs / groups : 0;
-    const int pairs = reps > 0 ? groups * reps : max_pairs;
+    const int reps = groups <= sms ? sms / groups : 0;
+    const int grid_fb = reps > 0 ? groups * reps : sms;
     cudaError_t e = cudaFuncSetAttribute(fb_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          FB<D>::SMEM);
     if (e != cudaSuccess) return e;
     {
       TraceScope ts("tc_fwd_bwd", st);
-      fb_kernel<D><<<2 * pairs, FB<D>::THREADS, FB<D>::SMEM, st>>>(
+      fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
           mK, mV, mW1, mW3, mW2t, mUs, mD1s, mD3s, eta, p.n, p.H, p.hid, reps, err);
     }
     e = cudaGetLastError();
