@@ -1,6 +1,6 @@
 // bf16 tensor-core path of the TTT update and apply on sm_100a: tcgen05 MMAs
 // with fp32 accumulators in tensor memory (TMEM), operands staged in shared
-// memory by TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast), warp
+// memory by TMA (cp.async.bulk.tensor, 128-byte swizzle, each CTA loads its own tiles), warp
 // specialised (one TMA producer thread, one MMA issuer thread, epilogue
 // warps), every wait bounded.
 //
