@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stream", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -376,6 +377,9 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
         line["e2e"] = e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta,
                           Win, Wout, shadow, ws_buf, O, Or, layers, T, M, world, barrier,
                           rank_max)
+    # -------------------------------------------------- streaming (stream256)
+    if not args.no_stream:
+        line["stream"] = stream_bench(R, torch, dev, rank_max)
     # -------------------------------------------------- CPU baseline
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -384,6 +388,57 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def stream_bench(R, torch, dev, rank_max, warm_frames: int = 8) -> dict:
+    """The streaming row: stream256 (256 frames of 1374 tokens, 4 heads x 256,
+    hidden 512) fed one frame per ttt_stream_step call (update in place, then
+    apply to the frame's queries).  Per-frame latency from CUDA events on the
+    stream around each call (it includes host launch time when the host is
+    slower than the GPU); tokens/s over all frames."""
+    w = wl.WORKLOADS["stream256"]
+    x = wl.make_inputs(w, bits=True)
+    to_bf = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa
+    K, V, Q = to_bf(x.K), to_bf(x.V), to_bf(x.Q)
+    eta = torch.from_numpy(x.eta).to(dev)
+    cfg = R.make_config(w.heads, w.d, w.hidden, renorm=R.RENORM_ROW)
+    W1, W2, W3 = (torch.from_numpy(a).to(dev) for a in (x.W1, x.W2, x.W3))
+    shadow = R.alloc_shadow(cfg, dev)
+    p = w.p
+    ws = R.alloc_workspace(cfg, p, dev)
+    O = torch.empty((p, w.heads * w.d), dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.current_stream(dev)
+
+    def frame(f):
+        s, e = f * p, (f + 1) * p
+        R.ttt_stream_step(cfg, W1, W2, W3, shadow, K[s:e], V[s:e], eta[s:e], Q[s:e], O,
+                          workspace=ws, stream=st)
+
+    for f in range(warm_frames):
+        frame(f)
+    W1.copy_(torch.from_numpy(x.W1))
+    W2.copy_(torch.from_numpy(x.W2))
+    W3.copy_(torch.from_numpy(x.W3))
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.frames + 1)]
+    ev[0].record(st)
+    h0 = time.perf_counter()
+    for f in range(w.frames):
+        frame(f)
+        ev[f + 1].record(st)
+    host_ms = (time.perf_counter() - h0) * 1e3 / w.frames
+    torch.cuda.synchronize(dev)
+    R.ttt_check_device_error()
+    lat = sorted(ev[f].elapsed_time(ev[f + 1]) for f in range(w.frames))
+    total_ms = rank_max(ev[0].elapsed_time(ev[-1]))
+    flops = (12 + 6) * w.d * w.hidden * w.heads * p * w.frames
+    return {"workload": f"stream256: {w.frames} frames x {p} tokens, {w.heads} heads x d={w.d}, "
+                        f"hidden {w.hidden}, one ttt_stream_step per frame",
+            "frame_ms_p50": lat[len(lat) // 2], "frame_ms_p99": lat[min(len(lat) - 1,
+                                                                      int(0.99 * len(lat)))],
+            "host_enqueue_ms_per_frame": host_ms,
+            "tokens_per_s": w.frames * p / (total_ms / 1e3),
+            "achieved_tflops": flops / (total_ms / 1e3) / 1e12}
 
 
 def e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta, Win, Wout,

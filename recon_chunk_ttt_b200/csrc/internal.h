@@ -7,6 +7,9 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <unordered_map>
+
 namespace ttt {
 
 // Problem description after validation.
@@ -72,6 +75,29 @@ class TraceScope {
   cudaStream_t st_;
   void* a_;
 };
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+// Kernels of one signature share a pointer type, so the record is keyed by
+// the kernel's address.
+template <typename Kern>
+cudaError_t ensure_smem_attr(Kern kernel, int smem) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;  // bit = device
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const void* key = reinterpret_cast<const void*>(kernel);
+  if (dev < 0 || dev >= 64)
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  std::lock_guard<std::mutex> lk(mu);
+  uint64_t& bits = done[key];
+  if (!(bits >> dev & 1)) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    bits |= 1ull << dev;
+  }
+  return cudaSuccess;
+}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -10,6 +10,8 @@
 // partials in increasing s, and a butterfly sum of squares, so the result is
 // the same bit pattern on every run.
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -71,16 +73,21 @@ __global__ void __launch_bounds__(256) reduce_renorm_kernel(
   // only rounding left on Ŵ - W is the final fp32 store.
   double wn[kMaxRowPerLane];
   double s_old = 0.0, s_new = 0.0;
+  // Sum the S partials element by element in increasing s; the loads of one
+  // partial are issued together so the row's reads overlap.
+#pragma unroll
+  for (int k = 0; k < kMaxRowPerLane; ++k) wn[k] = 0.0;
+  for (int s = 0; s < S; ++s) {
+    const float* P = partials + (((size_t)s * H + r.head) * 3 + pblk) * mat + (size_t)r.row * r.len;
+#pragma unroll
+    for (int k = 0; k < kMaxRowPerLane; ++k)
+      if (k < per_lane) wn[k] += (double)P[lane + 32 * k];
+  }
 #pragma unroll
   for (int k = 0; k < kMaxRowPerLane; ++k) {
     if (k < per_lane) {
-      const int idx = lane + 32 * k;
-      const double w = (double)W[base + idx];
-      double g = 0.0;
-      for (int s = 0; s < S; ++s)
-        g += (double)partials[(((size_t)s * H + r.head) * 3 + pblk) * mat +
-                              (size_t)r.row * r.len + idx];
-      const double wp = w + (double)sign * g;
+      const double w = (double)W[base + lane + 32 * k];
+      const double wp = w + (double)sign * wn[k];
       wn[k] = wp;
       s_old = fma(w, w, s_old);
       s_new = fma(wp, wp, s_new);
@@ -165,9 +172,18 @@ cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const 
 }
 
 int* device_error_ptr() {
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-  return static_cast<int*>(p);
+  // Looked up once per device.
+  static std::mutex mu;
+  static int* addr[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
 }
 
 cudaError_t read_and_clear_device_error(int* value) {

@@ -307,8 +307,8 @@ cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const 
                       const float* Q, float* O, cudaStream_t st) {
   if (p.n == 0) return cudaSuccess;
   const size_t smem = (size_t)kQ * p.hid * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(f32_apply_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // The limit is raised once, to what the largest supported hidden width needs.
+  cudaError_t e = ensure_smem_attr(f32_apply_kernel, (int)(kQ * 512 * sizeof(float)));
   if (e != cudaSuccess) return e;
   dim3 g((unsigned)((p.n + kQ - 1) / kQ), p.H);
   TraceScope ts("f32_apply", st);

@@ -102,15 +102,25 @@ __global__ void convert_weights_kernel(int H, int d, int hid, const float* __res
                                        const float* __restrict__ W2, const float* __restrict__ W3,
                                        __nv_bfloat16* __restrict__ b1, __nv_bfloat16* __restrict__ b3,
                                        __nv_bfloat16* __restrict__ b2t) {
-  const size_t total = (size_t)H * hid * d;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
-       i += (size_t)gridDim.x * blockDim.x) {
+  // One block per 32 x 32 tile (hidden rows j0.., d columns c0..) of one head;
+  // the W2 tile is transposed through shared memory so that both its read and
+  // its write are coalesced.
+  __shared__ float tile[32][33];
+  const int tiles_c = d / 32, tiles_j = hid / 32;
+  const int h = blockIdx.x / (tiles_c * tiles_j);
+  const int t = blockIdx.x % (tiles_c * tiles_j);
+  const int j0 = (t / tiles_c) * 32, c0 = (t % tiles_c) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const size_t mat = (size_t)h * hid * d;
+  for (int r = ty; r < 32; r += 8) {
+    const size_t i = mat + (size_t)(j0 + r) * d + c0 + tx;
     b1[i] = __float2bfloat16_rn(W1[i]);
     b3[i] = __float2bfloat16_rn(W3[i]);
-    const size_t h = i / ((size_t)hid * d), r = i % ((size_t)hid * d);
-    const size_t j = r / d, c = r % d;
-    b2t[i] = __float2bfloat16_rn(W2[h * (size_t)hid * d + c * hid + j]);
+    tile[r][tx] = W2[mat + (size_t)(c0 + r) * hid + j0 + tx];
   }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8)
+    b2t[mat + (size_t)(j0 + r) * d + c0 + tx] = __float2bfloat16_rn(tile[tx][r]);
 }
 
 // ----------------------------------------------------------------------------
@@ -903,10 +913,17 @@ int grad_ctas_per_split(const Problem& p) {
 }
 
 int num_sms() {
+  static std::mutex mu;
+  static int cached[64] = {};
   int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms > 0 ? sms : 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cached[dev] == 0) {
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+    cached[dev] = sms;
+  }
+  return cached[dev];
 }
 
 template <int D>
@@ -919,10 +936,9 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   if (err == nullptr) return cudaErrorInvalidDevice;
   const size_t wsz = (size_t)p.H * p.hid * p.d;
   if (p.n > 0) {
-    int cb = (int)((wsz + 255) / 256);
-    if (cb > 1184) cb = 1184;
     {
       TraceScope ts("tc_convert_weights", st);
+      const int cb = p.H * (p.hid / 32) * (p.d / 32);
       convert_weights_kernel<<<cb, 256, 0, st>>>(p.H, p.d, p.hid, W1, W2, W3, w.b1, w.b3, w.b2t);
     }
     CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg, mUs, mD1s, mD3s;
@@ -966,8 +982,7 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     const int groups = p.H * (p.hid / HS);
     const int reps = groups <= sms ? sms / groups : 0;
     const int grid_fb = reps > 0 ? groups * reps : sms;
-    cudaError_t e = cudaFuncSetAttribute(fb_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         FB<D>::SMEM);
+    cudaError_t e = ensure_smem_attr(fb_kernel<D>, FB<D>::SMEM);
     if (e != cudaSuccess) return e;
     {
       TraceScope ts("tc_fwd_bwd", st);
@@ -978,8 +993,7 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
     if (e != cudaSuccess) return e;
     const int tiles = p.hid / BM;
     const int k0 = p.H * tiles, k1 = p.H * ((tiles + 1) / 2);
-    e = cudaFuncSetAttribute(grad_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GR<D>::SMEM);
+    e = ensure_smem_attr(grad_kernel<D>, GR<D>::SMEM);
     if (e != cudaSuccess) return e;
     {
       TraceScope ts("tc_grad", st);
@@ -1024,8 +1038,7 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
     const uint32_t box[2] = {CH, (uint32_t)D};
     if (!make_map(&mW2, s2, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(apply_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, AP<D>::SMEM);
+  cudaError_t e = ensure_smem_attr(apply_kernel<D>, AP<D>::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t items = (p.n + BM - 1) / BM * p.H;
   const int sms = num_sms();
