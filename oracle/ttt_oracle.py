@@ -38,8 +38,15 @@ the design notes):
     of W2 of length hidden) to the pre-update row norm, no epsilon; a zero
     updated row is left as is.  "frobenius" (whole matrix per head, the
     literal reading of the unindexed norm) and "off" are kept as switches.
-  * Newton-Schulz orthonormalisation of the gradient is not applied (the
-    layer as specified for this build omits it).
+  * Newton-Schulz orthonormalisation of the gradient ([review] section 2,
+    the update after Eq. 3, "following the Muon optimizer") is a switch,
+    ns_steps, off (0) by default.  The pages give neither the polynomial nor
+    the step count; the reading taken is Muon's published quintic iteration
+    (Jordan et al. 2024, "Muon: An optimizer for hidden layers in neural
+    networks"): X0 = g / ||g||_F, then ns_steps times
+    X <- a X + b (X X^T) X + c (X X^T)^2 X with (a, b, c) =
+    (3.4445, -4.7750, 2.0315), worked on the wide orientation of g; each of
+    g1, g2, g3 is orthonormalised on its own, per head; g = 0 gives 0.
   * Heads are independent fast-weight MLPs.
 """
 from __future__ import annotations
@@ -173,9 +180,41 @@ def renorm(W, Wp, mode):
     raise ValueError(f"unknown renorm mode {mode}")
 
 
-def update_head(W1, W2, W3, K, V, eta, renorm_mode=RENORM_ROW):
-    """One TTT update of one head: Ŵ = renorm(W - g)."""
-    G1, G2, G3 = gradient(W1, W2, W3, K, V, eta)
+# --------------------------------------------------------------------------
+# Newton-Schulz orthonormalisation ([review] section 2, the update after
+# Eq. 3: Delta <- NewtonSchulz(g), following the Muon optimizer).  The
+# polynomial is Muon's quintic; see the module header for the reading.
+# --------------------------------------------------------------------------
+NS_COEFFS = (3.4445, -4.7750, 2.0315)
+
+
+def newton_schulz(G, steps, coeffs=NS_COEFFS):
+    """Approximate orthonormalisation of one matrix: with X0 = G/||G||_F,
+    repeat X <- a X + b A X + c A^2 X, A = X X^T, `steps` times.  A tall G is
+    worked as G^T (A is then the smaller Gram matrix; the result is the same
+    polynomial in the singular values either way) and transposed back."""
+    a, b, c = coeffs
+    X = _f64(G)
+    nrm = np.sqrt(np.sum(X * X))
+    if nrm == 0.0:
+        return np.zeros_like(X)
+    X = X / nrm
+    tall = X.shape[0] > X.shape[1]
+    if tall:
+        X = X.T
+    for _ in range(steps):
+        A = X @ X.T
+        X = a * X + (b * A + c * (A @ A)) @ X
+    return X.T if tall else X
+
+
+def update_head(W1, W2, W3, K, V, eta, renorm_mode=RENORM_ROW, ns_steps=0):
+    """One TTT update of one head: Ŵ = renorm(W - Delta) with Delta = g, or
+    Delta = NewtonSchulz(g) per matrix when ns_steps > 0."""
+    G = gradient(W1, W2, W3, K, V, eta)
+    if ns_steps > 0:
+        G = tuple(newton_schulz(g, ns_steps) for g in G)
+    G1, G2, G3 = G
     return (renorm(W1, _f64(W1) - G1, renorm_mode),
             renorm(W2, _f64(W2) - G2, renorm_mode),
             renorm(W3, _f64(W3) - G3, renorm_mode))
@@ -187,14 +226,14 @@ def _split_heads(X, heads):
     return X.reshape(n, heads, -1)
 
 
-def ttt_update(W1, W2, W3, K, V, eta, renorm_mode=RENORM_ROW):
+def ttt_update(W1, W2, W3, K, V, eta, renorm_mode=RENORM_ROW, ns_steps=0):
     """All heads.  W1, W3: [H, hidden, d]; W2: [H, d, hidden];
     K, V: [n, H*d]; eta: [n, H].  Returns (Ŵ1, Ŵ2, Ŵ3) in fp64."""
     H = np.shape(W1)[0]
     Kh, Vh = _split_heads(K, H), _split_heads(V, H)
     eta = _f64(eta).reshape(-1, H)
     out = [update_head(W1[h], W2[h], W3[h], Kh[:, h], Vh[:, h], eta[:, h],
-                       renorm_mode) for h in range(H)]
+                       renorm_mode, ns_steps) for h in range(H)]
     return tuple(np.stack([o[i] for o in out]) for i in range(3))
 
 
@@ -209,7 +248,8 @@ def ttt_apply(W1, W2, W3, Q):
     return O.reshape(m, -1)
 
 
-def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW):
+def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW,
+               ns_steps=0):
     """Streaming ([review] section 3, [notes] "流式更新"): for each frame t,
     W^(t) = TTTUpdate(W^(t-1); the frame's tokens), then the frame's queries
     read f_{W^(t)}.  Returns the final weights and the per-frame outputs
@@ -219,7 +259,7 @@ def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW):
     outs = []
     for s in range(0, n, frame_tokens):
         e = min(n, s + frame_tokens)
-        Ws = ttt_update(*Ws, K[s:e], V[s:e], eta[s:e], renorm_mode)
+        Ws = ttt_update(*Ws, K[s:e], V[s:e], eta[s:e], renorm_mode, ns_steps)
         outs.append(ttt_apply(*Ws, Q[s:e]))
     return Ws, np.concatenate(outs, axis=0)
 

@@ -366,3 +366,71 @@ def test_golden_tiny_regression():
         np.testing.assert_allclose(d.reshape(-1)[:8], g[name + "_head8"], rtol=1e-12, atol=1e-18)
     np.testing.assert_allclose(np.linalg.norm(out), g["O_fro"], rtol=1e-12)
     np.testing.assert_allclose(out.reshape(-1)[:8], g["O_head8"], rtol=1e-12, atol=1e-18)
+
+
+# ---------------------------------------------------- Newton-Schulz (switch)
+def _ns_scalar(x, steps):
+    """The scalar quintic that the matrix iteration applies to each singular
+    value of X0 = G/||G||_F (Muon's coefficients)."""
+    a, b, c = 3.4445, -4.7750, 2.0315
+    for _ in range(steps):
+        x = a * x + b * x ** 3 + c * x ** 5
+    return x
+
+
+@pytest.mark.parametrize("shape", [(6, 10), (10, 6), (7, 7)])
+@pytest.mark.parametrize("steps", [1, 2, 5])
+def test_newton_schulz_acts_on_singular_values(shape, steps):
+    """For G = U diag(s) V^T the iteration is U diag(p^k(s/||s||)) V^T: pins the
+    coefficient order, the Frobenius normalisation and the tall/wide handling
+    against an SVD built by hand (a rank-deficient part stays zero)."""
+    m, n = shape
+    r = min(m, n)
+    rng = np.random.default_rng(11 + steps)
+    U, _ = np.linalg.qr(rng.standard_normal((m, r)))
+    Vt, _ = np.linalg.qr(rng.standard_normal((n, r)))
+    s = np.linspace(3.0, 0.2, r)
+    s[-1] = 0.0  # one zero singular value
+    G = U @ np.diag(s) @ Vt.T
+    want = U @ np.diag(_ns_scalar(s / np.linalg.norm(s), steps)) @ Vt.T
+    np.testing.assert_allclose(O.newton_schulz(G, steps), want, rtol=0, atol=1e-12)
+
+
+def test_newton_schulz_worked_scalar_and_invariants():
+    # 1x1: X0 = sign(g), one step gives a + b + c = 0.701 with the sign kept
+    assert abs(O.newton_schulz(np.array([[-3.0]]), 1)[0, 0] + 0.701) < 1e-15
+    rng = np.random.default_rng(5)
+    G = rng.standard_normal((8, 12))
+    X = O.newton_schulz(G, 5)
+    np.testing.assert_allclose(O.newton_schulz(7.5 * G, 5), X, atol=1e-13)  # scale
+    np.testing.assert_allclose(O.newton_schulz(-G, 5), -X, atol=1e-13)      # odd
+    np.testing.assert_allclose(O.newton_schulz(G.T, 5), X.T, atol=1e-13)    # transpose
+    np.testing.assert_allclose(O.newton_schulz(G, 0), G / np.linalg.norm(G), atol=1e-15)
+    assert not np.any(O.newton_schulz(np.zeros((4, 6)), 5))
+    # five steps leave every singular value inside Muon's band around 1
+    sv = np.linalg.svd(X, compute_uv=False)
+    assert sv.min() > 0.6 and sv.max() < 1.25
+
+
+def test_update_with_newton_schulz():
+    """With NS the update shares the gradient's singular vectors (g^T Delta
+    and g Delta^T are symmetric positive semi-definite), it no longer depends
+    on the global scale of eta, and eta = 0 still leaves W bitwise."""
+    W1, W2, W3, K, V, eta = _tiny(seed=4, n=9, d=6, hidden=10)
+    G = O.gradient(W1, W2, W3, K, V, eta)
+    Wn = O.update_head(W1, W2, W3, K, V, eta, O.RENORM_OFF, ns_steps=5)
+    for g, W, Wh in zip(G, (W1, W2, W3), Wn):
+        D = W - Wh
+        for P in (g.T @ D, g @ D.T):
+            np.testing.assert_allclose(P, P.T, atol=1e-12)
+            assert np.linalg.eigvalsh(0.5 * (P + P.T)).min() > -1e-12
+    Wc = O.update_head(W1, W2, W3, K, V, 3.0 * eta, O.RENORM_OFF, ns_steps=5)
+    for a_, b_ in zip(Wn, Wc):
+        np.testing.assert_allclose(a_, b_, atol=1e-12)
+    Wz = O.update_head(W1, W2, W3, K, V, 0 * eta, O.RENORM_ROW, ns_steps=5)
+    for a_, b_ in zip(Wz, (W1, W2, W3)):
+        assert np.array_equal(a_, b_)
+    # renorm on: row norms kept
+    Wr = O.update_head(W1, W2, W3, K, V, eta, O.RENORM_ROW, ns_steps=3)
+    for a_, b_ in zip(Wr, (W1, W2, W3)):
+        np.testing.assert_allclose(np.linalg.norm(a_, axis=1), np.linalg.norm(b_, axis=1), rtol=1e-13)
