@@ -16,8 +16,17 @@
  * with the tokens of one frame at a time, the state carried across calls.
  * The renormalisation axis is row-wise (each row of W1, W3 of length d, each
  * row of W2 of length hidden, rescaled to its pre-update norm); "frobenius"
- * (one norm per matrix per head) and "off" are switches.  Newton–Schulz
- * orthonormalisation of g is not applied (ns_steps must be 0).
+ * (one norm per matrix per head) and "off" are switches.
+ *
+ * Newton–Schulz (same section, the update after Eq. 3: Δ ← NewtonSchulz(g),
+ * following the Muon optimizer; then Ŵ = ‖W‖ · (W − Δ)/‖W − Δ‖) is a switch,
+ * ns_steps (0 = off, the layer above).  The page gives neither the polynomial
+ * nor the step count; with ns_steps = k > 0 each of g1, g2, g3 of each head is
+ * replaced by k steps of Muon's quintic iteration on X0 = g/‖g‖_F:
+ *   X ← a X + (b A + c A²) X,  A = X Xᵀ,  (a, b, c) = (3.4445, −4.7750, 2.0315),
+ * worked on the wide (d × hidden) orientation; g = 0 gives Δ = 0.  In
+ * BF16_TC mode its GEMMs run on the tensor cores with each fp32 operand split
+ * into two bf16 parts (hi + lo, three products), the iterate kept in fp32.
  *
  * Conventions shared by every entry point
  *  - All pointers except `cfg` are DEVICE pointers on the current CUDA device,
@@ -69,6 +78,7 @@ typedef enum {
 enum { TTT_MLP_SWIGLU = 0 };
 enum { TTT_RENORM_OFF = 0, TTT_RENORM_ROW = 1, TTT_RENORM_FROB = 2 };
 enum { TTT_PREC_BF16_TC = 0, TTT_PREC_FP32_CHECK = 1 };
+enum { TTT_MAX_NS_STEPS = 32 };
 
 typedef struct {
   int32_t heads;     /* H, number of independent fast-weight MLPs          */
@@ -76,7 +86,7 @@ typedef struct {
   int32_t hidden;    /* fast-weight hidden width (128 or 512)              */
   int32_t mlp;       /* TTT_MLP_SWIGLU                                     */
   int32_t renorm;    /* TTT_RENORM_*                                       */
-  int32_t ns_steps;  /* Newton–Schulz iterations: must be 0                */
+  int32_t ns_steps;  /* Newton–Schulz steps on g: 0 (off) .. TTT_MAX_NS_STEPS */
   int32_t precision; /* TTT_PREC_BF16_TC: bf16 tensor-core operands, fp32
                         accumulation; TTT_PREC_FP32_CHECK: fp32 CUDA-core
                         arithmetic throughout                              */
@@ -94,7 +104,8 @@ size_t ttt_shadow_bytes(const ttt_config* cfg);
 
 /*
  * One TTT update of all heads (Eq. 1–3 and the renormalisation above):
- *   g = ∇_W Σ_{i<n} η_i (−f_W(k_i)^T v_i),  Ŵ = renorm(W − g).
+ *   g = ∇_W Σ_{i<n} η_i (−f_W(k_i)^T v_i),  Ŵ = renorm(W − Δ),
+ *   Δ = g (ns_steps = 0) or NewtonSchulz(g) (ns_steps > 0).
  * Inputs W1, W2, W3 (fp32), K, V, eta for n >= 0 tokens.  Writes Ŵ to
  * W1_out, W2_out, W3_out (fp32, may equal the inputs) and, when `shadow` is
  * not NULL, bf16 copies of Ŵ to `shadow` for ttt_apply.

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libttt.so")
 
 TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED_SHAPE, TTT_ERR_ALIGNMENT, \
     TTT_ERR_WORKSPACE, TTT_ERR_CUDA, TTT_ERR_DEVICE = range(7)
+MAX_NS_STEPS = 32  # TTT_MAX_NS_STEPS
 MLP_SWIGLU = 0
 RENORM_OFF, RENORM_ROW, RENORM_FROB = 0, 1, 2
 PREC_BF16_TC, PREC_FP32_CHECK = 0, 1

@@ -17,6 +17,7 @@ struct Problem {
   int H, d, hid;
   int64_t n;  // tokens (update) or queries (apply)
   int renorm;
+  int ns_steps;  // Newton-Schulz steps on the gradient (0: off)
 };
 
 // Split-K plan of the token reduction: S contiguous token ranges of `chunk`
@@ -44,6 +45,16 @@ cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const 
 cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const float* W1,
                           const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
                           __nv_bfloat16_raw* shadow, float* scratch, cudaStream_t st);
+// ---- optional Newton-Schulz orthonormalisation (kernels_ns.cu) ------------
+// Workspace it needs beyond the update's own (0 when ns_steps == 0).
+size_t ns_workspace_bytes(const Problem& p);
+// With ns_steps > 0 and n > 0: Delta = NewtonSchulz(sum of the S partials) per
+// head and matrix, then reduce_renorm of Delta as a single split; otherwise
+// reduce_renorm of the partials as they are.
+cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void* ns_ws,
+                           bool tensor_cores, const float* W1, const float* W2, const float* W3,
+                           float* W1o, float* W2o, float* W3o, __nv_bfloat16_raw* shadow,
+                           float* scratch, cudaStream_t st);
 cudaError_t pack_shadow(int H, int d, int hid, const float* W1, const float* W2,
                         const float* W3, __nv_bfloat16_raw* shadow, cudaStream_t st);
 

@@ -260,14 +260,18 @@ SplitPlan f32_split_plan(const Problem& p) {
   return {S, chunk};
 }
 
-size_t f32_workspace_bytes(const Problem& p) {
+// Bytes of the update's own workspace; the optional Newton-Schulz region
+// follows it at a 1024-byte boundary.
+static size_t f32_main_bytes(const Problem& p) {
   const SplitPlan sp = f32_split_plan(p);
   size_t b = 0;
   b += align_up(3 * (size_t)p.H * p.n * p.hid * sizeof(float), 256);
   b += align_up((size_t)sp.S * p.H * 3 * p.hid * p.d * sizeof(float), 256);
   b += align_up((size_t)p.H * (2 * p.hid + p.d) * 2 * sizeof(double), 256);
-  return b;
+  return align_up(b, 1024);
 }
+
+size_t f32_workspace_bytes(const Problem& p) { return f32_main_bytes(p) + ns_workspace_bytes(p); }
 
 cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const float* W3,
                        const float* K, const float* V, const float* eta, float* W1o, float* W2o,
@@ -300,7 +304,8 @@ cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return reduce_renorm(p, sp.S, partials, W1, W2, W3, W1o, W2o, W3o, shadow, scratch, st);
+  return ns_then_renorm(p, sp.S, partials, static_cast<char*>(ws) + f32_main_bytes(p), false, W1,
+                        W2, W3, W1o, W2o, W3o, shadow, scratch, st);
 }
 
 cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const float* W3,

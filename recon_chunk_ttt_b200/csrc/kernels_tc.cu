@@ -24,6 +24,11 @@
 #include "internal.h"
 
 namespace ttt {
+
+// Bytes of the update's own workspace (the optional Newton-Schulz region
+// follows it).
+size_t tc_main_bytes(const Problem& p);
+
 namespace {
 
 constexpr int BM = 128;          // MMA M: tokens (fb, apply) or hidden rows (grad)
@@ -1005,7 +1010,8 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   } else {
     cudaMemsetAsync(w.partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * 4, st);
   }
-  return reduce_renorm(p, sp.S, w.partials, W1, W2, W3, W1o, W2o, W3o, shadow, w.scratch, st);
+  return ns_then_renorm(p, sp.S, w.partials, static_cast<char*>(ws) + tc_main_bytes(p), true, W1,
+                        W2, W3, W1o, W2o, W3o, shadow, w.scratch, st);
 }
 
 template <int D>
@@ -1065,7 +1071,7 @@ SplitPlan tc_split_plan(const Problem& p) {
   return {S, chunk};
 }
 
-size_t tc_workspace_bytes(const Problem& p) {
+size_t tc_main_bytes(const Problem& p) {
   const SplitPlan sp = tc_split_plan(p);
   const size_t wsz = (size_t)p.H * p.hid * p.d;
   const size_t inter = (size_t)p.H * p.n * p.hid;
@@ -1075,6 +1081,8 @@ size_t tc_workspace_bytes(const Problem& p) {
   b += align_up((size_t)p.H * (2 * p.hid + p.d) * 2 * 8, 1024);
   return b;
 }
+
+size_t tc_workspace_bytes(const Problem& p) { return tc_main_bytes(p) + ns_workspace_bytes(p); }
 
 cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const float* W3,
                       const void* K, const void* V, const float* eta, float* W1o, float* W2o,

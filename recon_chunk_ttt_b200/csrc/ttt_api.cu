@@ -21,7 +21,7 @@ ttt_status check_cfg(const ttt_config* cfg) {
   if (cfg->renorm < TTT_RENORM_OFF || cfg->renorm > TTT_RENORM_FROB) return TTT_ERR_INVALID_ARG;
   if (cfg->precision != TTT_PREC_BF16_TC && cfg->precision != TTT_PREC_FP32_CHECK)
     return TTT_ERR_INVALID_ARG;
-  if (cfg->ns_steps != 0) return TTT_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->ns_steps < 0 || cfg->ns_steps > TTT_MAX_NS_STEPS) return TTT_ERR_INVALID_ARG;
   const bool ok = (cfg->d == 64 && cfg->hidden == 128) || (cfg->d == 256 && cfg->hidden == 512);
   if (!ok) return TTT_ERR_UNSUPPORTED_SHAPE;
   return TTT_OK;
@@ -34,6 +34,7 @@ Problem make_problem(const ttt_config* cfg, int64_t n) {
   p.hid = cfg->hidden;
   p.n = n;
   p.renorm = cfg->renorm;
+  p.ns_steps = cfg->ns_steps;
   return p;
 }
 

@@ -46,11 +46,11 @@ def oracle_inputs(x: wl.LayerInputs, precision: int):
     return x
 
 
-def run_update_apply(x: wl.LayerInputs, precision: int, renorm: int):
+def run_update_apply(x: wl.LayerInputs, precision: int, renorm: int, ns_steps: int = 0):
     import recon_chunk_ttt_b200 as R
     torch = torch_mod()
     H, hid, d = x.W1.shape
-    cfg = R.make_config(H, d, hid, renorm=renorm, precision=precision)
+    cfg = R.make_config(H, d, hid, renorm=renorm, precision=precision, ns_steps=ns_steps)
     g = gpu_inputs(x, precision)
     shadow = R.alloc_shadow(cfg)
     W1o, W2o, W3o = R.ttt_update(cfg, g["W1"], g["W2"], g["W3"], g["K"], g["V"], g["eta"],
@@ -62,9 +62,9 @@ def run_update_apply(x: wl.LayerInputs, precision: int, renorm: int):
             W3o.cpu().double().numpy(), O_.float().cpu().double().numpy())
 
 
-def oracle_update_apply(x: wl.LayerInputs, precision: int, renorm: int):
+def oracle_update_apply(x: wl.LayerInputs, precision: int, renorm: int, ns_steps: int = 0):
     xo = oracle_inputs(x, precision)
-    Wh = O.ttt_update(xo.W1, xo.W2, xo.W3, xo.K, xo.V, xo.eta, renorm)
+    Wh = O.ttt_update(xo.W1, xo.W2, xo.W3, xo.K, xo.V, xo.eta, renorm, ns_steps)
     return Wh, O.ttt_apply(*Wh, xo.Q)
 
 

@@ -64,6 +64,12 @@ def test_workspace_sizes(B):
     assert B.ttt_shadow_bytes(cfg) == 3 * 4 * 256 * 512 * 2
     assert B.ttt_update_workspace_bytes(_cfg(B, d=100), 10) == 0
     assert B.ttt_update_workspace_bytes(cfg, -1) == 0
+    # Newton-Schulz: two d x hidden iterates, two d x d products and Delta per
+    # matrix, on top of the update's own workspace (both precisions)
+    for prec in (B.PREC_BF16_TC, B.PREC_FP32_CHECK):
+        base = B.ttt_update_workspace_bytes(_cfg(B, precision=prec), 1000)
+        ns = B.ttt_update_workspace_bytes(_cfg(B, precision=prec, ns_steps=5), 1000)
+        assert ns - base >= 12 * (2 * 256 * 512 + 2 * 256 * 256 + 256 * 512) * 4
 
 
 FAKE = 0x10000  # aligned, never dereferenced: validation fails first
@@ -83,7 +89,8 @@ def _update(B, cfg, n=10, ws_bytes=1 << 40, **over):
 def test_update_rejects_bad_arguments(B):
     assert _update(B, None) == B.TTT_ERR_INVALID_ARG
     assert _update(B, _cfg(B, d=128, hidden=256)) == B.TTT_ERR_UNSUPPORTED_SHAPE
-    assert _update(B, _cfg(B, ns_steps=1)) == B.TTT_ERR_UNSUPPORTED_SHAPE
+    assert _update(B, _cfg(B, ns_steps=-1)) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B, ns_steps=B.MAX_NS_STEPS + 1)) == B.TTT_ERR_INVALID_ARG
     assert _update(B, _cfg(B, renorm=7)) == B.TTT_ERR_INVALID_ARG
     assert _update(B, _cfg(B, precision=5)) == B.TTT_ERR_INVALID_ARG
     assert _update(B, _cfg(B, heads=0)) == B.TTT_ERR_INVALID_ARG
