@@ -265,6 +265,53 @@ def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW,
 
 
 # --------------------------------------------------------------------------
+# Chunked orderings ([survey] part "二、LaCT", "3应用场景"): the sequence is cut
+# into consecutive chunks of b tokens (the last one shorter); per chunk the
+# update U and the apply A run in one of two orders, and U may be skipped on
+# chosen chunks:
+#   update-then-apply (block-causal):  W_i = U(W_{i-1}; c_i), o_i = A(W_i; c_i)
+#   apply-then-update (shifted):       o_i = A(W_{i-1}; c_i), W_i = U(W_{i-1}; c_i)
+#   update mask (cross-chunk causal):  U only where mask[i] is true
+# Fully bidirectional LaCT is apply-then-update with one chunk; the ZipMap
+# layer itself is update-then-apply with one chunk.
+# --------------------------------------------------------------------------
+ORDER_UPDATE_THEN_APPLY, ORDER_APPLY_THEN_UPDATE = 0, 1
+
+
+def chunked(update_fn, apply_fn, W, K, V, eta, Q, b, order, update_mask=None):
+    """Generic chunk loop over any fast-weight model: update_fn(W, K, V, eta)
+    returns the new state, apply_fn(W, Q) the outputs.  Returns the final
+    state and the outputs of every token, in order."""
+    n = np.shape(K)[0]
+    nchunks = (n + b - 1) // b
+    outs = []
+    for i in range(nchunks):
+        s, e = i * b, min(n, (i + 1) * b)
+        upd = True if update_mask is None else bool(update_mask[i])
+        if order == ORDER_APPLY_THEN_UPDATE:
+            outs.append(apply_fn(W, Q[s:e]))
+        if upd:
+            W = update_fn(W, K[s:e], V[s:e], eta[s:e])
+        if order == ORDER_UPDATE_THEN_APPLY:
+            outs.append(apply_fn(W, Q[s:e]))
+    O = np.concatenate(outs, axis=0) if outs else np.zeros((0, np.shape(Q)[1]))
+    return W, O
+
+
+def ttt_chunked(W1, W2, W3, K, V, eta, Q, b, order, update_mask=None,
+                renorm_mode=RENORM_ROW, ns_steps=0):
+    """The chunk loop over the SwiGLU layer (all heads)."""
+    def upd(W, K_, V_, e_):
+        return ttt_update(*W, K_, V_, e_, renorm_mode, ns_steps)
+
+    def app(W, Q_):
+        return ttt_apply(*W, Q_)
+
+    return chunked(upd, app, (_f64(W1), _f64(W2), _f64(W3)), K, V, eta, Q, b, order,
+                   update_mask)
+
+
+# --------------------------------------------------------------------------
 # Linear fast weights ([notes], "为什么它像 attention（线性情形的直观推导）"):
 #   f_W(k) = W k,  L = -(W k)^T v  =>  ∇_W L = -v k^T
 # --------------------------------------------------------------------------

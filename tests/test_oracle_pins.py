@@ -434,3 +434,67 @@ def test_update_with_newton_schulz():
     Wr = O.update_head(W1, W2, W3, K, V, eta, O.RENORM_ROW, ns_steps=3)
     for a_, b_ in zip(Wr, (W1, W2, W3)):
         np.testing.assert_allclose(np.linalg.norm(a_, axis=1), np.linalg.norm(b_, axis=1), rtol=1e-13)
+
+
+# ------------------------------------------------------- chunked orderings
+def _block_causal_linear_attention(W0, K, V, eta, Q, b, strict, mask=None):
+    """Brute force: o_t = W0 q_t + sum over earlier tokens s of eta_s v_s (k_s.q_t)
+    where s runs over the updating chunks before t's chunk, plus t's own chunk
+    unless `strict`.  This is linear attention with a block mask."""
+    n = K.shape[0]
+    O = Q @ W0.T
+    for t in range(n):
+        ct = t // b
+        for s_ in range(n):
+            cs = s_ // b
+            if mask is not None and not mask[cs]:
+                continue
+            if cs < ct or (cs == ct and not strict):
+                O[t] += eta[s_] * V[s_] * (K[s_] @ Q[t])
+    return O
+
+
+@pytest.mark.parametrize("b", [1, 3, 4, 11])
+def test_chunked_orders_are_block_causal_linear_attention(b):
+    """Linear fast weights, renorm off ([notes] linear case): update-then-apply
+    is inclusive block-causal linear attention, apply-then-update the strict
+    (shifted) one, and an update mask drops the masked chunks' keys."""
+    rng = np.random.default_rng(b)
+    n, d = 11, 5
+    W0 = rng.standard_normal((d, d)) * 0.3
+    K, V, Q = (rng.standard_normal((n, d)) for _ in range(3))
+    eta = 0.05 + rng.random(n)
+    upd = lambda W, K_, V_, e_: O.linear_update(W, K_, V_, e_, O.RENORM_OFF)  # noqa: E731
+    app = O.linear_apply
+    for order, strict in ((O.ORDER_UPDATE_THEN_APPLY, False), (O.ORDER_APPLY_THEN_UPDATE, True)):
+        Wf, Out = O.chunked(upd, app, W0, K, V, eta, Q, b, order)
+        np.testing.assert_allclose(Out, _block_causal_linear_attention(W0, K, V, eta, Q, b, strict),
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(Wf, O.linear_update(W0, K, V, eta), rtol=1e-12, atol=1e-12)
+    mask = [(i % 2) == 0 for i in range((n + b - 1) // b)]
+    _, Out = O.chunked(upd, app, W0, K, V, eta, Q, b, O.ORDER_UPDATE_THEN_APPLY, mask)
+    np.testing.assert_allclose(Out, _block_causal_linear_attention(W0, K, V, eta, Q, b, False, mask),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_chunked_swiglu_special_cases():
+    x = wl.make_inputs("tiny")
+    W = (x.W1, x.W2, x.W3)
+    n = x.K.shape[0]
+    # one chunk, update-then-apply: the ZipMap layer
+    Wf, Out = O.ttt_chunked(*W, x.K, x.V, x.eta, x.Q, n, O.ORDER_UPDATE_THEN_APPLY)
+    Wu = O.ttt_update(*W, x.K, x.V, x.eta)
+    np.testing.assert_allclose(Out, rtol=1e-13, atol=1e-15, desired=O.ttt_apply(*Wu, x.Q))
+    # one chunk, apply-then-update: outputs read the initial state
+    Wf, Out = O.ttt_chunked(*W, x.K, x.V, x.eta, x.Q, n, O.ORDER_APPLY_THEN_UPDATE)
+    np.testing.assert_allclose(Out, rtol=1e-13, atol=1e-15, desired=O.ttt_apply(*W, x.Q))
+    for a_, b_ in zip(Wf, Wu):
+        np.testing.assert_allclose(a_, b_, rtol=1e-13, atol=1e-15)
+    # no chunk updates: every output reads the initial state, W unchanged
+    Wf, Out = O.ttt_chunked(*W, x.K, x.V, x.eta, x.Q, 40, O.ORDER_UPDATE_THEN_APPLY,
+                            update_mask=[0, 0, 0])
+    np.testing.assert_allclose(Out, rtol=1e-13, atol=1e-15, desired=O.ttt_apply(*W, x.Q))
+    # update-then-apply with frame-sized chunks is the streaming recurrence
+    Wf, Out = O.ttt_chunked(*W, x.K, x.V, x.eta, x.Q, 49, O.ORDER_UPDATE_THEN_APPLY)
+    Ws, Os = O.ttt_stream(*W, x.K, x.V, x.eta, x.Q, 49)
+    np.testing.assert_allclose(Out, rtol=1e-13, atol=1e-15, desired=Os)
