@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-stream", action="store_true")
+    ap.add_argument("--ns-steps", type=int, default=0,
+                    help="Newton-Schulz steps on the gradient in the timed step (0: off)")
+    ap.add_argument("--no-ns-probe", action="store_true",
+                    help="skip the separate 5-step Newton-Schulz update measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -255,7 +259,10 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     layers = args.layers or w.layers
     H, d, hid = w.heads, w.d, w.hidden
     T, M = w.n_tokens, w.n_ray
-    cfg = R.make_config(H, d, hid, renorm=R.RENORM_ROW, precision=R.PREC_BF16_TC)
+    cfg = R.make_config(H, d, hid, renorm=R.RENORM_ROW, precision=R.PREC_BF16_TC,
+                        ns_steps=args.ns_steps)
+    cfg_ns = R.make_config(H, d, hid, renorm=R.RENORM_ROW, precision=R.PREC_BF16_TC,
+                           ns_steps=max(args.ns_steps, 5))
 
     x = wl.make_inputs(w, bits=True)
     to_bf = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)  # noqa: E731
@@ -278,7 +285,7 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     Win = [tuple(t.to(dev) for t in ws) for ws in hW]
     Wout = [tuple(torch.empty_like(t) for t in ws) for ws in Win]
     shadow = R.alloc_shadow(cfg, dev)
-    ws_buf = R.alloc_workspace(cfg, T, dev)
+    ws_buf = R.alloc_workspace(cfg_ns, T, dev)  # also large enough for cfg
     O = torch.empty((T, H * d), dtype=torch.bfloat16, device=dev)
     Or = torch.empty((M, H * d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -371,12 +378,18 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
                 "update_ms_per_layer": upd_ms / (layers * args.steps)},
             "kernels": per_kernel, "clocks": clk,
             "gpu_launches": int(sum(v[0] for v in trace.values()))}
+    if args.ns_steps:
+        line["config"]["ns_steps"] = args.ns_steps
 
     # -------------------------------------------------- e2e through host buffers
     if not args.no_e2e:
         line["e2e"] = e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta,
                           Win, Wout, shadow, ws_buf, O, Or, layers, T, M, world, barrier,
                           rank_max)
+    # -------------------------------------------------- Newton-Schulz update
+    if not args.no_ns_probe:
+        line["ns_update"] = ns_probe(R, torch, dev, cfg_ns, K, V, eta, Win[0], Wout[0], shadow,
+                                     ws_buf, stream, d, hid, H, pk, rank_max)
     # -------------------------------------------------- streaming (stream256)
     if not args.no_stream:
         line["stream"] = stream_bench(R, torch, dev, rank_max)
@@ -388,6 +401,44 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def ns_probe(R, torch, dev, cfg, K, V, eta, Win, Wout, shadow, ws, stream, d, hid, H, pk,
+             rank_max, reps: int = 5) -> dict:
+    """One layer's update with Newton-Schulz on (cfg.ns_steps steps of Muon's
+    quintic on each of the 3*H gradient matrices), after 2 untimed runs.
+    Reports the whole update per layer and the NS stages from the library's
+    trace (events on the stream).  Algorithmic NS flops per matrix and step:
+    2 Rp^2 hidden (X X^T) + 2 Rp^3 (A A) + 2 Rp^2 hidden (B X), Rp = d."""
+    steps = cfg.ns_steps
+    for _ in range(2):
+        R.ttt_update(cfg, *Win, K, V, eta, *Wout, shadow=shadow, workspace=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    R.ttt_trace_enable(True)
+    R.ttt_trace_read(reset=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        R.ttt_update(cfg, *Win, K, V, eta, *Wout, shadow=shadow, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    R.ttt_trace_enable(False)
+    tr = R.ttt_trace_read(reset=True)
+    R.ttt_check_device_error()
+    upd = rank_max(e0.elapsed_time(e1) / reps)
+    ns_names = ("ns_prepare", "ns_tc_iterate", "ns_finish")
+    ns_ms = sum(tr.get(k, (0, 0.0))[1] for k in ns_names) / reps
+    it_ms = tr.get("ns_tc_iterate", (0, 0.0))[1] / reps
+    flops = 3 * H * steps * (4 * d * d * hid + 2 * d ** 3)
+    ach = flops / (it_ms / 1e3) / 1e12 if it_ms else None
+    return {"ns_steps": steps, "update_ms_per_layer": upd,
+            "ns_stage_ms": ns_ms, "ns_iterate_ms": it_ms,
+            "ns_stage_share_of_update": ns_ms / upd if upd else None,
+            "ns_iterate_tflops": ach,
+            "ns_iterate_frac_of_burst": ach / pk["bf16_tflops"] if ach else None,
+            "stages_ms": {k: tr[k][1] / reps for k in ns_names if k in tr},
+            "note": "NS GEMMs issue 3 bf16 MMAs per product (hi/lo operand split); "
+                    "achieved counts the algorithmic flops once"}
 
 
 def stream_bench(R, torch, dev, rank_max, warm_frames: int = 8) -> dict:

@@ -161,6 +161,37 @@ ttt_status ttt_stream_step(const ttt_config* cfg,
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
 
 /*
+ * LaCT chunked orderings (mhpn.cn survey of TTSA3R / LaCT / ZipMap / LoGeR,
+ * part "二、LaCT", "3应用场景"): the n tokens are cut into consecutive chunks of
+ * `chunk` tokens (the last one shorter), and chunk i = tokens
+ * [i*chunk, min(n, (i+1)*chunk)) is processed in order:
+ *   TTT_ORDER_UPDATE_THEN_APPLY (block-causal): W <- U(W; chunk i) if the
+ *       chunk updates, then O[chunk i] = f_W(Q[chunk i]);
+ *   TTT_ORDER_APPLY_THEN_UPDATE (shifted block-causal): O[chunk i] =
+ *       f_W(Q[chunk i]) with the state before the chunk, then W <- U(W; chunk i)
+ *       if the chunk updates.
+ * U is the update of ttt_update (with cfg's renorm and ns_steps), in place.
+ * `update_mask` is a HOST array of ceil(n/chunk) bytes (nonzero = the chunk
+ * updates) or NULL (every chunk updates); updating only chosen chunks gives the
+ * cross-chunk causal pattern.  One chunk with APPLY_THEN_UPDATE is LaCT's
+ * fully bidirectional pattern; one chunk with UPDATE_THEN_APPLY is the ZipMap
+ * layer, and frame-sized chunks its streaming recurrence.
+ *  - Arguments as in ttt_stream_step, with Q and O for the same n tokens
+ *    (each token has a query): K, V, Q [n][H*d], eta [n][H], O [n][H*d].
+ *  - BF16_TC: `shadow` is required; when the first operation is an apply it
+ *    is first packed from W (the caller's contents do not matter).
+ *    FP32_CHECK: `shadow` may be NULL.
+ *  - chunk >= 1 and chunk * heads a multiple of 4 (every chunk's eta rows
+ *    then start 16-byte aligned); workspace: ttt_update_workspace_bytes(cfg,
+ *    min(chunk, n)).  Every argument is checked before anything is enqueued.
+ */
+enum { TTT_ORDER_UPDATE_THEN_APPLY = 0, TTT_ORDER_APPLY_THEN_UPDATE = 1 };
+ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, void* shadow,
+                       const void* K, const void* V, const float* eta, const void* Q,
+                       int64_t n, int64_t chunk, int32_t order, const uint8_t* update_mask,
+                       void* O, void* workspace, size_t workspace_bytes, ttt_stream_t stream);
+
+/*
  * Allocation-free streaming step (the pages have no counterpart: this is a
  * deployment aid).  Same arguments and result as ttt_stream_step() minus the
  * workspace: the scratch is a fixed TTT_STATIC_SCRATCH_BYTES device array

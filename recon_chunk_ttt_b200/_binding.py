@@ -77,6 +77,9 @@ def lib() -> ctypes.CDLL:
         L.ttt_stream_step.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P, _P,
                                       ctypes.c_size_t, _P]
         L.ttt_stream_step.restype = ctypes.c_int
+        L.ttt_chunked.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
+                                  ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
+        L.ttt_chunked.restype = ctypes.c_int
         L.ttt_check_device_error.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
         L.ttt_check_device_error.restype = ctypes.c_int
         L.ttt_trace_enable.argtypes = [ctypes.c_int32]
@@ -182,6 +185,32 @@ def ttt_stream_step(cfg: ttt_config, W1, W2, W3, shadow, K, V, eta, Q, O=None,
     _check(lib().ttt_stream_step(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W3), _ptr(shadow),
                                  _ptr(K), _ptr(V), _ptr(eta), n, _ptr(Q), m, _ptr(O),
                                  _ptr(workspace), nbytes, _stream(stream)), "ttt_stream_step")
+    return O
+
+
+ORDER_UPDATE_THEN_APPLY, ORDER_APPLY_THEN_UPDATE = 0, 1  # TTT_ORDER_*
+
+
+def ttt_chunked(cfg: ttt_config, W1, W2, W3, shadow, K, V, eta, Q, chunk: int,
+                order: int = ORDER_UPDATE_THEN_APPLY, update_mask=None, O=None,
+                workspace=None, stream=None):
+    """Chunk loop over the n tokens (update and apply per chunk in `order`,
+    updates only where update_mask is nonzero); the state (W1, W2, W3,
+    shadow) is updated in place; returns O for all n tokens."""
+    n = int(K.shape[0])
+    if O is None:
+        O = torch.empty((n, cfg.heads * cfg.d), dtype=_token_dtype(cfg), device=Q.device)
+    first = min(int(chunk), n) if n else 0
+    if workspace is None:
+        workspace = alloc_workspace(cfg, first, W1.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    mask = None
+    if update_mask is not None:
+        mask = (ctypes.c_uint8 * len(update_mask))(*[1 if m else 0 for m in update_mask])
+    _check(lib().ttt_chunked(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W3), _ptr(shadow),
+                             _ptr(K), _ptr(V), _ptr(eta), _ptr(Q), n, int(chunk), int(order),
+                             mask, _ptr(O), _ptr(workspace), nbytes, _stream(stream)),
+           "ttt_chunked")
     return O
 
 

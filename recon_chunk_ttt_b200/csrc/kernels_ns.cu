@@ -56,16 +56,25 @@ __global__ void __launch_bounds__(256) ns_gather_kernel(const float* __restrict_
   const int c0 = (t / tiles_j) * 32, j0 = (t % tiles_j) * 32;  // working rows c, cols j
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const size_t mat = (size_t)hid * d;
+  // blocks 0/1: read G rows j (coalesced along c); block 2: read rows c
+  // (coalesced along j).  tile[a][b] holds working element (c0+b, j0+a) for
+  // blocks 0/1 and (c0+a, j0+b) for block 2.  Each thread owns 4 elements
+  // (rows ty, ty+8, ...) and sums them over s in increasing order.
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int s = 0; s < S; ++s) {
+    const float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 8 * i;
+      const size_t off = blk < 2 ? (size_t)(j0 + r) * d + c0 + tx : (size_t)(c0 + r) * hid + j0 + tx;
+      acc[i] += (double)P[off];
+    }
+  }
   double ss = 0.0;
-  for (int r = ty; r < 32; r += 8) {
-    // blocks 0/1: read G rows j (coalesced along c); block 2: read rows c
-    // (coalesced along j).  tile[a][b] holds working element (c0+b, j0+a) for
-    // blocks 0/1 and (c0+a, j0+b) for block 2.
-    const size_t off = blk < 2 ? (size_t)(j0 + r) * d + c0 + tx : (size_t)(c0 + r) * hid + j0 + tx;
-    double acc = 0.0;
-    for (int s = 0; s < S; ++s) acc += (double)partials[(((size_t)s * H + head) * 3 + blk) * mat + off];
-    const float v = blk < 2 ? (float)acc : (float)(-acc);
-    tile[r][tx] = v;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float v = blk < 2 ? (float)acc[i] : (float)(-acc[i]);
+    tile[ty + 8 * i][tx] = v;
     ss = fma((double)v, (double)v, ss);
   }
   __syncthreads();
@@ -94,10 +103,13 @@ __global__ void __launch_bounds__(256) ns_scale_kernel(int d, int hid, int Rp, i
                                                        float* __restrict__ X) {
   __shared__ double inv;
   const int m = blockIdx.y;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
+    // lane l sums tiles l, l+32, ... in order; then a fixed butterfly
     double s = 0.0;
-    for (int i = 0; i < tiles; ++i) s += tile_ss[(size_t)m * tiles + i];
-    inv = s > 0.0 ? 1.0 / sqrt(s) : 0.0;
+    for (int i = threadIdx.x; i < tiles; i += 32) s += tile_ss[(size_t)m * tiles + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (threadIdx.x == 0) inv = s > 0.0 ? 1.0 / sqrt(s) : 0.0;
   }
   __syncthreads();
   const int rows_per = Rp / gridDim.x;
@@ -261,35 +273,67 @@ __device__ __forceinline__ void split_store(uint8_t* hi, uint8_t* lo, uint32_t o
 }
 
 // K-major tile: 128 rows (r0..) x 64 k (k0..) of a row-major fp32 matrix.
-// Row r holds 128 bytes; its 16-byte unit u sits at unit u ^ (r & 7).
-__device__ __forceinline__ void fill_kmajor(uint8_t* hi, uint8_t* lo, const float* M, int ld,
-                                            int r0, int k0) {
-  for (int u = threadIdx.x; u < 128 * 8; u += NSL<256, 512>::THREADS) {
+// Row r holds 128 bytes; its 16-byte unit u sits at unit u ^ (r & 7).  The
+// 1024 units (8 floats each) are split 4 per thread; all loads are issued
+// before the first conversion so the L2 round trips overlap.
+struct KTile {
+  float4 v[4][2];
+};
+__device__ __forceinline__ void load_kmajor(KTile& t, const float* M, int ld, int r0, int k0) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int u = threadIdx.x + 256 * i;
     const int row = u >> 3, cu = u & 7;
     const float4* src = reinterpret_cast<const float4*>(M + (size_t)(r0 + row) * ld + k0 + cu * 8);
-    split_store(hi, lo, row * 128 + ((cu ^ (row & 7)) << 4), __ldcg(src), __ldcg(src + 1));
+    t.v[i][0] = __ldcg(src);
+    t.v[i][1] = __ldcg(src + 1);
+  }
+}
+__device__ __forceinline__ void store_kmajor(const KTile& t, uint8_t* hi, uint8_t* lo) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int u = threadIdx.x + 256 * i;
+    const int row = u >> 3, cu = u & 7;
+    split_store(hi, lo, row * 128 + ((cu ^ (row & 7)) << 4), t.v[i][0], t.v[i][1]);
   }
 }
 
 // MN-major tile: 64 k rows (k0..) x N columns (n0..) of a row-major fp32
 // matrix.  Column block nb of 64 sits at nb * 8192; inside it k row k holds
-// 128 bytes with unit u at u ^ (k & 7).
+// 128 bytes with unit u at u ^ (k & 7).  64 * N / 8 units, N / 32 per thread.
 template <int N>
-__device__ __forceinline__ void fill_mnmajor(uint8_t* hi, uint8_t* lo, const float* M, int ld,
-                                             int k0, int n0) {
+struct MTile {
+  float4 v[N / 32][2];
+};
+template <int N>
+__device__ __forceinline__ void load_mnmajor(MTile<N>& t, const float* M, int ld, int k0, int n0) {
   constexpr int UPR = N / 8;  // 16-byte units per k row
-  for (int u = threadIdx.x; u < 64 * UPR; u += NSL<256, 512>::THREADS) {
+#pragma unroll
+  for (int i = 0; i < N / 32; ++i) {
+    const int u = threadIdx.x + 256 * i;
+    const int k = u / UPR, cn = u % UPR;
+    const float4* src = reinterpret_cast<const float4*>(M + (size_t)(k0 + k) * ld + n0 + cn * 8);
+    t.v[i][0] = __ldcg(src);
+    t.v[i][1] = __ldcg(src + 1);
+  }
+}
+template <int N>
+__device__ __forceinline__ void store_mnmajor(const MTile<N>& t, uint8_t* hi, uint8_t* lo) {
+  constexpr int UPR = N / 8;
+#pragma unroll
+  for (int i = 0; i < N / 32; ++i) {
+    const int u = threadIdx.x + 256 * i;
     const int k = u / UPR, cn = u % UPR;
     const int nb = cn >> 3, cu = cn & 7;
-    const float4* src = reinterpret_cast<const float4*>(M + (size_t)(k0 + k) * ld + n0 + cn * 8);
-    split_store(hi, lo, nb * 8192 + k * 128 + ((cu ^ (k & 7)) << 4), __ldcg(src), __ldcg(src + 1));
+    split_store(hi, lo, nb * 8192 + k * 128 + ((cu ^ (k & 7)) << 4), t.v[i][0], t.v[i][1]);
   }
 }
 
 // acc[TMEM cols 0..N) = A-op (rows a_r0 of Am, K-major) x B-op over `nchunks`
 // k chunks of 64.  B-op: rows b_off of Bm (K-major, N = 128) or, when B_MN,
 // columns b_off.. of Bm (MN-major).  gchunk counts chunks over the kernel
-// (stage = gchunk & 1, use = gchunk >> 1).  Returns once the MMAs completed.
+// (stage = gchunk & 1, use = gchunk >> 1).  Returns with the MMAs in flight;
+// the epilogue waits for them.
 template <int N, bool B_MN, class L>
 __device__ __forceinline__ void ns_gemm(uint8_t* smem, uint64_t* bars, uint32_t tmem, int& gchunk,
                                         int nchunks, const float* Am, int lda, int a_r0,
@@ -298,14 +342,24 @@ __device__ __forceinline__ void ns_gemm(uint8_t* smem, uint64_t* bars, uint32_t 
   const uint32_t idesc = idesc_bf16_f32(128, N, false, B_MN);
   for (int j = 0; j < nchunks; ++j, ++gchunk) {
     const int s = gchunk & 1;
-    if (gchunk >= 2) mbar_wait(&bars[s], ((gchunk >> 1) - 1) & 1, abort, err, kErrWaitEmpty);
     uint8_t* st = smem + s * L::STAGE;
     uint8_t* bst = st + 2 * L::A_T;
-    fill_kmajor(st, st + L::A_T, Am, lda, a_r0, j * 64);
-    if (B_MN)
-      fill_mnmajor<N>(bst, bst + L::B_T, Bm, ldb, j * 64, b_off);
-    else
-      fill_kmajor(bst, bst + L::B_T, Bm, ldb, b_off, j * 64);
+    // loads first (registers only), then wait for the stage's previous MMAs
+    KTile ta;
+    load_kmajor(ta, Am, lda, a_r0, j * 64);
+    if constexpr (B_MN) {
+      MTile<N> tb;
+      load_mnmajor<N>(tb, Bm, ldb, j * 64, b_off);
+      if (gchunk >= 2) mbar_wait(&bars[s], ((gchunk >> 1) - 1) & 1, abort, err, kErrWaitEmpty);
+      store_kmajor(ta, st, st + L::A_T);
+      store_mnmajor<N>(tb, bst, bst + L::B_T);
+    } else {
+      KTile tb;
+      load_kmajor(tb, Bm, ldb, b_off, j * 64);
+      if (gchunk >= 2) mbar_wait(&bars[s], ((gchunk >> 1) - 1) & 1, abort, err, kErrWaitEmpty);
+      store_kmajor(ta, st, st + L::A_T);
+      store_kmajor(tb, bst, bst + L::B_T);
+    }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -326,42 +380,46 @@ __device__ __forceinline__ void ns_gemm(uint8_t* smem, uint64_t* bars, uint32_t 
       umma_commit(&bars[s]);
     }
   }
-  const int last = gchunk - 1;
-  mbar_wait(&bars[last & 1], (last >> 1) & 1, abort, err, kErrWaitAcc);
-  tc_fence_after();
 }
 
 // Epilogue of one 128 x N tile: warp w reads TMEM lanes 32*(w%4).. (its rows)
 // and half (w/4) of the columns.  MODE 0: O = acc; 1: O = b R + c acc;
-// 2: O = a R + acc.  R has O's pitch and position.
+// 2: O = a R + acc.  R has O's pitch and position.  R is read before the
+// wait for the MMAs (chunk `last`), so its round trip overlaps them.
 template <int N, int MODE>
-__device__ __forceinline__ void ns_epilogue(uint32_t tmem, float* O, const float* R, int ld,
-                                            int r0, int c0) {
+__device__ __forceinline__ void ns_epilogue(uint64_t* bars, int last, uint32_t tmem, float* O,
+                                            const float* R, int ld, int r0, int c0,
+                                            volatile int* abort, int* err) {
+  constexpr int HALF = N / 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, half = warp >> 2;
-  const size_t row = (size_t)(r0 + 32 * q + lane) * ld;
-#pragma unroll 1
-  for (int j = 0; j < N / 64; ++j) {
-    const int col = half * (N / 2) + 32 * j;
+  const size_t base = (size_t)(r0 + 32 * q + lane) * ld + c0 + half * HALF;
+  float4 rv[MODE != 0 ? HALF / 4 : 1];
+  if constexpr (MODE != 0) {
+#pragma unroll
+    for (int i = 0; i < HALF / 4; ++i) rv[i] = __ldcg(reinterpret_cast<const float4*>(R + base) + i);
+  }
+  mbar_wait(&bars[last & 1], (last >> 1) & 1, abort, err, kErrWaitAcc);
+  tc_fence_after();
+#pragma unroll
+  for (int j = 0; j < HALF / 32; ++j) {
     uint32_t v[32];
-    tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, v);
+    tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HALF + 32 * j), v);
     tmem_ld_wait();
-    float* o = O + row + c0 + col;
-    const float* rr = R + row + c0 + col;
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
       float4 x = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
                              __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-      if (MODE == 1) {
-        const float4 y = __ldcg(reinterpret_cast<const float4*>(rr + i));
+      if constexpr (MODE == 1) {
+        const float4 y = rv[(32 * j + i) / 4];
         x = make_float4(fmaf(kNsC, x.x, kNsB * y.x), fmaf(kNsC, x.y, kNsB * y.y),
                         fmaf(kNsC, x.z, kNsB * y.z), fmaf(kNsC, x.w, kNsB * y.w));
-      } else if (MODE == 2) {
-        const float4 y = __ldcg(reinterpret_cast<const float4*>(rr + i));
+      } else if constexpr (MODE == 2) {
+        const float4 y = rv[(32 * j + i) / 4];
         x = make_float4(fmaf(kNsA, y.x, x.x), fmaf(kNsA, y.y, x.y), fmaf(kNsA, y.z, x.z),
                         fmaf(kNsA, y.w, x.w));
       }
-      __stcg(reinterpret_cast<float4*>(o + i), x);
+      __stcg(reinterpret_cast<float4*>(O + base + 32 * j + i), x);
     }
   }
   tc_fence_before();
@@ -412,15 +470,15 @@ __global__ void __launch_bounds__(256, 1) ns_tc_kernel(float* X0, float* X1, flo
     float* Xn = (it & 1) ? Xa : Xb;
     ns_gemm<128, false, L>(smem, bars, tmem, g, C / 64, Xc, C, mi * 128, Xc, C, ni * 128,
                            abort_flag, err);
-    ns_epilogue<128, 0>(tmem, A, nullptr, RP, mi * 128, ni * 128);
+    ns_epilogue<128, 0>(bars, g - 1, tmem, A, nullptr, RP, mi * 128, ni * 128, abort_flag, err);
     ns_sync<L::CL>();
     ns_gemm<128, false, L>(smem, bars, tmem, g, RP / 64, A, RP, mi * 128, A, RP, ni * 128,
                            abort_flag, err);
-    ns_epilogue<128, 1>(tmem, B, A, RP, mi * 128, ni * 128);
+    ns_epilogue<128, 1>(bars, g - 1, tmem, B, A, RP, mi * 128, ni * 128, abort_flag, err);
     ns_sync<L::CL>();
     ns_gemm<L::N3, true, L>(smem, bars, tmem, g, RP / 64, B, RP, mi * 128, Xc, C, ni * L::N3,
                             abort_flag, err);
-    ns_epilogue<L::N3, 2>(tmem, Xn, Xc, C, mi * 128, ni * L::N3);
+    ns_epilogue<L::N3, 2>(bars, g - 1, tmem, Xn, Xc, C, mi * 128, ni * L::N3, abort_flag, err);
     ns_sync<L::CL>();
   }
   tc_fence_before();

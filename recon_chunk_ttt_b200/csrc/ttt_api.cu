@@ -154,6 +154,67 @@ ttt_status ttt_stream_step(const ttt_config* cfg, float* W1, float* W2, float* W
   return ttt_apply(cfg, W1, W2, W3, shadow, Q, m, O, stream);
 }
 
+ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, void* shadow,
+                       const void* K, const void* V, const float* eta, const void* Q,
+                       int64_t n, int64_t chunk, int32_t order, const uint8_t* update_mask,
+                       void* O, void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (n < 0 || n > kMaxTokens || chunk < 1) return TTT_ERR_INVALID_ARG;
+  if (order != TTT_ORDER_UPDATE_THEN_APPLY && order != TTT_ORDER_APPLY_THEN_UPDATE)
+    return TTT_ERR_INVALID_ARG;
+  if (!W1 || !W2 || !W3) return TTT_ERR_INVALID_ARG;
+  const bool tc = cfg->precision == TTT_PREC_BF16_TC;
+  if (tc && !shadow) return TTT_ERR_INVALID_ARG;
+  if (n == 0) return TTT_OK;
+  if (!K || !V || !eta || !Q || !O) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {W1, W2, W3, shadow, K, V, eta, Q, O, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  if ((chunk * cfg->heads) % 4 != 0) return TTT_ERR_ALIGNMENT;
+  const int64_t first = chunk < n ? chunk : n;
+  const int64_t nchunks = (n + chunk - 1) / chunk;
+  bool any_update = false;
+  for (int64_t i = 0; i < nchunks; ++i) any_update |= update_mask == nullptr || update_mask[i] != 0;
+  if (any_update) {
+    const Problem p = make_problem(cfg, first);
+    const size_t need = tc ? ttt::tc_workspace_bytes(p) : ttt::f32_workspace_bytes(p);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  }
+  // Every chunk's pointers keep the base alignment (token rows are multiples
+  // of 128 bytes, eta rows start at multiples of 16 bytes), and no chunk is
+  // longer than the first, so the per-chunk calls below pass their checks.
+  const size_t tok = (size_t)cfg->heads * cfg->d * (tc ? 2 : 4);
+  const char* k8 = static_cast<const char*>(K);
+  const char* v8 = static_cast<const char*>(V);
+  const char* q8 = static_cast<const char*>(Q);
+  char* o8 = static_cast<char*>(O);
+  const bool first_is_apply = order == TTT_ORDER_APPLY_THEN_UPDATE ||
+                              (update_mask != nullptr && update_mask[0] == 0);
+  if (tc && first_is_apply) {
+    s = ttt_pack_shadow(cfg, W1, W2, W3, shadow, stream);
+    if (s != TTT_OK) return s;
+  }
+  for (int64_t i = 0; i < nchunks; ++i) {
+    const int64_t s0 = i * chunk, len = (s0 + chunk <= n ? chunk : n - s0);
+    const bool upd = update_mask == nullptr || update_mask[i] != 0;
+    if (order == TTT_ORDER_APPLY_THEN_UPDATE) {
+      s = ttt_apply(cfg, W1, W2, W3, shadow, q8 + s0 * tok, len, o8 + s0 * tok, stream);
+      if (s != TTT_OK) return s;
+    }
+    if (upd) {
+      s = ttt_update(cfg, W1, W2, W3, k8 + s0 * tok, v8 + s0 * tok, eta + s0 * cfg->heads, len,
+                     W1, W2, W3, shadow, workspace, workspace_bytes, stream);
+      if (s != TTT_OK) return s;
+    }
+    if (order == TTT_ORDER_UPDATE_THEN_APPLY) {
+      s = ttt_apply(cfg, W1, W2, W3, shadow, q8 + s0 * tok, len, o8 + s0 * tok, stream);
+      if (s != TTT_OK) return s;
+    }
+  }
+  return TTT_OK;
+}
+
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return TTT_ERR_CUDA;

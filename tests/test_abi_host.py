@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("ttt_update", "ttt_apply", "ttt_stream_step", "ttt_update_workspace_bytes",
               "ttt_status_string", "ttt_shadow_bytes", "ttt_pack_shadow",
-              "ttt_check_device_error"):
+              "ttt_check_device_error", "ttt_chunked"):
         assert n in names
 
 
@@ -131,3 +131,34 @@ def test_product_path_does_not_touch_the_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "ttt_oracle" not in txt, f
+
+
+def test_chunked_rejects_bad_arguments(B):
+    """Validation of ttt_chunked happens before any launch (FAKE pointers are
+    never dereferenced)."""
+    L = B.lib()
+    cfg = _cfg(B)
+
+    def call(cfg_, n=100, chunk=16, order=0, shadow=FAKE, eta=FAKE, ws=FAKE, ws_bytes=1 << 40,
+             mask=None):
+        return L.ttt_chunked(ctypes.byref(cfg_), FAKE, FAKE, FAKE, shadow, FAKE, FAKE, eta, FAKE,
+                             n, chunk, order, mask, FAKE, ws, ws_bytes, None)
+
+    assert call(cfg, order=2) == B.TTT_ERR_INVALID_ARG
+    assert call(cfg, chunk=0) == B.TTT_ERR_INVALID_ARG
+    assert call(cfg, n=-1) == B.TTT_ERR_INVALID_ARG
+    assert call(cfg, shadow=None) == B.TTT_ERR_INVALID_ARG      # bf16 needs the shadow
+    assert call(cfg, eta=FAKE + 4) == B.TTT_ERR_ALIGNMENT
+    one_head = _cfg(B, heads=1)
+    assert call(one_head, chunk=6) == B.TTT_ERR_ALIGNMENT       # eta rows of chunk 2 misaligned
+    assert call(cfg, ws=None) == B.TTT_ERR_WORKSPACE
+    assert call(cfg, ws_bytes=100) == B.TTT_ERR_WORKSPACE
+    # the workspace is sized for the first (longest) chunk
+    need = B.ttt_update_workspace_bytes(cfg, 16)
+    assert need > 0 and call(cfg, ws_bytes=need - 1) == B.TTT_ERR_WORKSPACE
+    # no chunk updates: no workspace needed; n = 0 is a no-op
+    none = (ctypes.c_uint8 * 7)(*([0] * 7))
+    assert call(cfg, n=0, ws=None) == B.TTT_OK
+    f32 = _cfg(B, precision=B.PREC_FP32_CHECK)
+    assert call(f32, n=0, shadow=None) == B.TTT_OK
+    assert call(cfg, ws=None, mask=none, n=0) == B.TTT_OK
