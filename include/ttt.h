@@ -161,6 +161,37 @@ ttt_status ttt_stream_step(const ttt_config* cfg,
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
 
 /*
+ * Token-sharded update across ranks (one chunk's tokens split over several
+ * GPUs; the pages describe one GPU, this is the data-parallel form of the
+ * same sum).  Eq. 3's g is a sum over tokens, so each rank reduces its own
+ * tokens to a partial and the ranks exchange partials (an all-gather, e.g.
+ * NCCL over NVLink, done by the caller); every rank then forms the same Ŵ.
+ *
+ * ttt_update_partial: the gradient partial of this rank's n tokens (weights
+ *   W, tokens K, V, eta as in ttt_update) into `partial`, fp32, layout
+ *   [H][3][hidden*d]: block 0 = g1 ([hidden][d]), block 1 = g3 ([hidden][d]),
+ *   block 2 = −g2 ([d][hidden]); ttt_partial_floats(cfg) floats.  Partials add
+ *   elementwise.  Workspace: ttt_update_workspace_bytes(cfg, n).  n = 0 gives
+ *   zeros.
+ * ttt_update_finish: Ŵ from `ranks` partials stored one after another
+ *   ([ranks][H][3][hidden*d]), summed in rank order in fp64 (so the result
+ *   does not depend on which rank computes it, and all ranks agree bitwise),
+ *   then NewtonSchulz (cfg.ns_steps > 0) and the renormalisation as in
+ *   ttt_update, against the pre-update W.  Outputs and shadow as in
+ *   ttt_update (may alias W).  Workspace: ttt_finish_workspace_bytes(cfg).
+ */
+size_t ttt_partial_floats(const ttt_config* cfg);
+size_t ttt_finish_workspace_bytes(const ttt_config* cfg);
+ttt_status ttt_update_partial(const ttt_config* cfg, const float* W1, const float* W2,
+                              const float* W3, const void* K, const void* V, const float* eta,
+                              int64_t n, float* partial, void* workspace, size_t workspace_bytes,
+                              ttt_stream_t stream);
+ttt_status ttt_update_finish(const ttt_config* cfg, const float* W1, const float* W2,
+                             const float* W3, const float* partials, int32_t ranks,
+                             float* W1_out, float* W2_out, float* W3_out, void* shadow,
+                             void* workspace, size_t workspace_bytes, ttt_stream_t stream);
+
+/*
  * LaCT chunked orderings (mhpn.cn survey of TTSA3R / LaCT / ZipMap / LoGeR,
  * part "二、LaCT", "3应用场景"): the n tokens are cut into consecutive chunks of
  * `chunk` tokens (the last one shorter), and chunk i = tokens

@@ -265,6 +265,39 @@ def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW,
 
 
 # --------------------------------------------------------------------------
+# Token-sharded form of Eq. 3 ([review] section 2: g sums over every token, so
+# any split of the tokens into shards sums to the same g).  Partial layout per
+# head: [g1 (hidden x d), g3 (hidden x d), -g2 (d x hidden)], flattened.
+# --------------------------------------------------------------------------
+def gradient_partial(W1, W2, W3, K, V, eta):
+    """All heads' gradient partial of the given tokens, [H, 3, hidden*d]."""
+    H = np.shape(W1)[0]
+    Kh, Vh = _split_heads(K, H), _split_heads(V, H)
+    eta = _f64(eta).reshape(-1, H)
+    out = []
+    for h in range(H):
+        G1, G2, G3 = gradient(W1[h], W2[h], W3[h], Kh[:, h], Vh[:, h], eta[:, h])
+        out.append(np.stack([G1.reshape(-1), G3.reshape(-1), -G2.reshape(-1)]))
+    return np.stack(out)
+
+
+def update_from_partials(W1, W2, W3, partials, renorm_mode=RENORM_ROW, ns_steps=0):
+    """Ŵ from partials [ranks, H, 3, hidden*d] summed in rank order."""
+    P = np.zeros_like(_f64(partials[0]))
+    for r in range(len(partials)):
+        P = P + _f64(partials[r])
+    H, hid, d = np.shape(W1)
+    outs = ([], [], [])
+    for h in range(H):
+        G = (P[h, 0].reshape(hid, d), -P[h, 2].reshape(d, hid), P[h, 1].reshape(hid, d))
+        if ns_steps > 0:
+            G = tuple(newton_schulz(g, ns_steps) for g in G)
+        for i, W in enumerate((W1, W2, W3)):
+            outs[i].append(renorm(W[h], _f64(W[h]) - G[i], renorm_mode))
+    return tuple(np.stack(o) for o in outs)
+
+
+# --------------------------------------------------------------------------
 # Chunked orderings ([survey] part "二、LaCT", "3应用场景"): the sequence is cut
 # into consecutive chunks of b tokens (the last one shorter); per chunk the
 # update U and the apply A run in one of two orders, and U may be skipped on

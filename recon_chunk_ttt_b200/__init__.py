@@ -19,7 +19,8 @@ _EXPORTS = {
     "TTTError", "lib", "RENORM_OFF", "RENORM_ROW", "RENORM_FROB", "PREC_BF16_TC",
     "PREC_FP32_CHECK", "LIB_PATH", "ttt_trace_enable", "ttt_trace_read",
     "ttt_stream_step_static", "MAX_NS_STEPS", "ttt_chunked", "ORDER_UPDATE_THEN_APPLY",
-    "ORDER_APPLY_THEN_UPDATE",
+    "ORDER_APPLY_THEN_UPDATE", "ttt_partial_floats", "ttt_finish_workspace_bytes",
+    "ttt_update_partial", "ttt_update_finish",
 }
 
 

@@ -77,6 +77,16 @@ def lib() -> ctypes.CDLL:
         L.ttt_stream_step.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P, _P,
                                       ctypes.c_size_t, _P]
         L.ttt_stream_step.restype = ctypes.c_int
+        L.ttt_partial_floats.argtypes = [_CFG]
+        L.ttt_partial_floats.restype = ctypes.c_size_t
+        L.ttt_finish_workspace_bytes.argtypes = [_CFG]
+        L.ttt_finish_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_update_partial.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _I64, _P, _P,
+                                         ctypes.c_size_t, _P]
+        L.ttt_update_partial.restype = ctypes.c_int
+        L.ttt_update_finish.argtypes = [_CFG, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]
+        L.ttt_update_finish.restype = ctypes.c_int
         L.ttt_chunked.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
                                   ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
         L.ttt_chunked.restype = ctypes.c_int
@@ -186,6 +196,47 @@ def ttt_stream_step(cfg: ttt_config, W1, W2, W3, shadow, K, V, eta, Q, O=None,
                                  _ptr(K), _ptr(V), _ptr(eta), n, _ptr(Q), m, _ptr(O),
                                  _ptr(workspace), nbytes, _stream(stream)), "ttt_stream_step")
     return O
+
+
+def ttt_partial_floats(cfg: ttt_config) -> int:
+    return int(lib().ttt_partial_floats(ctypes.byref(cfg)))
+
+
+def ttt_finish_workspace_bytes(cfg: ttt_config) -> int:
+    return int(lib().ttt_finish_workspace_bytes(ctypes.byref(cfg)))
+
+
+def ttt_update_partial(cfg: ttt_config, W1, W2, W3, K, V, eta, partial=None, workspace=None,
+                       stream=None):
+    """This rank's gradient partial ([H][3][hidden*d] fp32: g1, g3, -g2)."""
+    n = int(K.shape[0])
+    if partial is None:
+        partial = torch.empty(ttt_partial_floats(cfg), dtype=torch.float32, device=W1.device)
+    if workspace is None:
+        workspace = alloc_workspace(cfg, n, W1.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().ttt_update_partial(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W3), _ptr(K),
+                                    _ptr(V), _ptr(eta), n, _ptr(partial), _ptr(workspace), nbytes,
+                                    _stream(stream)), "ttt_update_partial")
+    return partial
+
+
+def ttt_update_finish(cfg: ttt_config, W1, W2, W3, partials, W1_out=None, W2_out=None,
+                      W3_out=None, shadow=None, workspace=None, stream=None):
+    """Ŵ from the ranks' partials ([ranks, partial_floats], summed in rank
+    order); returns (W1_out, W2_out, W3_out)."""
+    ranks = int(partials.shape[0]) if partials.dim() == 2 else 1
+    outs = [o if o is not None else torch.empty_like(w)
+            for o, w in ((W1_out, W1), (W2_out, W2), (W3_out, W3))]
+    if workspace is None:
+        workspace = torch.empty(max(ttt_finish_workspace_bytes(cfg), 1), dtype=torch.uint8,
+                                device=W1.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().ttt_update_finish(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W3),
+                                   _ptr(partials), ranks, _ptr(outs[0]), _ptr(outs[1]),
+                                   _ptr(outs[2]), _ptr(shadow), _ptr(workspace), nbytes,
+                                   _stream(stream)), "ttt_update_finish")
+    return tuple(outs)
 
 
 ORDER_UPDATE_THEN_APPLY, ORDER_APPLY_THEN_UPDATE = 0, 1  # TTT_ORDER_*

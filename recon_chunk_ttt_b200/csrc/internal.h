@@ -31,9 +31,13 @@ struct SplitPlan {
 // ---- fp32 CUDA-core check mode -------------------------------------------
 SplitPlan f32_split_plan(const Problem& p);
 size_t f32_workspace_bytes(const Problem& p);
+// With partial_out != nullptr the update stops after the token reduction and
+// writes the fixed-order sum of its splits there (layout of one split, below)
+// instead of updating the weights.
 cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const float* W3,
                        const float* K, const float* V, const float* eta, float* W1o, float* W2o,
-                       float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st);
+                       float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st,
+                       float* partial_out = nullptr);
 cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const float* W3,
                       const float* Q, float* O, cudaStream_t st);
 
@@ -55,6 +59,8 @@ cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void*
                            bool tensor_cores, const float* W1, const float* W2, const float* W3,
                            float* W1o, float* W2o, float* W3o, __nv_bfloat16_raw* shadow,
                            float* scratch, cudaStream_t st);
+// out[i] = sum over s = 0..S-1 of partials[s * count + i], in that order.
+cudaError_t sum_splits(int S, size_t count, const float* partials, float* out, cudaStream_t st);
 cudaError_t pack_shadow(int H, int d, int hid, const float* W1, const float* W2,
                         const float* W3, __nv_bfloat16_raw* shadow, cudaStream_t st);
 
@@ -63,7 +69,8 @@ SplitPlan tc_split_plan(const Problem& p);
 size_t tc_workspace_bytes(const Problem& p);
 cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const float* W3,
                       const void* K, const void* V, const float* eta, float* W1o, float* W2o,
-                      float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st);
+                      float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st,
+                      float* partial_out = nullptr);
 cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,
                      cudaStream_t st);
 

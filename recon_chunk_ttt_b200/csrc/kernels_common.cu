@@ -154,6 +154,24 @@ __global__ void pack_shadow_kernel(size_t mat_total, const float* __restrict__ W
   }
 }
 
+// Fixed-order sum of S split partials (fp64 accumulation), four elements per
+// thread so a thread's loads of one split are issued together.
+__global__ void __launch_bounds__(256) sum_splits_kernel(const float* __restrict__ partials, int S,
+                                                         size_t count, float* __restrict__ out) {
+  const size_t q = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) * 4;
+  if (q >= count) return;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int s = 0; s < S; ++s) {
+    const float4 v = *reinterpret_cast<const float4*>(partials + (size_t)s * count + q);
+    acc[0] += v.x;
+    acc[1] += v.y;
+    acc[2] += v.z;
+    acc[3] += v.w;
+  }
+  *reinterpret_cast<float4*>(out + q) =
+      make_float4((float)acc[0], (float)acc[1], (float)acc[2], (float)acc[3]);
+}
+
 }  // namespace
 
 cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const float* W1,
@@ -168,6 +186,14 @@ cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const 
   if (p.renorm == 2)
     frob_scale_kernel<<<p.H * 3, 256, 0, st>>>(p.H, p.d, p.hid, reinterpret_cast<double*>(scratch),
                                               W1o, W2o, W3o, shadow);
+  return cudaGetLastError();
+}
+
+cudaError_t sum_splits(int S, size_t count, const float* partials, float* out, cudaStream_t st) {
+  // count = 3 * H * hidden * d is a multiple of 4 for every supported shape
+  const size_t threads = (count + 3) / 4;
+  TraceScope ts("sum_splits", st);
+  sum_splits_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(partials, S, count, out);
   return cudaGetLastError();
 }
 

@@ -275,7 +275,8 @@ size_t f32_workspace_bytes(const Problem& p) { return f32_main_bytes(p) + ns_wor
 
 cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const float* W3,
                        const float* K, const float* V, const float* eta, float* W1o, float* W2o,
-                       float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st) {
+                       float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st,
+                       float* partial_out) {
   const SplitPlan sp = f32_split_plan(p);
   char* w = static_cast<char*>(ws);
   const size_t inter = (size_t)p.H * p.n * p.hid;
@@ -304,6 +305,8 @@ cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (partial_out != nullptr)
+    return sum_splits(sp.S, (size_t)p.H * 3 * p.hid * p.d, partials, partial_out, st);
   return ns_then_renorm(p, sp.S, partials, static_cast<char*>(ws) + f32_main_bytes(p), false, W1,
                         W2, W3, W1o, W2o, W3o, shadow, scratch, st);
 }

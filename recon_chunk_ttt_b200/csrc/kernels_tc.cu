@@ -934,7 +934,8 @@ int num_sms() {
 template <int D>
 cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, const float* W3,
                            const void* K, const void* V, const float* eta, float* W1o, float* W2o,
-                           float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st) {
+                           float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st,
+                           float* partial_out) {
   const SplitPlan sp = tc_split_plan(p);
   TcWs w = carve(p, ws, sp.S);
   int* err = device_error_ptr();
@@ -1010,6 +1011,8 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   } else {
     cudaMemsetAsync(w.partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * 4, st);
   }
+  if (partial_out != nullptr)
+    return sum_splits(sp.S, (size_t)p.H * 3 * p.hid * p.d, w.partials, partial_out, st);
   return ns_then_renorm(p, sp.S, w.partials, static_cast<char*>(ws) + tc_main_bytes(p), true, W1,
                         W2, W3, W1o, W2o, W3o, shadow, w.scratch, st);
 }
@@ -1086,9 +1089,13 @@ size_t tc_workspace_bytes(const Problem& p) { return tc_main_bytes(p) + ns_works
 
 cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const float* W3,
                       const void* K, const void* V, const float* eta, float* W1o, float* W2o,
-                      float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st) {
-  if (p.d == 256) return tc_update_impl<256>(p, W1, W2, W3, K, V, eta, W1o, W2o, W3o, shadow, ws, st);
-  return tc_update_impl<64>(p, W1, W2, W3, K, V, eta, W1o, W2o, W3o, shadow, ws, st);
+                      float* W3o, __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st,
+                      float* partial_out) {
+  if (p.d == 256)
+    return tc_update_impl<256>(p, W1, W2, W3, K, V, eta, W1o, W2o, W3o, shadow, ws, st,
+                               partial_out);
+  return tc_update_impl<64>(p, W1, W2, W3, K, V, eta, W1o, W2o, W3o, shadow, ws, st,
+                            partial_out);
 }
 
 cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,

@@ -154,6 +154,68 @@ ttt_status ttt_stream_step(const ttt_config* cfg, float* W1, float* W2, float* W
   return ttt_apply(cfg, W1, W2, W3, shadow, Q, m, O, stream);
 }
 
+size_t ttt_partial_floats(const ttt_config* cfg) {
+  if (check_cfg(cfg) != TTT_OK) return 0;
+  return (size_t)3 * cfg->heads * cfg->d * cfg->hidden;
+}
+
+size_t ttt_finish_workspace_bytes(const ttt_config* cfg) {
+  if (check_cfg(cfg) != TTT_OK) return 0;
+  const Problem p = make_problem(cfg, 1);
+  const size_t scratch = ttt::align_up((size_t)p.H * (2 * p.hid + p.d) * 2 * sizeof(double), 1024);
+  return scratch + ttt::ns_workspace_bytes(p);
+}
+
+ttt_status ttt_update_partial(const ttt_config* cfg, const float* W1, const float* W2,
+                              const float* W3, const void* K, const void* V, const float* eta,
+                              int64_t n, float* partial, void* workspace, size_t workspace_bytes,
+                              ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (n < 0 || n > kMaxTokens) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !W2 || !W3 || !partial) return TTT_ERR_INVALID_ARG;
+  if (n > 0 && (!K || !V || !eta)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {W1, W2, W3, K, V, eta, partial, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const Problem p = make_problem(cfg, n);
+  const bool tc = cfg->precision == TTT_PREC_BF16_TC;
+  const size_t need = tc ? ttt::tc_workspace_bytes(p) : ttt::f32_workspace_bytes(p);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!tc)
+    return cuda_status(ttt::f32_update(p, W1, W2, W3, static_cast<const float*>(K),
+                                       static_cast<const float*>(V), eta, nullptr, nullptr,
+                                       nullptr, nullptr, workspace, st, partial));
+  return cuda_status(ttt::tc_update(p, W1, W2, W3, K, V, eta, nullptr, nullptr, nullptr, nullptr,
+                                    workspace, st, partial));
+}
+
+ttt_status ttt_update_finish(const ttt_config* cfg, const float* W1, const float* W2,
+                             const float* W3, const float* partials, int32_t ranks,
+                             float* W1_out, float* W2_out, float* W3_out, void* shadow,
+                             void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (ranks < 1 || ranks > 65536) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !W2 || !W3 || !partials || !W1_out || !W2_out || !W3_out) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {W1, W2, W3, partials, W1_out, W2_out, W3_out, shadow, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const size_t need = ttt_finish_workspace_bytes(cfg);
+  if (workspace == nullptr || workspace_bytes < need) return TTT_ERR_WORKSPACE;
+  // n only gates the Newton-Schulz stage (skipped for an empty update); the
+  // partials carry the tokens.
+  const Problem p = make_problem(cfg, 1);
+  char* ws = static_cast<char*>(workspace);
+  float* scratch = reinterpret_cast<float*>(ws);
+  void* ns_ws = ws + ttt::align_up((size_t)p.H * (2 * p.hid + p.d) * 2 * sizeof(double), 1024);
+  return cuda_status(ttt::ns_then_renorm(p, ranks, partials, ns_ws,
+                                         cfg->precision == TTT_PREC_BF16_TC, W1, W2, W3, W1_out,
+                                         W2_out, W3_out, static_cast<__nv_bfloat16_raw*>(shadow),
+                                         scratch, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, void* shadow,
                        const void* K, const void* V, const float* eta, const void* Q,
                        int64_t n, int64_t chunk, int32_t order, const uint8_t* update_mask,

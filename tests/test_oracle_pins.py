@@ -498,3 +498,28 @@ def test_chunked_swiglu_special_cases():
     Wf, Out = O.ttt_chunked(*W, x.K, x.V, x.eta, x.Q, 49, O.ORDER_UPDATE_THEN_APPLY)
     Ws, Os = O.ttt_stream(*W, x.K, x.V, x.eta, x.Q, 49)
     np.testing.assert_allclose(Out, rtol=1e-13, atol=1e-15, desired=Os)
+
+
+# --------------------------------------------------- token-sharded update
+def test_partials_sum_to_the_full_update():
+    """Any split of the tokens: the shards' partials, summed, give the one-chunk
+    update (Eq. 3 is a sum over tokens); block 2 holds -g2."""
+    x = wl.make_inputs("tiny")
+    W = (x.W1, x.W2, x.W3)
+    full = O.ttt_update(*W, x.K, x.V, x.eta)
+    for cuts in ([0, 108], [0, 40, 108], [0, 1, 2, 57, 108]):
+        parts = [O.gradient_partial(*W, x.K[a:b], x.V[a:b], x.eta[a:b])
+                 for a, b in zip(cuts[:-1], cuts[1:])]
+        got = O.update_from_partials(*W, parts)
+        for g, f in zip(got, full):
+            np.testing.assert_allclose(g, f, rtol=1e-12, atol=1e-14)
+    P = O.gradient_partial(*W, x.K, x.V, x.eta)
+    G1, G2, G3 = O.gradient(x.W1[0], x.W2[0], x.W3[0], x.K, x.V, x.eta[:, 0])
+    np.testing.assert_allclose(P[0, 2].reshape(G2.shape), -G2, rtol=1e-15)
+    # with Newton-Schulz the orthonormalised sum matches the one-chunk path
+    got = O.update_from_partials(*W, [O.gradient_partial(*W, x.K[:50], x.V[:50], x.eta[:50]),
+                                      O.gradient_partial(*W, x.K[50:], x.V[50:], x.eta[50:])],
+                                 ns_steps=5)
+    want = O.ttt_update(*W, x.K, x.V, x.eta, ns_steps=5)
+    for g, f in zip(got, want):
+        np.testing.assert_allclose(g, f, rtol=1e-10, atol=1e-12)
