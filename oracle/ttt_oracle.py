@@ -27,7 +27,7 @@ GPU receives, upcast exactly.  Per head:
   eta    : [n]
 
 Readings taken where the pages are silent or ambiguous (each is also listed in
-the design notes):
+the design notes; the gated output unit's readings sit with gated_output):
   * SiLU(x) = x * sigmoid(x) with the logistic sigmoid (the pages name SiLU
     without defining it).
   * One gradient step (the review says one step; the notes say "one (or a
@@ -262,6 +262,29 @@ def ttt_stream(W1, W2, W3, K, V, eta, Q, frame_tokens, renorm_mode=RENORM_ROW,
         Ws = ttt_update(*Ws, K[s:e], V[s:e], eta[s:e], renorm_mode, ns_steps)
         outs.append(ttt_apply(*Ws, Q[s:e]))
     return Ws, np.concatenate(outs, axis=0)
+
+
+# --------------------------------------------------------------------------
+# Gated output unit ([review] section 2, the last equation of "Feature
+# Backbone"): o = RMSNorm(o') * SiLU(W_g o').  Readings: per head (o' of one
+# head is a d-vector, W_g is d x d, rows = outputs), RMSNorm(x) =
+# x / sqrt(mean(x^2) + eps) with eps = 1e-6 and no learned gain.
+# --------------------------------------------------------------------------
+GATE_EPS = 1e-6
+
+
+def rms_norm(X, eps=GATE_EPS):
+    X = _f64(X)
+    return X / np.sqrt(np.mean(X * X, axis=-1, keepdims=True) + eps)
+
+
+def gated_output(Oprime, Wg, eps=GATE_EPS):
+    """Oprime: [m, H*d]; Wg: [H, d, d].  Returns o for every row and head."""
+    H = np.shape(Wg)[0]
+    X = _split_heads(Oprime, H)
+    out = np.stack([rms_norm(X[:, h], eps) * silu(X[:, h] @ _f64(Wg[h]).T)
+                    for h in range(H)], axis=1)
+    return out.reshape(X.shape[0], -1)
 
 
 # --------------------------------------------------------------------------

@@ -523,3 +523,34 @@ def test_partials_sum_to_the_full_update():
     want = O.ttt_update(*W, x.K, x.V, x.eta, ns_steps=5)
     for g, f in zip(got, want):
         np.testing.assert_allclose(g, f, rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------- gated output unit
+def test_gated_output_against_torch_and_closed_forms():
+    import torch
+    rng = np.random.default_rng(9)
+    m, H, d = 7, 3, 16
+    Op = rng.standard_normal((m, H * d))
+    Wg = rng.standard_normal((H, d, d)) / 4
+    got = O.gated_output(Op, Wg)
+    # library routines: torch's rms_norm, linear and silu, per head
+    X = torch.from_numpy(Op).view(m, H, d)
+    want = torch.stack([torch.nn.functional.rms_norm(X[:, h], (d,), eps=1e-6) *
+                        torch.nn.functional.silu(torch.nn.functional.linear(
+                            X[:, h], torch.from_numpy(Wg[h])))
+                        for h in range(H)], dim=1).reshape(m, -1).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+    # W_g = 0: SiLU(0) = 0 silences the unit
+    assert not np.any(O.gated_output(Op, np.zeros_like(Wg)))
+    # constant o' = c 1 and W_g = a I: o_j = c / sqrt(c^2 + eps) * SiLU(a c)
+    c, a = -0.7, 1.3
+    got = O.gated_output(np.full((1, d), c), a * np.eye(d)[None])
+    silu = a * c / (1.0 + math.exp(-a * c))
+    np.testing.assert_allclose(got, np.full((1, d), c / math.sqrt(c * c + 1e-6) * silu),
+                               rtol=1e-14)
+    # heads do not mix: changing head 1's o' leaves heads 0 and 2
+    Op2 = Op.copy()
+    Op2[:, d:2 * d] += 1.0
+    g2 = O.gated_output(Op2, Wg)
+    np.testing.assert_array_equal(g2[:, :d], O.gated_output(Op, Wg)[:, :d])
+    np.testing.assert_array_equal(g2[:, 2 * d:], O.gated_output(Op, Wg)[:, 2 * d:])
