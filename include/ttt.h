@@ -161,6 +161,22 @@ ttt_status ttt_stream_step(const ttt_config* cfg,
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
 
 /*
+ * Gated output unit (kimjy99 review, section 2 "Feature Backbone", the last
+ * equation): o = RMSNorm(o') ⊙ SiLU(W_g o'), applied per head to the layer
+ * output o' (e.g. ttt_apply's O).  The page does not say whether the unit
+ * spans heads; heads being independent here, it is read per head:
+ *   RMSNorm(x) = x / sqrt(mean_j x_j² + TTT_GATE_EPS)   (no learned gain)
+ *   W_g: [H][d][d], row = output; bf16 (BF16_TC) or float (FP32_CHECK)
+ *   O_prime, O: [m][H*d], the token type of the precision; O may equal
+ *   O_prime (in place).
+ * BF16_TC: W_g o' on the tensor cores (fp32 accumulation), RMS and gate in
+ * fp32, o rounded to bf16.
+ */
+#define TTT_GATE_EPS 1e-6f
+ttt_status ttt_gate(const ttt_config* cfg, const void* Wg, const void* O_prime, int64_t m,
+                    void* O, ttt_stream_t stream);
+
+/*
  * Token-sharded update across ranks (one chunk's tokens split over several
  * GPUs; the pages describe one GPU, this is the data-parallel form of the
  * same sum).  Eq. 3's g is a sum over tokens, so each rank reduces its own

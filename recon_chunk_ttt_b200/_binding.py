@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_stream_step.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P, _P,
                                       ctypes.c_size_t, _P]
         L.ttt_stream_step.restype = ctypes.c_int
+        L.ttt_gate.argtypes = [_CFG, _P, _P, _I64, _P, _P]
+        L.ttt_gate.restype = ctypes.c_int
         L.ttt_partial_floats.argtypes = [_CFG]
         L.ttt_partial_floats.restype = ctypes.c_size_t
         L.ttt_finish_workspace_bytes.argtypes = [_CFG]
@@ -195,6 +197,19 @@ def ttt_stream_step(cfg: ttt_config, W1, W2, W3, shadow, K, V, eta, Q, O=None,
     _check(lib().ttt_stream_step(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W3), _ptr(shadow),
                                  _ptr(K), _ptr(V), _ptr(eta), n, _ptr(Q), m, _ptr(O),
                                  _ptr(workspace), nbytes, _stream(stream)), "ttt_stream_step")
+    return O
+
+
+GATE_EPS = 1e-6  # TTT_GATE_EPS
+
+
+def ttt_gate(cfg: ttt_config, Wg, O_prime, O=None, stream=None):
+    """o = RMSNorm(o') * SiLU(W_g o') per head; O may be O_prime (in place)."""
+    m = int(O_prime.shape[0])
+    if O is None:
+        O = torch.empty_like(O_prime)
+    _check(lib().ttt_gate(ctypes.byref(cfg), _ptr(Wg), _ptr(O_prime), m, _ptr(O),
+                          _stream(stream)), "ttt_gate")
     return O
 
 

@@ -74,6 +74,13 @@ cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const 
 cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,
                      cudaStream_t st);
 
+// ---- gated output unit: o = RMSNorm(o') * SiLU(W_g o') per head ------------
+// p.n = rows.  W_g [H][d][d] (row = output); bf16 (tc) or float (f32).
+cudaError_t tc_gate(const Problem& p, const void* Wg, const void* Oin, void* Oout, float eps,
+                    cudaStream_t st);
+cudaError_t f32_gate(const Problem& p, const float* Wg, const float* Oin, float* Oout, float eps,
+                     cudaStream_t st);
+
 // The per-device error word (defined in kernels_common.cu).
 int* device_error_ptr();                       // device address, nullptr on failure
 cudaError_t read_and_clear_device_error(int* value);

@@ -247,6 +247,47 @@ __global__ void __launch_bounds__(256) f32_apply_kernel(
   }
 }
 
+// Gated output unit, fp32: block (16 rows, head); o' rows staged in shared
+// memory, one thread per output column j computes g_j = W_g[j,:] o' for the
+// 16 rows, the RMS is formed in fp64 per row.
+constexpr int kGR = 16;
+__global__ void __launch_bounds__(256) f32_gate_kernel(const float* __restrict__ Wg,
+                                                       const float* Oin, float* Oout, int64_t m,
+                                                       int H, int d, float eps) {
+  __shared__ float so[kGR][256];
+  __shared__ float inv[kGR];
+  const int head = blockIdx.y;
+  const int64_t r0 = (int64_t)blockIdx.x * kGR;
+  const size_t ld = (size_t)H * d;
+  for (int i = threadIdx.x; i < kGR * d; i += blockDim.x) {
+    const int t = i / d, c = i % d;
+    so[t][c] = r0 + t < m ? Oin[(size_t)(r0 + t) * ld + (size_t)head * d + c] : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x < kGR) {
+    double ss = 0.0;
+    for (int c = 0; c < d; ++c) ss += (double)so[threadIdx.x][c] * so[threadIdx.x][c];
+    inv[threadIdx.x] = (float)(1.0 / sqrt(ss / d + (double)eps));
+  }
+  __syncthreads();
+  const float* W = Wg + (size_t)head * d * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float acc[kGR];
+#pragma unroll
+    for (int t = 0; t < kGR; ++t) acc[t] = 0.f;
+    for (int k = 0; k < d; ++k) {
+      const float w = W[(size_t)j * d + k];
+#pragma unroll
+      for (int t = 0; t < kGR; ++t) acc[t] = fmaf(w, so[t][k], acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < kGR; ++t)
+      if (r0 + t < m)
+        Oout[(size_t)(r0 + t) * ld + (size_t)head * d + j] =
+            so[t][j] * inv[t] * (acc[t] / (1.f + expf(-acc[t])));
+  }
+}
+
 }  // namespace
 
 SplitPlan f32_split_plan(const Problem& p) {
@@ -321,6 +362,15 @@ cudaError_t f32_apply(const Problem& p, const float* W1, const float* W2, const 
   dim3 g((unsigned)((p.n + kQ - 1) / kQ), p.H);
   TraceScope ts("f32_apply", st);
   f32_apply_kernel<<<g, 256, smem, st>>>(Q, W1, W2, W3, p.n, p.H, p.d, p.hid, O);
+  return cudaGetLastError();
+}
+
+cudaError_t f32_gate(const Problem& p, const float* Wg, const float* Oin, float* Oout, float eps,
+                     cudaStream_t st) {
+  if (p.n == 0) return cudaSuccess;
+  dim3 g((unsigned)((p.n + kGR - 1) / kGR), p.H);
+  TraceScope ts("f32_gate", st);
+  f32_gate_kernel<<<g, 256, 0, st>>>(Wg, Oin, Oout, p.n, p.H, p.d, eps);
   return cudaGetLastError();
 }
 

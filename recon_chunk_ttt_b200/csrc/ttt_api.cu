@@ -154,6 +154,25 @@ ttt_status ttt_stream_step(const ttt_config* cfg, float* W1, float* W2, float* W
   return ttt_apply(cfg, W1, W2, W3, shadow, Q, m, O, stream);
 }
 
+ttt_status ttt_gate(const ttt_config* cfg, const void* Wg, const void* O_prime, int64_t m,
+                    void* O, ttt_stream_t stream) {
+  ttt_status s = check_cfg(cfg);
+  if (s != TTT_OK) return s;
+  if (m < 0 || m > kMaxTokens) return TTT_ERR_INVALID_ARG;
+  if (!Wg) return TTT_ERR_INVALID_ARG;
+  if (m > 0 && (!O_prime || !O)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Wg, O_prime, O};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const Problem p = make_problem(cfg, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->precision == TTT_PREC_FP32_CHECK)
+    return cuda_status(ttt::f32_gate(p, static_cast<const float*>(Wg),
+                                     static_cast<const float*>(O_prime), static_cast<float*>(O),
+                                     TTT_GATE_EPS, st));
+  return cuda_status(ttt::tc_gate(p, Wg, O_prime, O, TTT_GATE_EPS, st));
+}
+
 size_t ttt_partial_floats(const ttt_config* cfg) {
   if (check_cfg(cfg) != TTT_OK) return 0;
   return (size_t)3 * cfg->heads * cfg->d * cfg->hidden;
