@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-stream", action="store_true")
     ap.add_argument("--ns-steps", type=int, default=0,
                     help="Newton-Schulz steps on the gradient in the timed step (0: off)")
+    ap.add_argument("--no-gate-probe", action="store_true",
+                    help="skip the gated-output-unit measurement")
     ap.add_argument("--no-ns-probe", action="store_true",
                     help="skip the separate 5-step Newton-Schulz update measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -390,6 +392,9 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     if not args.no_ns_probe:
         line["ns_update"] = ns_probe(R, torch, dev, cfg_ns, K, V, eta, Win[0], Wout[0], shadow,
                                      ws_buf, stream, d, hid, H, pk, rank_max)
+    # -------------------------------------------------- gated output unit
+    if not args.no_gate_probe:
+        line["gate"] = gate_probe(R, torch, dev, cfg, O, H, d, T, stream, pk, rank_max)
     # -------------------------------------------------- streaming (stream256)
     if not args.no_stream:
         line["stream"] = stream_bench(R, torch, dev, rank_max)
@@ -439,6 +444,32 @@ def ns_probe(R, torch, dev, cfg, K, V, eta, Win, Wout, shadow, ws, stream, d, hi
             "stages_ms": {k: tr[k][1] / reps for k in ns_names if k in tr},
             "note": "NS GEMMs issue 3 bf16 MMAs per product (hi/lo operand split); "
                     "achieved counts the algorithmic flops once"}
+
+
+def gate_probe(R, torch, dev, cfg, O, H, d, T, stream, pk, rank_max, reps: int = 5) -> dict:
+    """The gated output unit on the layer's image output (T x H*d bf16, larger
+    than L2), in place, after 2 untimed runs; W_g ~ N(0, 1/d), bf16.
+    Algorithmic bytes per launch: o' read + o written, 4 * T * H * d; flops
+    2 d^2 per row and head (128 flop/B: HBM-bound)."""
+    rng = np.random.default_rng(8)
+    Wg = torch.from_numpy((rng.standard_normal((H, d, d)) / np.sqrt(d)).astype(np.float32))
+    Wg = Wg.to(torch.bfloat16).to(dev)
+    for _ in range(2):
+        R.ttt_gate(cfg, Wg, O, O=O, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        R.ttt_gate(cfg, Wg, O, O=O, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    R.ttt_check_device_error()
+    ms = rank_max(e0.elapsed_time(e1) / reps)
+    by = 4.0 * T * H * d
+    gbs = by / (ms / 1e3) / 1e9
+    return {"ms_per_launch": ms, "rows": T, "achieved_gbs": gbs,
+            "frac_of_hbm": gbs / pk["hbm_gbs"], "tflops": 2.0 * d * d * T * H / (ms / 1e3) / 1e12,
+            "bytes_per_launch": by}
 
 
 def stream_bench(R, torch, dev, rank_max, warm_frames: int = 8) -> dict:
