@@ -1,0 +1,264 @@
+// Gated output unit on the tensor cores (kimjy99 ZipMap review, section 2
+// "Feature Backbone", last equation): o = RMSNorm(o') ⊙ SiLU(W_g o') per head.
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_util.cuh"
+
+namespace ttt {
+namespace {
+
+// ----------------------------------------------------------------------------
+// Gated output unit (ZipMap review, section 2, last equation of "Feature
+// Backbone"): o = RMSNorm(o') ⊙ SiLU(W_g o') per head, RMSNorm(x) =
+// x / sqrt(mean(x²) + eps).  Persistent: CTA b serves head b % H and token
+// tiles b / H, b / H + gridDim / H, ...  W_g of its head ([d out][d in] bf16,
+// K-major) stays in shared memory; o' tiles stream through a 4-slot ring of
+// [128 x 64] chunks; the gate pre-activation W_g o' accumulates in one of two
+// TMEM buffers while the epilogue drains the other.  Two epilogue warps per
+// TMEM lane quadrant split a row's columns: each loads its half of the o'
+// row (global memory, L2-resident: the tile was just loaded) in one batch,
+// the halves' sums of squares meet in shared memory (summed in a fixed
+// order), and o is written in bf16.  o may overwrite o': a half-row is held in
+// registers before any of it is written, and only its own CTA touches it.
+// ----------------------------------------------------------------------------
+template <int D>
+struct GT {
+  static constexpr int NCH = D / CH;
+  static constexpr int WG = D * 128;        // one 64-wide K chunk of W_g: D rows x 128 B
+  static constexpr int NSLOT = 4;
+  static constexpr int SLOT = BM * 128;     // 16 KB: 128 tokens x 64 d
+  static constexpr int OFF_WG = 0;
+  static constexpr int OFF_A = OFF_WG + NCH * WG;
+  static constexpr int OFF_SS = OFF_A + NSLOT * SLOT;  // [2 parity][2 half][BM] floats
+  static constexpr int OFF_BAR = OFF_SS + 2 * 2 * BM * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int EPI_WARPS = 8;       // two per TMEM lane quadrant
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr uint32_t TMEM_COLS = 2 * D <= 128 ? 128 : 2 * D;  // two accumulators
+};
+
+template <int D>
+__global__ void __launch_bounds__(GT<D>::THREADS, 1)
+    gate_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mA,
+                const __nv_bfloat16* Oin, __nv_bfloat16* Oout, int64_t m, int H, float eps,
+                int* err) {
+  using L = GT<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + L::NSLOT;
+  uint64_t* acc_full = empty + L::NSLOT;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* wfull = acc_empty + 2;
+  uint64_t* done = wfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int head = (int)(blockIdx.x % H);
+  const int64_t t0 = blockIdx.x / H, tstride = gridDim.x / H;
+  const int64_t ntiles = (m + BM - 1) / BM;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NSLOT; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], L::EPI_WARPS);
+    }
+    mbar_init(wfull, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&mA);
+    mbar_arrive_expect_tx(wfull, L::NCH * L::WG);
+    for (int c = 0; c < L::NCH; ++c)
+      tma_load_2d(smem + L::OFF_WG + c * L::WG, &mWg, wfull, c * CH, head * D);
+    int slot = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t t = t0; t < ntiles && ok; t += tstride) {
+      for (int c = 0; c < L::NCH; ++c) {
+        if (!mbar_wait(&empty[slot], phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[slot], L::SLOT);
+        tma_load_2d(smem + L::OFF_A + slot * L::SLOT, &mA, &full[slot], head * D + c * CH,
+                    (int)(t * BM));
+        ++issued;
+        if (++slot == L::NSLOT) { slot = 0; phase ^= 1; }
+      }
+    }
+    drain_ring(full, L::NSLOT, issued, err);
+    drain_ring(wfull, 1, 1, err);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(BM, D, false, false);
+    const uint32_t sbase = smem_u32(smem);
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = mbar_wait(wfull, 0, abort_flag, err, kErrWaitFull);
+    tc_fence_after();
+    for (int64_t t = t0, i = 0; t < ntiles && ok; t += tstride, ++i) {
+      const int b = (int)(i & 1);
+      if (!mbar_wait(&acc_empty[b], (uint32_t)((i >> 1) & 1) ^ 1, abort_flag, err,
+                     kErrWaitAccFree))
+        break;
+      tc_fence_after();
+      for (int c = 0; c < L::NCH; ++c) {
+        if (!mbar_wait(&full[slot], phase, abort_flag, err, kErrWaitFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = sbase + L::OFF_A + slot * L::SLOT;
+        const uint32_t w = sbase + L::OFF_WG + c * L::WG;
+#pragma unroll
+        for (int kk = 0; kk < CH / 16; ++kk)
+          umma_bf16(tmem + b * D, sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024),
+                    sdesc_sw128(w + kk * KSTEP_BYTES, 16, 1024), idesc, (c | kk) != 0);
+        umma_commit(&empty[slot]);
+        if (++slot == L::NSLOT) { slot = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      umma_commit(&acc_full[b]);
+    }
+    umma_commit(done);
+    volatile int never = 0;
+    mbar_wait(done, 0, &never, err, kErrWaitFinal);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    constexpr int HALF = D / 2;
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const size_t ld = (size_t)H * D;
+    float* ss_part = reinterpret_cast<float*>(smem + L::OFF_SS);
+    for (int64_t t = t0, i = 0; t < ntiles; t += tstride, ++i) {
+      const int b = (int)(i & 1);
+      const int64_t r = t * BM + row;
+      const bool valid = r < m;
+      const __nv_bfloat16* orow = Oin + (valid ? r : 0) * ld + (size_t)head * D + half * HALF;
+      // this half of the o' row, all loads issued together (before the wait)
+      uint4 ov[HALF / 8];
+#pragma unroll
+      for (int v = 0; v < HALF / 8; ++v)
+        ov[v] = valid ? *reinterpret_cast<const uint4*>(orow + 8 * v) : make_uint4(0, 0, 0, 0);
+      float ss = 0.f;
+#pragma unroll
+      for (int v = 0; v < HALF / 8; ++v) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&ov[v]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+        }
+      }
+      ss_part[((b * 2) + half) * BM + row] = ss;
+      const bool got = mbar_wait(&acc_full[b], (uint32_t)((i >> 1) & 1), abort_flag, err,
+                                 kErrWaitAcc);
+      // the pair meets here: partial sums visible, and a failed wait in either
+      // warp sends both out together
+      if (named_bar_any(1 + q, 64, !got)) break;
+      tc_fence_after();
+      const float tot = ss_part[(b * 2 + 0) * BM + row] + ss_part[(b * 2 + 1) * BM + row];
+      const float inv = rsqrtf(tot / (float)D + eps);
+#pragma unroll
+      for (int g = 0; g < HALF / 32; ++g) {
+        uint32_t acc[32];
+        tmem_ld_32x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * D + half * HALF + 32 * g),
+                      acc);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&ov[(32 * g + e) / 8]);
+          const float2 o = __bfloat1622float2(h2[(e % 8) / 2]);
+          const float g0 = __uint_as_float(acc[e]), g1 = __uint_as_float(acc[e + 1]);
+          pk[e / 2] = pack_bf16x2(o.x * inv * g0 * sigmoid_fast(g0),
+                                  o.y * inv * g1 * sigmoid_fast(g1));
+        }
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(Oout + r * ld + (size_t)head * D + half * HALF +
+                                                32 * g);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t tc_gate_impl(const Problem& p, const __nv_bfloat16* Wg, const void* Oin, void* Oout,
+                         float eps, cudaStream_t st) {
+  if (p.n == 0) return cudaSuccess;
+  int* err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidDevice;
+  CUtensorMap mWg, mA;
+  {
+    const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * D}, str[1] = {(uint64_t)D * 2};
+    const uint32_t box[2] = {CH, (uint32_t)D};
+    if (!make_map(&mWg, Wg, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t ld = (uint64_t)p.H * D;
+    const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
+    const uint32_t box[2] = {CH, BM};
+    if (!make_map(&mA, Oin, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  cudaError_t e = ensure_smem_attr(gate_kernel<D>, GT<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (p.n + BM - 1) / BM;
+  const int per_head = num_sms() / p.H;
+  const int64_t ctas_per_head = tiles < per_head ? tiles : (per_head > 0 ? per_head : 1);
+  const unsigned grid = (unsigned)(ctas_per_head * p.H);
+  {
+    TraceScope ts("tc_gate", st);
+    gate_kernel<D><<<grid, GT<D>::THREADS, GT<D>::SMEM, st>>>(
+        mWg, mA, static_cast<const __nv_bfloat16*>(Oin), static_cast<__nv_bfloat16*>(Oout), p.n,
+        p.H, eps, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t tc_gate(const Problem& p, const void* Wg, const void* Oin, void* Oout, float eps,
+                    cudaStream_t st) {
+  const auto* w = static_cast<const __nv_bfloat16*>(Wg);
+  if (p.d == 256) return tc_gate_impl<256>(p, w, Oin, Oout, eps, st);
+  return tc_gate_impl<64>(p, w, Oin, Oout, eps, st);
+}
+
+}  // namespace ttt
