@@ -18,11 +18,12 @@ namespace {
 // K-major) stays in shared memory; o' tiles stream through a 4-slot ring of
 // [128 x 64] chunks; the gate pre-activation W_g o' accumulates in one of two
 // TMEM buffers while the epilogue drains the other.  Two epilogue warps per
-// TMEM lane quadrant split a row's columns: each loads its half of the o'
-// row (global memory, L2-resident: the tile was just loaded) in one batch,
-// the halves' sums of squares meet in shared memory (summed in a fixed
-// order), and o is written in bf16.  o may overwrite o': a half-row is held in
-// registers before any of it is written, and only its own CTA touches it.
+// TMEM lane quadrant split a row's columns: each copies its half of the o'
+// row out of the ring slots the MMA just consumed (a slot is refilled only
+// after the MMA and all epilogue warps released it), the halves' sums of
+// squares meet in shared memory (summed in a fixed order), and o is written
+// in bf16.  o may overwrite o': o' is read only through TMA, before o of that
+// tile is written, and only its own CTA touches the tile.
 // ----------------------------------------------------------------------------
 template <int D>
 struct GT {
@@ -43,7 +44,7 @@ struct GT {
 template <int D>
 __global__ void __launch_bounds__(GT<D>::THREADS, 1)
     gate_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mA,
-                const __nv_bfloat16* Oin, __nv_bfloat16* Oout, int64_t m, int H, float eps,
+                __nv_bfloat16* Oout, int64_t m, int H, float eps,
                 int* err) {
   using L = GT<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NSLOT; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], 1 + L::EPI_WARPS);  // MMA commit + every epilogue warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -157,12 +158,28 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
       const int b = (int)(i & 1);
       const int64_t r = t * BM + row;
       const bool valid = r < m;
-      const __nv_bfloat16* orow = Oin + (valid ? r : 0) * ld + (size_t)head * D + half * HALF;
-      // this half of the o' row, all loads issued together (before the wait)
+      const bool got = mbar_wait(&acc_full[b], (uint32_t)((i >> 1) & 1), abort_flag, err,
+                                 kErrWaitAcc);
+      // this half of the o' row from the tile's ring slots: chunk c of tile i
+      // sits in slot (i*NCH + c) % NSLOT, 128-byte rows, 16-byte unit u of
+      // row r at unit u ^ (r % 8); the chunk's full barrier (already
+      // complete) makes the TMA data visible to this thread
       uint4 ov[HALF / 8];
 #pragma unroll
-      for (int v = 0; v < HALF / 8; ++v)
-        ov[v] = valid ? *reinterpret_cast<const uint4*>(orow + 8 * v) : make_uint4(0, 0, 0, 0);
+      for (int v = 0; v < HALF / 8; ++v) {
+        const int col = half * HALF + 8 * v;
+        const int c = col / CH, u = (col % CH) / 8;
+        const int64_t cg = i * L::NCH + c;
+        const int slot = (int)(cg % L::NSLOT);
+        if (got && (v == 0 || (col % CH) == 0))
+          mbar_wait(&full[slot], (uint32_t)((cg / L::NSLOT) & 1), abort_flag, err, kErrWaitFull);
+        ov[v] = *reinterpret_cast<const uint4*>(smem + L::OFF_A + slot * L::SLOT + row * 128 +
+                                                ((u ^ (row & 7)) << 4));
+      }
+      // release the tile's slots (this warp's share)
+      __syncwarp();
+      if (lane == 0)
+        for (int c = 0; c < L::NCH; ++c) mbar_arrive(&empty[(int)((i * L::NCH + c) % L::NSLOT)]);
       float ss = 0.f;
 #pragma unroll
       for (int v = 0; v < HALF / 8; ++v) {
@@ -174,8 +191,6 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
         }
       }
       ss_part[((b * 2) + half) * BM + row] = ss;
-      const bool got = mbar_wait(&acc_full[b], (uint32_t)((i >> 1) & 1), abort_flag, err,
-                                 kErrWaitAcc);
       // the pair meets here: partial sums visible, and a failed wait in either
       // warp sends both out together
       if (named_bar_any(1 + q, 64, !got)) break;
@@ -246,7 +261,7 @@ cudaError_t tc_gate_impl(const Problem& p, const __nv_bfloat16* Wg, const void* 
   {
     TraceScope ts("tc_gate", st);
     gate_kernel<D><<<grid, GT<D>::THREADS, GT<D>::SMEM, st>>>(
-        mWg, mA, static_cast<const __nv_bfloat16*>(Oin), static_cast<__nv_bfloat16*>(Oout), p.n,
+        mWg, mA, static_cast<__nv_bfloat16*>(Oout), p.n,
         p.H, eps, err);
   }
   return cudaGetLastError();

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_util.cuh"
 
 namespace ttt {
 namespace {
@@ -100,7 +101,9 @@ __global__ void __launch_bounds__(256) ns_gather_kernel(const float* __restrict_
 // gradient -> zero) and clears the padding rows.
 __global__ void __launch_bounds__(256) ns_scale_kernel(int d, int hid, int Rp, int tiles,
                                                        const double* __restrict__ tile_ss,
-                                                       float* __restrict__ X) {
+                                                       float* __restrict__ X,
+                                                       __nv_bfloat16* __restrict__ Xh,
+                                                       __nv_bfloat16* __restrict__ Xl) {
   __shared__ double inv;
   const int m = blockIdx.y;
   if (threadIdx.x < 32) {
@@ -113,11 +116,16 @@ __global__ void __launch_bounds__(256) ns_scale_kernel(int d, int hid, int Rp, i
   }
   __syncthreads();
   const int rows_per = Rp / gridDim.x;
-  float* Xm = X + (size_t)m * Rp * hid;
+  const size_t mo = (size_t)m * Rp * hid;
   for (int i = threadIdx.x; i < rows_per * hid; i += blockDim.x) {
     const int row = blockIdx.x * rows_per + i / hid, col = i % hid;
-    float* x = Xm + (size_t)row * hid + col;
-    *x = row < d ? (float)((double)*x * inv) : 0.f;
+    const size_t o = mo + (size_t)row * hid + col;
+    const float v = row < d ? (float)((double)X[o] * inv) : 0.f;
+    X[o] = v;
+    // the bf16 pair the tensor-core iteration reads: hi + lo carries ~16 bits
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    Xh[o] = h;
+    Xl[o] = __float2bfloat16_rn(v - __bfloat162float(h));
   }
 }
 
@@ -215,16 +223,22 @@ __global__ void __launch_bounds__(256) ns_f32_gemm_kernel(
 
 // ----------------------------------------------------------------------------
 // Tensor-core iteration.  One cluster of (Rp/128)^2 CTAs per working matrix
-// runs every step; between the three GEMMs of a step the cluster meets at a
-// hardware cluster barrier (release/acquire), and operands travel through
-// global memory (L2-resident, read with .cg loads).  Per CTA (rank r,
-// mi = r / RB, ni = r % RB, RB = Rp / 128):
-//   A  = X X^T        tile rows mi*128, cols ni*128  (K = hidden, B K-major)
-//   B  = b A + c A A  same tile                      (K = Rp, A symmetric)
-//   X' = a X + B X    rows mi*128, cols ni*N3        (K = Rp, X as MN-major B)
-// Operands are staged per 64-deep k chunk, fp32 -> (hi, lo) bf16, in the
-// 128-byte swizzled layouts the MMA descriptors expect; two stages, the fill
-// of one overlapping the MMAs of the other.
+// runs every step.  Each GEMM's epilogue writes its result in fp32 (where a
+// later epilogue needs it) and as a bf16 pair hi = bf16(x), lo = bf16(x - hi);
+// the next GEMM's operands are those pairs, loaded by TMA (128-byte swizzle)
+// into a two-stage ring, and each product is hi*hi + hi*lo + lo*hi with fp32
+// accumulation in TMEM.  Per CTA (cluster rank r, mi = r / RB, ni = r % RB,
+// RB = Rp / 128):
+//   phase 0  A  = X X^T        tile rows mi*128, cols ni*128  (K = hidden)
+//   phase 1  B  = b A + c A A  same tile                      (K = Rp; A is
+//                              symmetric, so rows of A serve as B operand)
+//   phase 2  X' = a X + B X    rows mi*128, cols ni*N3        (K = Rp, X as
+//                              MN-major B operand)
+// The cluster meets at a hardware barrier (release/acquire) after every
+// phase; the epilogues' generic stores are fenced against the next phase's
+// TMA loads on both sides of that barrier.  Warps: 0 TMA producer (one
+// thread), 1 MMA issuer (one thread), 2..9 epilogue (two per TMEM lane
+// quadrant, each half of the tile's columns).
 // ----------------------------------------------------------------------------
 template <int RP, int C>
 struct NSL {
@@ -238,9 +252,25 @@ struct NSL {
   static constexpr int OFF_BAR = NST * STAGE;
   static constexpr int SMEM = OFF_BAR + 64 + 1024;  // + alignment slack
   static constexpr int TMEM = N3 <= 128 ? 128 : 256;
-  static constexpr int THREADS = 256;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(N3 % 64 == 0 && N3 <= 256, "X' tile width");
   static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// Tensor maps of the iterates (bf16, 128-byte swizzle, 64-element inner box).
+struct NsMaps {
+  CUtensorMap xh[2], xl[2];    // X hi / lo, K-major view: box {64 k, 128 rows}
+  CUtensorMap xhm[2], xlm[2];  // X hi / lo, MN-major view: box {64 cols, 64 k rows,
+                               // N3/64 column blocks}, landing as [block][row][128 B]
+  CUtensorMap ah, al, bh, bl;  // A, B hi / lo, K-major: box {64 k, 128 rows}
+};
+// Global buffers of all matrices (matrix m at m * Rp * C or m * Rp * Rp).
+struct NsBufs {
+  float* xf[2];
+  __nv_bfloat16 *xh[2], *xl[2];
+  float* af;
+  __nv_bfloat16 *ah, *al, *bh, *bl;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -255,174 +285,8 @@ __device__ __forceinline__ void cluster_barrier() {
       "barrier.cluster.arrive.release.aligned;\n\t"
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-
-// 8 fp32 -> 8 bf16 (hi) and 8 bf16 of the remainders (lo), 16 B each.
-__device__ __forceinline__ void split_store(uint8_t* hi, uint8_t* lo, uint32_t off, float4 x0,
-                                            float4 x1) {
-  const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat16 a = __float2bfloat16_rn(v[2 * i]);
-    const __nv_bfloat16 b = __float2bfloat16_rn(v[2 * i + 1]);
-    h[i] = pack_bf16x2(__bfloat162float(a), __bfloat162float(b));
-    l[i] = pack_bf16x2(v[2 * i] - __bfloat162float(a), v[2 * i + 1] - __bfloat162float(b));
-  }
-  *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
-  *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-// K-major tile: 128 rows (r0..) x 64 k (k0..) of a row-major fp32 matrix.
-// Row r holds 128 bytes; its 16-byte unit u sits at unit u ^ (r & 7).  The
-// 1024 units (8 floats each) are split 4 per thread; all loads are issued
-// before the first conversion so the L2 round trips overlap.
-struct KTile {
-  float4 v[4][2];
-};
-__device__ __forceinline__ void load_kmajor(KTile& t, const float* M, int ld, int r0, int k0) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int u = threadIdx.x + 256 * i;
-    const int row = u >> 3, cu = u & 7;
-    const float4* src = reinterpret_cast<const float4*>(M + (size_t)(r0 + row) * ld + k0 + cu * 8);
-    t.v[i][0] = __ldcg(src);
-    t.v[i][1] = __ldcg(src + 1);
-  }
-}
-__device__ __forceinline__ void store_kmajor(const KTile& t, uint8_t* hi, uint8_t* lo) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int u = threadIdx.x + 256 * i;
-    const int row = u >> 3, cu = u & 7;
-    split_store(hi, lo, row * 128 + ((cu ^ (row & 7)) << 4), t.v[i][0], t.v[i][1]);
-  }
-}
-
-// MN-major tile: 64 k rows (k0..) x N columns (n0..) of a row-major fp32
-// matrix.  Column block nb of 64 sits at nb * 8192; inside it k row k holds
-// 128 bytes with unit u at u ^ (k & 7).  64 * N / 8 units, N / 32 per thread.
-template <int N>
-struct MTile {
-  float4 v[N / 32][2];
-};
-template <int N>
-__device__ __forceinline__ void load_mnmajor(MTile<N>& t, const float* M, int ld, int k0, int n0) {
-  constexpr int UPR = N / 8;  // 16-byte units per k row
-#pragma unroll
-  for (int i = 0; i < N / 32; ++i) {
-    const int u = threadIdx.x + 256 * i;
-    const int k = u / UPR, cn = u % UPR;
-    const float4* src = reinterpret_cast<const float4*>(M + (size_t)(k0 + k) * ld + n0 + cn * 8);
-    t.v[i][0] = __ldcg(src);
-    t.v[i][1] = __ldcg(src + 1);
-  }
-}
-template <int N>
-__device__ __forceinline__ void store_mnmajor(const MTile<N>& t, uint8_t* hi, uint8_t* lo) {
-  constexpr int UPR = N / 8;
-#pragma unroll
-  for (int i = 0; i < N / 32; ++i) {
-    const int u = threadIdx.x + 256 * i;
-    const int k = u / UPR, cn = u % UPR;
-    const int nb = cn >> 3, cu = cn & 7;
-    split_store(hi, lo, nb * 8192 + k * 128 + ((cu ^ (k & 7)) << 4), t.v[i][0], t.v[i][1]);
-  }
-}
-
-// acc[TMEM cols 0..N) = A-op (rows a_r0 of Am, K-major) x B-op over `nchunks`
-// k chunks of 64.  B-op: rows b_off of Bm (K-major, N = 128) or, when B_MN,
-// columns b_off.. of Bm (MN-major).  gchunk counts chunks over the kernel
-// (stage = gchunk & 1, use = gchunk >> 1).  Returns with the MMAs in flight;
-// the epilogue waits for them.
-template <int N, bool B_MN, class L>
-__device__ __forceinline__ void ns_gemm(uint8_t* smem, uint64_t* bars, uint32_t tmem, int& gchunk,
-                                        int nchunks, const float* Am, int lda, int a_r0,
-                                        const float* Bm, int ldb, int b_off,
-                                        volatile int* abort, int* err) {
-  const uint32_t idesc = idesc_bf16_f32(128, N, false, B_MN);
-  for (int j = 0; j < nchunks; ++j, ++gchunk) {
-    const int s = gchunk & 1;
-    uint8_t* st = smem + s * L::STAGE;
-    uint8_t* bst = st + 2 * L::A_T;
-    // loads first (registers only), then wait for the stage's previous MMAs
-    KTile ta;
-    load_kmajor(ta, Am, lda, a_r0, j * 64);
-    if constexpr (B_MN) {
-      MTile<N> tb;
-      load_mnmajor<N>(tb, Bm, ldb, j * 64, b_off);
-      if (gchunk >= 2) mbar_wait(&bars[s], ((gchunk >> 1) - 1) & 1, abort, err, kErrWaitEmpty);
-      store_kmajor(ta, st, st + L::A_T);
-      store_mnmajor<N>(tb, bst, bst + L::B_T);
-    } else {
-      KTile tb;
-      load_kmajor(tb, Bm, ldb, b_off, j * 64);
-      if (gchunk >= 2) mbar_wait(&bars[s], ((gchunk >> 1) - 1) & 1, abort, err, kErrWaitEmpty);
-      store_kmajor(ta, st, st + L::A_T);
-      store_kmajor(tb, bst, bst + L::B_T);
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      const uint32_t a = smem_u32(st), b = smem_u32(bst);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ah = sdesc_sw128(a + kk * 32, 16, 1024);
-        const uint64_t al = sdesc_sw128(a + L::A_T + kk * 32, 16, 1024);
-        const uint64_t bh = B_MN ? sdesc_sw128(b + kk * 2048, 8192, 1024)
-                                 : sdesc_sw128(b + kk * 32, 16, 1024);
-        const uint64_t bl = B_MN ? sdesc_sw128(b + L::B_T + kk * 2048, 8192, 1024)
-                                 : sdesc_sw128(b + L::B_T + kk * 32, 16, 1024);
-        umma_bf16(tmem, ah, bh, idesc, (j | kk) != 0);
-        umma_bf16(tmem, ah, bl, idesc, 1);
-        umma_bf16(tmem, al, bh, idesc, 1);
-      }
-      umma_commit(&bars[s]);
-    }
-  }
-}
-
-// Epilogue of one 128 x N tile: warp w reads TMEM lanes 32*(w%4).. (its rows)
-// and half (w/4) of the columns.  MODE 0: O = acc; 1: O = b R + c acc;
-// 2: O = a R + acc.  R has O's pitch and position.  R is read before the
-// wait for the MMAs (chunk `last`), so its round trip overlaps them.
-template <int N, int MODE>
-__device__ __forceinline__ void ns_epilogue(uint64_t* bars, int last, uint32_t tmem, float* O,
-                                            const float* R, int ld, int r0, int c0,
-                                            volatile int* abort, int* err) {
-  constexpr int HALF = N / 2;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp & 3, half = warp >> 2;
-  const size_t base = (size_t)(r0 + 32 * q + lane) * ld + c0 + half * HALF;
-  float4 rv[MODE != 0 ? HALF / 4 : 1];
-  if constexpr (MODE != 0) {
-#pragma unroll
-    for (int i = 0; i < HALF / 4; ++i) rv[i] = __ldcg(reinterpret_cast<const float4*>(R + base) + i);
-  }
-  mbar_wait(&bars[last & 1], (last >> 1) & 1, abort, err, kErrWaitAcc);
-  tc_fence_after();
-#pragma unroll
-  for (int j = 0; j < HALF / 32; ++j) {
-    uint32_t v[32];
-    tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HALF + 32 * j), v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      float4 x = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                             __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-      if constexpr (MODE == 1) {
-        const float4 y = rv[(32 * j + i) / 4];
-        x = make_float4(fmaf(kNsC, x.x, kNsB * y.x), fmaf(kNsC, x.y, kNsB * y.y),
-                        fmaf(kNsC, x.z, kNsB * y.z), fmaf(kNsC, x.w, kNsB * y.w));
-      } else if constexpr (MODE == 2) {
-        const float4 y = rv[(32 * j + i) / 4];
-        x = make_float4(fmaf(kNsA, y.x, x.x), fmaf(kNsA, y.y, x.y), fmaf(kNsA, y.z, x.z),
-                        fmaf(kNsA, y.w, x.w));
-      }
-      __stcg(reinterpret_cast<float4*>(O + base + 32 * j + i), x);
-    }
-  }
-  tc_fence_before();
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 template <int CL>
@@ -433,30 +297,106 @@ __device__ __forceinline__ void ns_sync() {
     __syncthreads();
 }
 
+// Epilogue of one 128 x N tile at (r0, c0) of a matrix with pitch ld: warp w
+// reads TMEM lanes 32*(w%4).. (its rows) and half (w-2)/4 of the columns, in
+// rounds of up to 64 columns; R (MODE != 0) is read before the accumulator
+// wait of the first round.  MODE 0: x = acc (A: fp32 + hi/lo); MODE 1:
+// x = b R + c acc (B: hi/lo only); MODE 2: x = a R + acc (X': fp32 + hi/lo).
+template <int N, int MODE>
+__device__ __forceinline__ void ns_epilogue(uint64_t* acc_full, uint32_t parity, uint32_t tmem,
+                                            const float* R, float* of, __nv_bfloat16* oh,
+                                            __nv_bfloat16* ol, int ld, int r0, int c0,
+                                            volatile int* abort, int* err) {
+  constexpr int HALF = N / 2;
+  constexpr int RND = HALF < 64 ? HALF : 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, half = (warp - 2) >> 2;
+  const size_t row = (size_t)(r0 + 32 * q + lane) * ld + c0 + half * HALF;
+#pragma unroll 1
+  for (int rd = 0; rd < HALF / RND; ++rd) {
+    float4 rv[MODE != 0 ? RND / 4 : 1];
+    if constexpr (MODE != 0) {
+#pragma unroll
+      for (int i = 0; i < RND / 4; ++i)
+        rv[i] = __ldcg(reinterpret_cast<const float4*>(R + row + rd * RND) + i);
+    }
+    if (rd == 0) {
+      mbar_wait(acc_full, parity, abort, err, kErrWaitAcc);
+      tc_fence_after();
+    }
+#pragma unroll
+    for (int j = 0; j < RND / 32; ++j) {
+      const int col = rd * RND + 32 * j;
+      uint32_t v[32];
+      tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HALF + col), v);
+      tmem_ld_wait();
+      float x[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float acc = __uint_as_float(v[e]);
+        if constexpr (MODE == 0) {
+          x[e] = acc;
+        } else {
+          const float4 y4 = rv[(32 * j + e) / 4];
+          const float y = (e & 3) == 0 ? y4.x : (e & 3) == 1 ? y4.y : (e & 3) == 2 ? y4.z : y4.w;
+          x[e] = MODE == 1 ? fmaf(kNsC, acc, kNsB * y) : fmaf(kNsA, y, acc);
+        }
+      }
+      if constexpr (MODE != 1) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          __stcg(reinterpret_cast<float4*>(of + row + col + e),
+                 make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]));
+      }
+      uint32_t h[16], l[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const __nv_bfloat16 a0 = __float2bfloat16_rn(x[e]), a1 = __float2bfloat16_rn(x[e + 1]);
+        h[e / 2] = pack_bf16x2(__bfloat162float(a0), __bfloat162float(a1));
+        l[e / 2] = pack_bf16x2(x[e] - __bfloat162float(a0), x[e + 1] - __bfloat162float(a1));
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __stcg(reinterpret_cast<uint4*>(oh + row + col) + e,
+               make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]));
+        __stcg(reinterpret_cast<uint4*>(ol + row + col) + e,
+               make_uint4(l[4 * e], l[4 * e + 1], l[4 * e + 2], l[4 * e + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  fence_proxy_async_global();
+}
+
 template <int RP, int C>
-__global__ void __launch_bounds__(256, 1) ns_tc_kernel(float* X0, float* X1, float* Abuf,
-                                                       float* Bbuf, int steps, int* err) {
+__global__ void __launch_bounds__(NSL<RP, C>::THREADS, 1)
+    ns_tc_kernel(const __grid_constant__ NsMaps maps, const NsBufs buf, int steps, int* err) {
   using L = NSL<RP, C>;
   extern __shared__ uint8_t ns_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ns_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint8_t* smem = align1024(ns_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + 2;
+  uint64_t* acc_full = empty + 2;
+  uint64_t* done = acc_full + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = L::CL > 1 ? (int)cluster_rank() : 0;
   const int m = blockIdx.x / L::CL;
   const int mi = rank / L::RB, ni = rank % L::RB;
-  float* Xa = X0 + (size_t)m * RP * C;
-  float* Xb = X1 + (size_t)m * RP * C;
-  float* A = Abuf + (size_t)m * RP * RP;
-  float* B = Bbuf + (size_t)m * RP * RP;
+  const int mrow = m * RP;  // first row of this matrix in the stacked views
+  const size_t xo = (size_t)m * RP * C, ao = (size_t)m * RP * RP;
   if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < 32) {
+  if (warp == 1) {
     tmem_alloc(tslot, L::TMEM);
     tmem_relinquish();
   }
@@ -464,52 +404,138 @@ __global__ void __launch_bounds__(256, 1) ns_tc_kernel(float* X0, float* X1, flo
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  int g = 0;
+  int g = 0;   // k chunks so far: ring slot g & 1, its (g >> 1)-th use
+  int ph = 0;  // phases so far: parity of acc_full
   for (int it = 0; it < steps; ++it) {
-    const float* Xc = (it & 1) ? Xb : Xa;
-    float* Xn = (it & 1) ? Xa : Xb;
-    ns_gemm<128, false, L>(smem, bars, tmem, g, C / 64, Xc, C, mi * 128, Xc, C, ni * 128,
-                           abort_flag, err);
-    ns_epilogue<128, 0>(bars, g - 1, tmem, A, nullptr, RP, mi * 128, ni * 128, abort_flag, err);
-    ns_sync<L::CL>();
-    ns_gemm<128, false, L>(smem, bars, tmem, g, RP / 64, A, RP, mi * 128, A, RP, ni * 128,
-                           abort_flag, err);
-    ns_epilogue<128, 1>(bars, g - 1, tmem, B, A, RP, mi * 128, ni * 128, abort_flag, err);
-    ns_sync<L::CL>();
-    ns_gemm<L::N3, true, L>(smem, bars, tmem, g, RP / 64, B, RP, mi * 128, Xc, C, ni * L::N3,
-                            abort_flag, err);
-    ns_epilogue<L::N3, 2>(bars, g - 1, tmem, Xn, Xc, C, mi * 128, ni * L::N3, abort_flag, err);
-    ns_sync<L::CL>();
+    const int cur = it & 1, nxt = cur ^ 1;
+    for (int p = 0; p < 3; ++p, ++ph) {
+      const int nchunks = p == 0 ? C / 64 : RP / 64;
+      if (warp == 0) {
+        if (lane == 0) {
+          // ------------------------------------------------ TMA producer
+          fence_proxy_async_global();
+          for (int j = 0; j < nchunks; ++j) {
+            const int gj = g + j, s = gj & 1;
+            if (gj >= 2) mbar_wait(&empty[s], ((gj >> 1) - 1) & 1, abort_flag, err, kErrWaitEmpty);
+            uint8_t* st = smem + s * L::STAGE;
+            uint8_t* bst = st + 2 * L::A_T;
+            const int k0 = j * 64;
+            if (p == 0) {
+              mbar_arrive_expect_tx(&full[s], 4 * L::A_T);
+              tma_load_2d(st, &maps.xh[cur], &full[s], k0, mrow + mi * 128);
+              tma_load_2d(st + L::A_T, &maps.xl[cur], &full[s], k0, mrow + mi * 128);
+              tma_load_2d(bst, &maps.xh[cur], &full[s], k0, mrow + ni * 128);
+              tma_load_2d(bst + L::B_T, &maps.xl[cur], &full[s], k0, mrow + ni * 128);
+            } else if (p == 1) {
+              mbar_arrive_expect_tx(&full[s], 4 * L::A_T);
+              tma_load_2d(st, &maps.ah, &full[s], k0, mrow + mi * 128);
+              tma_load_2d(st + L::A_T, &maps.al, &full[s], k0, mrow + mi * 128);
+              tma_load_2d(bst, &maps.ah, &full[s], k0, mrow + ni * 128);
+              tma_load_2d(bst + L::B_T, &maps.al, &full[s], k0, mrow + ni * 128);
+            } else {
+              mbar_arrive_expect_tx(&full[s], 2 * L::A_T + 2 * L::B_T);
+              tma_load_2d(st, &maps.bh, &full[s], k0, mrow + mi * 128);
+              tma_load_2d(st + L::A_T, &maps.bl, &full[s], k0, mrow + mi * 128);
+              tma_load_3d(bst, &maps.xhm[cur], &full[s], 0, mrow + k0, ni * (L::N3 / 64));
+              tma_load_3d(bst + L::B_T, &maps.xlm[cur], &full[s], 0, mrow + k0, ni * (L::N3 / 64));
+            }
+          }
+        }
+      } else if (warp == 1) {
+        if (lane == 0) {
+          // ------------------------------------------------ MMA issuer
+          const uint32_t idesc = p == 2 ? idesc_bf16_f32(128, L::N3, false, true)
+                                        : idesc_bf16_f32(128, 128, false, false);
+          for (int j = 0; j < nchunks; ++j) {
+            const int gj = g + j, s = gj & 1;
+            mbar_wait(&full[s], (gj >> 1) & 1, abort_flag, err, kErrWaitFull);
+            tc_fence_after();
+            const uint32_t a = smem_u32(smem + s * L::STAGE), b = a + 2 * L::A_T;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ah = sdesc_sw128(a + kk * 32, 16, 1024);
+              const uint64_t al = sdesc_sw128(a + L::A_T + kk * 32, 16, 1024);
+              const uint64_t bh = p == 2 ? sdesc_sw128(b + kk * 2048, 8192, 1024)
+                                         : sdesc_sw128(b + kk * 32, 16, 1024);
+              const uint64_t bl = p == 2 ? sdesc_sw128(b + L::B_T + kk * 2048, 8192, 1024)
+                                         : sdesc_sw128(b + L::B_T + kk * 32, 16, 1024);
+              umma_bf16(tmem, ah, bh, idesc, (j | kk) != 0);
+              umma_bf16(tmem, ah, bl, idesc, 1);
+              umma_bf16(tmem, al, bh, idesc, 1);
+            }
+            umma_commit(&empty[s]);
+          }
+          umma_commit(acc_full);
+        }
+      } else {
+        // ------------------------------------------------ epilogue
+        const uint32_t par = (uint32_t)(ph & 1);
+        if (p == 0)
+          ns_epilogue<128, 0>(acc_full, par, tmem, nullptr, buf.af + ao, buf.ah + ao, buf.al + ao,
+                              RP, mi * 128, ni * 128, abort_flag, err);
+        else if (p == 1)
+          ns_epilogue<128, 1>(acc_full, par, tmem, buf.af + ao, nullptr, buf.bh + ao,
+                              buf.bl + ao, RP, mi * 128, ni * 128, abort_flag, err);
+        else
+          ns_epilogue<L::N3, 2>(acc_full, par, tmem, buf.xf[cur] + xo, buf.xf[nxt] + xo,
+                                buf.xh[nxt] + xo, buf.xl[nxt] + xo, C, mi * 128, ni * L::N3,
+                                abort_flag, err);
+      }
+      g += nchunks;
+      __syncwarp();
+      ns_sync<L::CL>();
+    }
+  }
+  if (warp == 0 && lane == 0) drain_ring(full, 2, g, err);
+  if (warp == 1 && lane == 0) {
+    umma_commit(done);
+    volatile int never = 0;
+    mbar_wait(done, 0, &never, err, kErrWaitFinal);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x < 32) {
+  if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, L::TMEM);
   }
 }
 
 struct NsWs {
-  float *X0, *X1, *A, *B, *delta;
+  float *X[2], *A, *B, *delta;     // fp32 iterates and products (B: check mode)
+  __nv_bfloat16 *Xh[2], *Xl[2], *Ah, *Al, *Bh, *Bl;  // bf16 pairs (tensor cores)
   double* tile_ss;
 };
 
 NsWs ns_carve(const Problem& p, void* ws) {
   const int Rp = ns_rows(p.d);
   const size_t M = 3 * (size_t)p.H;
+  const size_t xs = M * Rp * p.hid, as = M * Rp * Rp;
   char* c = static_cast<char*>(ws);
   NsWs w;
-  w.X0 = reinterpret_cast<float*>(c);
-  c += align_up(M * Rp * p.hid * 4, 1024);
-  w.X1 = reinterpret_cast<float*>(c);
-  c += align_up(M * Rp * p.hid * 4, 1024);
-  w.A = reinterpret_cast<float*>(c);
-  c += align_up(M * Rp * Rp * 4, 1024);
-  w.B = reinterpret_cast<float*>(c);
-  c += align_up(M * Rp * Rp * 4, 1024);
-  w.delta = reinterpret_cast<float*>(c);
-  c += align_up(M * p.hid * p.d * 4, 1024);
+  auto f32 = [&](size_t n) {
+    float* r = reinterpret_cast<float*>(c);
+    c += align_up(n * 4, 1024);
+    return r;
+  };
+  auto b16 = [&](size_t n) {
+    __nv_bfloat16* r = reinterpret_cast<__nv_bfloat16*>(c);
+    c += align_up(n * 2, 1024);
+    return r;
+  };
+  w.X[0] = f32(xs);
+  w.X[1] = f32(xs);
+  w.A = f32(as);
+  w.B = f32(as);
+  w.delta = f32(M * p.hid * p.d);
+  w.Xh[0] = b16(xs);
+  w.Xh[1] = b16(xs);
+  w.Xl[0] = b16(xs);
+  w.Xl[1] = b16(xs);
+  w.Ah = b16(as);
+  w.Al = b16(as);
+  w.Bh = b16(as);
+  w.Bl = b16(as);
   w.tile_ss = reinterpret_cast<double*>(c);
   return w;
 }
@@ -517,6 +543,37 @@ NsWs ns_carve(const Problem& p, void* ws) {
 template <int RP, int C>
 cudaError_t launch_ns_tc(const Problem& p, const NsWs& w, int* err, cudaStream_t st) {
   using L = NSL<RP, C>;
+  const uint64_t rows = (uint64_t)3 * p.H * RP;  // all matrices stacked
+  NsMaps maps;
+  for (int b = 0; b < 2; ++b) {
+    const uint64_t dk[2] = {(uint64_t)C, rows}, sk[1] = {(uint64_t)C * 2};
+    const uint32_t bk[2] = {64, 128};
+    const uint64_t dm[3] = {64, rows, (uint64_t)C / 64}, sm[2] = {(uint64_t)C * 2, 128};
+    const uint32_t bm[3] = {64, 64, (uint32_t)(L::N3 / 64)};
+    if (!make_map(&maps.xh[b], w.Xh[b], 2, dk, sk, bk) ||
+        !make_map(&maps.xl[b], w.Xl[b], 2, dk, sk, bk) ||
+        !make_map(&maps.xhm[b], w.Xh[b], 3, dm, sm, bm) ||
+        !make_map(&maps.xlm[b], w.Xl[b], 3, dm, sm, bm))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t da[2] = {(uint64_t)RP, rows}, sa[1] = {(uint64_t)RP * 2};
+    const uint32_t ba[2] = {64, 128};
+    if (!make_map(&maps.ah, w.Ah, 2, da, sa, ba) || !make_map(&maps.al, w.Al, 2, da, sa, ba) ||
+        !make_map(&maps.bh, w.Bh, 2, da, sa, ba) || !make_map(&maps.bl, w.Bl, 2, da, sa, ba))
+      return cudaErrorInvalidValue;
+  }
+  NsBufs buf;
+  for (int b = 0; b < 2; ++b) {
+    buf.xf[b] = w.X[b];
+    buf.xh[b] = w.Xh[b];
+    buf.xl[b] = w.Xl[b];
+  }
+  buf.af = w.A;
+  buf.ah = w.Ah;
+  buf.al = w.Al;
+  buf.bh = w.Bh;
+  buf.bl = w.Bl;
   cudaError_t e = ensure_smem_attr(ns_tc_kernel<RP, C>, L::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -532,7 +589,7 @@ cudaError_t launch_ns_tc(const Problem& p, const NsWs& w, int* err, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = L::CL > 1 ? 1 : 0;
   TraceScope ts("ns_tc_iterate", st);
-  return cudaLaunchKernelEx(&cfg, ns_tc_kernel<RP, C>, w.X0, w.X1, w.A, w.B, p.ns_steps, err);
+  return cudaLaunchKernelEx(&cfg, ns_tc_kernel<RP, C>, maps, buf, p.ns_steps, err);
 }
 
 }  // namespace
@@ -542,8 +599,10 @@ size_t ns_workspace_bytes(const Problem& p) {
   const int Rp = ns_rows(p.d);
   const size_t M = 3 * (size_t)p.H;
   const size_t tiles = (size_t)(p.d / 32) * (p.hid / 32);
-  return 2 * align_up(M * Rp * p.hid * 4, 1024) + 2 * align_up(M * Rp * Rp * 4, 1024) +
-         align_up(M * p.hid * p.d * 4, 1024) + align_up(M * tiles * 8, 1024);
+  const size_t xs = M * Rp * p.hid, as = M * Rp * Rp;
+  return 2 * align_up(xs * 4, 1024) + 2 * align_up(as * 4, 1024) +
+         align_up(M * p.hid * p.d * 4, 1024) + 4 * align_up(xs * 2, 1024) +
+         4 * align_up(as * 2, 1024) + align_up(M * tiles * 8, 1024);
 }
 
 cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void* ns_ws,
@@ -558,8 +617,10 @@ cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void*
   const int tiles = (p.d / 32) * (p.hid / 32);
   {
     TraceScope ts("ns_prepare", st);
-    ns_gather_kernel<<<M * tiles, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, Rp, w.X0, w.tile_ss);
-    ns_scale_kernel<<<dim3(Rp / 8, M), 256, 0, st>>>(p.d, p.hid, Rp, tiles, w.tile_ss, w.X0);
+    ns_gather_kernel<<<M * tiles, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, Rp, w.X[0],
+                                                w.tile_ss);
+    ns_scale_kernel<<<dim3(Rp / 8, M), 256, 0, st>>>(p.d, p.hid, Rp, tiles, w.tile_ss, w.X[0],
+                                                     w.Xh[0], w.Xl[0]);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -572,8 +633,8 @@ cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void*
     TraceScope ts("ns_f32_iterate", st);
     const size_t xs = (size_t)Rp * p.hid, as = (size_t)Rp * Rp;
     for (int it = 0; it < p.ns_steps; ++it) {
-      const float* Xc = (it & 1) ? w.X1 : w.X0;
-      float* Xn = (it & 1) ? w.X0 : w.X1;
+      const float* Xc = w.X[it & 1];
+      float* Xn = w.X[(it & 1) ^ 1];
       ns_f32_gemm_kernel<true><<<dim3(Rp / 64, Rp / 64, M), 256, 0, st>>>(
           Xc, Xc, nullptr, w.A, p.hid, p.hid, p.hid, Rp, xs, xs, as, 1.f, 0.f);
       ns_f32_gemm_kernel<false><<<dim3(Rp / 64, Rp / 64, M), 256, 0, st>>>(
@@ -586,7 +647,7 @@ cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void*
   }
   {
     TraceScope ts("ns_finish", st);
-    const float* Xf = (p.ns_steps & 1) ? w.X1 : w.X0;
+    const float* Xf = w.X[p.ns_steps & 1];
     ns_finish_kernel<<<M * tiles, 256, 0, st>>>(Xf, p.H, p.d, p.hid, Rp, w.delta);
   }
   e = cudaGetLastError();
