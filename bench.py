@@ -359,7 +359,7 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
         with open(tp) as f:
             tj = json.load(f)
         ent = tj.get(dom)
-        if ent and ent.get("source_sha") == kernel_source_sha():
+        if ent and ent.get("source_sha") == kernel_source_sha(ent.get("sources")):
             units_per_launch = (T + M) * H / 2 if dom == "tc_apply" else T * H
             roof["traffic"] = ent["bytes_per_unit"] * units_per_launch
     gemm_upd_ms = trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1]
@@ -592,11 +592,13 @@ def e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta, W
             "steps": args.e2e_steps}
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(files=None) -> str:
+    """Hash of the kernel sources (all of csrc/, or the listed files of it)."""
     import hashlib
+    csrc = os.path.join(ROOT, "recon_chunk_ttt_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "recon_chunk_ttt_b200", "csrc"))):
-        with open(os.path.join(ROOT, "recon_chunk_ttt_b200", "csrc", f), "rb") as fh:
+    for f in sorted(files if files else os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 

@@ -251,7 +251,7 @@ struct NSL {
   static constexpr int NST = 2;
   static constexpr int OFF_BAR = NST * STAGE;
   static constexpr int SMEM = OFF_BAR + 64 + 1024;  // + alignment slack
-  static constexpr int TMEM = N3 <= 128 ? 128 : 256;
+  static constexpr int TMEM = 512;  // accumulator, A tile, X tile (see kAR, kXR)
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(N3 % 64 == 0 && N3 <= 256, "X' tile width");
@@ -297,75 +297,96 @@ __device__ __forceinline__ void ns_sync() {
     __syncthreads();
 }
 
-// Epilogue of one 128 x N tile at (r0, c0) of a matrix with pitch ld: warp w
-// reads TMEM lanes 32*(w%4).. (its rows) and half (w-2)/4 of the columns, in
-// rounds of up to 64 columns; R (MODE != 0) is read before the accumulator
-// wait of the first round.  MODE 0: x = acc (A: fp32 + hi/lo); MODE 1:
-// x = b R + c acc (B: hi/lo only); MODE 2: x = a R + acc (X': fp32 + hi/lo).
+// TMEM columns: [0, N) the accumulator; [kAR, kAR + 128) this CTA's A tile
+// in fp32, from phase 0's epilogue to phase 1's (phase 0/1 accumulators use
+// only [0, 128)); [kXR, kXR + N3) this CTA's X tile in fp32, kept across
+// steps (phase 2 reads it and writes X' back).  So no epilogue reads fp32
+// operands from global memory.
+constexpr uint32_t kAR = 128, kXR = 256, kNsTmemCols = 512;
+
+// Epilogue of one 128 x N tile: warp w reads TMEM lanes 32*(w%4).. (its rows)
+// and half (w-2)/4 of the columns.  MODE 0: x = acc, kept in TMEM for phase
+// 1; MODE 1: x = b A + c acc (A from TMEM); MODE 2: x = a X + acc (X from
+// TMEM, x written back; on the last step also stored in fp32 to xf_out).
+// hi/lo of x are staged in the (idle) ring as 128-byte-swizzled [128 x 64]
+// chunks and written with TMA bulk stores through maps mh / ml at column x0,
+// row y0; the stores have completed when the function returns.
 template <int N, int MODE>
 __device__ __forceinline__ void ns_epilogue(uint64_t* acc_full, uint32_t parity, uint32_t tmem,
-                                            const float* R, float* of, __nv_bfloat16* oh,
-                                            __nv_bfloat16* ol, int ld, int r0, int c0,
-                                            volatile int* abort, int* err) {
+                                            uint8_t* stage, const CUtensorMap* mh,
+                                            const CUtensorMap* ml, int x0, int y0,
+                                            float* xf_out, int ldf, volatile int* abort,
+                                            int* err) {
   constexpr int HALF = N / 2;
-  constexpr int RND = HALF < 64 ? HALF : 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, half = (warp - 2) >> 2;
-  const size_t row = (size_t)(r0 + 32 * q + lane) * ld + c0 + half * HALF;
+  const int row = 32 * q + lane;
+  const uint32_t lanes = (uint32_t)(32 * q) << 16;
+  uint8_t* hi = stage;
+  uint8_t* lo = stage + N * 256;  // N/64 chunks of 16 KB
+  mbar_wait(acc_full, parity, abort, err, kErrWaitAcc);
+  tc_fence_after();
 #pragma unroll 1
-  for (int rd = 0; rd < HALF / RND; ++rd) {
-    float4 rv[MODE != 0 ? RND / 4 : 1];
-    if constexpr (MODE != 0) {
+  for (int j = 0; j < HALF / 32; ++j) {
+    const int col = half * HALF + 32 * j;
+    uint32_t v[32];
+    tmem_ld_32x32(tmem + lanes + (uint32_t)col, v);
+    uint32_t rr[32];
+    if constexpr (MODE == 1) tmem_ld_32x32(tmem + lanes + kAR + (uint32_t)col, rr);
+    if constexpr (MODE == 2) tmem_ld_32x32(tmem + lanes + kXR + (uint32_t)col, rr);
+    tmem_ld_wait();
+    uint32_t xb[32];
 #pragma unroll
-      for (int i = 0; i < RND / 4; ++i)
-        rv[i] = __ldcg(reinterpret_cast<const float4*>(R + row + rd * RND) + i);
+    for (int e = 0; e < 32; ++e) {
+      const float acc = __uint_as_float(v[e]);
+      float x = acc;
+      if constexpr (MODE == 1) x = fmaf(kNsC, acc, kNsB * __uint_as_float(rr[e]));
+      if constexpr (MODE == 2) x = fmaf(kNsA, __uint_as_float(rr[e]), acc);
+      xb[e] = __float_as_uint(x);
     }
-    if (rd == 0) {
-      mbar_wait(acc_full, parity, abort, err, kErrWaitAcc);
-      tc_fence_after();
-    }
-#pragma unroll
-    for (int j = 0; j < RND / 32; ++j) {
-      const int col = rd * RND + 32 * j;
-      uint32_t v[32];
-      tmem_ld_32x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HALF + col), v);
-      tmem_ld_wait();
-      float x[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float acc = __uint_as_float(v[e]);
-        if constexpr (MODE == 0) {
-          x[e] = acc;
-        } else {
-          const float4 y4 = rv[(32 * j + e) / 4];
-          const float y = (e & 3) == 0 ? y4.x : (e & 3) == 1 ? y4.y : (e & 3) == 2 ? y4.z : y4.w;
-          x[e] = MODE == 1 ? fmaf(kNsC, acc, kNsB * y) : fmaf(kNsA, y, acc);
-        }
-      }
-      if constexpr (MODE != 1) {
+    if constexpr (MODE == 0) tmem_st_32x32(tmem + lanes + kAR + (uint32_t)col, xb);
+    if constexpr (MODE == 2) {
+      tmem_st_32x32(tmem + lanes + kXR + (uint32_t)col, xb);
+      if (xf_out != nullptr) {
+        float* o = xf_out + (size_t)row * ldf + col;
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
-          __stcg(reinterpret_cast<float4*>(of + row + col + e),
-                 make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]));
-      }
-      uint32_t h[16], l[16];
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const __nv_bfloat16 a0 = __float2bfloat16_rn(x[e]), a1 = __float2bfloat16_rn(x[e + 1]);
-        h[e / 2] = pack_bf16x2(__bfloat162float(a0), __bfloat162float(a1));
-        l[e / 2] = pack_bf16x2(x[e] - __bfloat162float(a0), x[e + 1] - __bfloat162float(a1));
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __stcg(reinterpret_cast<uint4*>(oh + row + col) + e,
-               make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]));
-        __stcg(reinterpret_cast<uint4*>(ol + row + col) + e,
-               make_uint4(l[4 * e], l[4 * e + 1], l[4 * e + 2], l[4 * e + 3]));
+          __stcg(reinterpret_cast<float4*>(o + e),
+                 make_float4(__uint_as_float(xb[e]), __uint_as_float(xb[e + 1]),
+                             __uint_as_float(xb[e + 2]), __uint_as_float(xb[e + 3])));
       }
     }
+    uint32_t h[16], l[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const float x0f = __uint_as_float(xb[e]), x1f = __uint_as_float(xb[e + 1]);
+      const __nv_bfloat16 a0 = __float2bfloat16_rn(x0f), a1 = __float2bfloat16_rn(x1f);
+      h[e / 2] = pack_bf16x2(__bfloat162float(a0), __bfloat162float(a1));
+      l[e / 2] = pack_bf16x2(x0f - __bfloat162float(a0), x1f - __bfloat162float(a1));
+    }
+    // 32 columns = 4 16-byte units of one 64-column chunk
+    const int chunk = col / 64, u0 = (col % 64) / 8;
+    const int base = chunk * 16384 + row * 128;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int off = base + (((u0 + e) ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]);
+      *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[4 * e], l[4 * e + 1], l[4 * e + 2], l[4 * e + 3]);
+    }
   }
+  if constexpr (MODE != 1) tmem_st_wait();
   tc_fence_before();
-  fence_proxy_async_global();
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  named_bar_sync(5, 32 * (NSL<256, 512>::EPI_WARPS));
+  if (warp == 2 && lane == 0) {
+    for (int c = 0; c < N / 64; ++c) {
+      tma_store_2d(mh, hi + c * 16384, x0 + 64 * c, y0);
+      tma_store_2d(ml, lo + c * 16384, x0 + 64 * c, y0);
+    }
+    bulk_commit_group();
+    bulk_wait_group0();
+    fence_proxy_async_global();
+  }
 }
 
 template <int RP, int C>
@@ -404,6 +425,29 @@ __global__ void __launch_bounds__(NSL<RP, C>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  if (warp >= 2) {
+    // this CTA's X tile (rows mi*128.., cols ni*N3..) into TMEM, fp32
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const float* xr = buf.xf[0] + xo + (size_t)(mi * 128 + 32 * q + lane) * C + ni * L::N3;
+#pragma unroll 1
+    for (int j = 0; j < L::N3 / 64; ++j) {
+      const int col = half * (L::N3 / 2) + 32 * j;
+      uint32_t xb[32];
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(xr + col + e));
+        xb[e] = __float_as_uint(f.x);
+        xb[e + 1] = __float_as_uint(f.y);
+        xb[e + 2] = __float_as_uint(f.z);
+        xb[e + 3] = __float_as_uint(f.w);
+      }
+      tmem_st_32x32(tmem + ((uint32_t)(32 * q) << 16) + kXR + (uint32_t)col, xb);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   int g = 0;   // k chunks so far: ring slot g & 1, its (g >> 1)-th use
   int ph = 0;  // phases so far: parity of acc_full
   for (int it = 0; it < steps; ++it) {
@@ -470,16 +514,20 @@ __global__ void __launch_bounds__(NSL<RP, C>::THREADS, 1)
       } else {
         // ------------------------------------------------ epilogue
         const uint32_t par = (uint32_t)(ph & 1);
+        const int y0 = mrow + mi * 128;
         if (p == 0)
-          ns_epilogue<128, 0>(acc_full, par, tmem, nullptr, buf.af + ao, buf.ah + ao, buf.al + ao,
-                              RP, mi * 128, ni * 128, abort_flag, err);
+          ns_epilogue<128, 0>(acc_full, par, tmem, smem, &maps.ah, &maps.al, ni * 128, y0,
+                              nullptr, 0, abort_flag, err);
         else if (p == 1)
-          ns_epilogue<128, 1>(acc_full, par, tmem, buf.af + ao, nullptr, buf.bh + ao,
-                              buf.bl + ao, RP, mi * 128, ni * 128, abort_flag, err);
+          ns_epilogue<128, 1>(acc_full, par, tmem, smem, &maps.bh, &maps.bl, ni * 128, y0,
+                              nullptr, 0, abort_flag, err);
         else
-          ns_epilogue<L::N3, 2>(acc_full, par, tmem, buf.xf[cur] + xo, buf.xf[nxt] + xo,
-                                buf.xh[nxt] + xo, buf.xl[nxt] + xo, C, mi * 128, ni * L::N3,
-                                abort_flag, err);
+          ns_epilogue<L::N3, 2>(acc_full, par, tmem, smem, &maps.xh[nxt], &maps.xl[nxt],
+                                ni * L::N3, y0,
+                                it == steps - 1 ? buf.xf[nxt] + xo + (size_t)mi * 128 * C +
+                                                      ni * L::N3
+                                                : nullptr,
+                                C, abort_flag, err);
       }
       g += nchunks;
       __syncwarp();
