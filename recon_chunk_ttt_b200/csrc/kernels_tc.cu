@@ -988,7 +988,9 @@ SplitPlan tc_split_plan(const Problem& p) {
   const int per = grad_ctas_per_split(p);
   int S = 148 / per;
   if (S < 1) S = 1;
-  const int64_t max_s = (p.n + TK - 1) / TK;
+  // at least 512 tokens per split: below that the fp32 partials (6.3 MB per
+  // split for 4 heads of d 256) cost more than the parallelism gains
+  const int64_t max_s = (p.n + 511) / 512;
   if (S > max_s) S = (int)(max_s < 1 ? 1 : max_s);
   int64_t chunk = (p.n + S - 1) / S;
   chunk = (chunk + TK - 1) / TK * TK;
