@@ -61,15 +61,29 @@ __global__ void __launch_bounds__(256) ns_gather_kernel(const float* __restrict_
   // (coalesced along j).  tile[a][b] holds working element (c0+b, j0+a) for
   // blocks 0/1 and (c0+a, j0+b) for block 2.  Each thread owns 4 elements
   // (rows ty, ty+8, ...) and sums them over s in increasing order.
+  size_t off[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty + 8 * i;
+    off[i] = blk < 2 ? (size_t)(j0 + r) * d + c0 + tx : (size_t)(c0 + r) * hid + j0 + tx;
+  }
+  const size_t sstride = (size_t)H * 3 * mat;
+  const float* P = partials + ((size_t)head * 3 + blk) * mat;
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int s = 0; s < S; ++s) {
-    const float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat;
+  int s = 0;
+  for (; s + 2 <= S; s += 2) {  // two splits' loads in flight, added in split order
+    float a[4], b[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int r = ty + 8 * i;
-      const size_t off = blk < 2 ? (size_t)(j0 + r) * d + c0 + tx : (size_t)(c0 + r) * hid + j0 + tx;
-      acc[i] += (double)P[off];
+      a[i] = P[(size_t)s * sstride + off[i]];
+      b[i] = P[(size_t)(s + 1) * sstride + off[i]];
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = (acc[i] + (double)a[i]) + (double)b[i];
+  }
+  if (s < S) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] += (double)P[(size_t)s * sstride + off[i]];
   }
   double ss = 0.0;
 #pragma unroll
@@ -116,16 +130,29 @@ __global__ void __launch_bounds__(256) ns_scale_kernel(int d, int hid, int Rp, i
   }
   __syncthreads();
   const int rows_per = Rp / gridDim.x;
+  const int q_per_row = hid / 4;  // 4 columns per thread step
   const size_t mo = (size_t)m * Rp * hid;
-  for (int i = threadIdx.x; i < rows_per * hid; i += blockDim.x) {
-    const int row = blockIdx.x * rows_per + i / hid, col = i % hid;
+  for (int i = threadIdx.x; i < rows_per * q_per_row; i += blockDim.x) {
+    const int row = blockIdx.x * rows_per + i / q_per_row, col = 4 * (i % q_per_row);
     const size_t o = mo + (size_t)row * hid + col;
-    const float v = row < d ? (float)((double)X[o] * inv) : 0.f;
-    X[o] = v;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < d) {
+      const float4 x = *reinterpret_cast<const float4*>(X + o);
+      v = make_float4((float)((double)x.x * inv), (float)((double)x.y * inv),
+                      (float)((double)x.z * inv), (float)((double)x.w * inv));
+    }
+    *reinterpret_cast<float4*>(X + o) = v;
     // the bf16 pair the tensor-core iteration reads: hi + lo carries ~16 bits
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    Xh[o] = h;
-    Xl[o] = __float2bfloat16_rn(v - __bfloat162float(h));
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    uint32_t hp[2], lp[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * k]), h1 = __float2bfloat16_rn(f[2 * k + 1]);
+      hp[k] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      lp[k] = pack_bf16x2(f[2 * k] - __bfloat162float(h0), f[2 * k + 1] - __bfloat162float(h1));
+    }
+    *reinterpret_cast<uint2*>(Xh + o) = make_uint2(hp[0], hp[1]);
+    *reinterpret_cast<uint2*>(Xl + o) = make_uint2(lp[0], lp[1]);
   }
 }
 
