@@ -70,8 +70,9 @@ def peaks():
 
 def workload_config(w: wl.Workload, layers: int) -> dict:
     return {
-        "workload": (f"{w.name}: {w.frames} frames x {w.p} tokens = {w.n_tokens} tokens in one "
-                     f"chunk, {w.heads} heads x d={w.d}, SwiGLU hidden {w.hidden}, {layers} "
+        "workload": (f"{w.name}: {w.frames} frames x {w.p} tokens = {w.n_tokens} tokens "
+                     f"{'fed one frame per update' if w.name.startswith('stream') else 'in one chunk'}"
+                     f", {w.heads} heads x d={w.d}, SwiGLU hidden {w.hidden}, {layers} "
                      f"layers, {w.n_ray} ray queries"),
         "tokens": w.n_tokens, "ray_queries": w.n_ray, "layers": layers, "heads": w.heads,
         "d": w.d, "hidden": w.hidden, "renorm": "row",
@@ -181,8 +182,12 @@ def oracle_sample(w: wl.Workload, frames: int, seed_layer: int = 0):
     import oracle as O
     x = wl.make_inputs(w, n_tokens=frames * w.p, layer=seed_layer)
     t0 = time.perf_counter()
-    Wh = O.ttt_update(x.W1, x.W2, x.W3, x.K, x.V, x.eta, O.RENORM_ROW)
-    O.ttt_apply(*Wh, x.Q)
+    if w.name.startswith("stream"):
+        # streaming: one update + apply per frame, the state carried over
+        O.ttt_stream(x.W1, x.W2, x.W3, x.K, x.V, x.eta, x.Q, w.p, O.RENORM_ROW)
+    else:
+        Wh = O.ttt_update(x.W1, x.W2, x.W3, x.K, x.V, x.eta, O.RENORM_ROW)
+        O.ttt_apply(*Wh, x.Q)
     return frames * w.p, time.perf_counter() - t0
 
 
@@ -221,7 +226,9 @@ def run_reference(args, w: wl.Workload, world: int, rank: int):
         times.append(dt)
     t = sum(times) / len(times)
     value = tok / t
-    sample = (f"fp64 numpy oracle, one layer of {w.name}: update + image apply on {frames} "
+    what = ("per-frame update + apply (streaming)" if w.name.startswith("stream")
+            else "update + image apply")
+    sample = (f"fp64 numpy oracle, one layer of {w.name}: {what} on {frames} "
               f"frames ({tok} tokens, {w.heads} heads) per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -383,6 +390,20 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     if args.ns_steps:
         line["config"]["ns_steps"] = args.ns_steps
 
+    # -------------------------------------------------- ray queries on their own
+    if M:
+        er0, er1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        er0.record(stream)
+        for _ in range(5):
+            R.ttt_apply(cfg, Qr, Or, shadow=shadow, stream=stream)
+        er1.record(stream)
+        torch.cuda.synchronize(dev)
+        ray_ms = rank_max(er0.elapsed_time(er1) / 5)
+        img_ms = ms / layers - ray_ms
+        line["ray_apply"] = {"queries": M, "ms_per_layer": ray_ms,
+                             "update_plus_image_apply_ms_per_layer": img_ms,
+                             "tokens_per_s_update_plus_image_apply":
+                                 aggregate_value(world, T, 1, img_ms)}
     # -------------------------------------------------- e2e through host buffers
     if not args.no_e2e:
         line["e2e"] = e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta,
