@@ -21,9 +21,12 @@ namespace {
 // TMEM lane quadrant split a row's columns: each copies its half of the o'
 // row out of the ring slots the MMA just consumed (a slot is refilled only
 // after the MMA and all epilogue warps released it), the halves' sums of
-// squares meet in shared memory (summed in a fixed order), and o is written
-// in bf16.  o may overwrite o': o' is read only through TMA, before o of that
-// tile is written, and only its own CTA touches the tile.
+// squares meet in shared memory (summed in a fixed order), and each warp
+// writes its 32 rows x 32 columns of o (bf16) into a private 2 KB buffer
+// (64-byte swizzle) and stores them with its own TMA box, so the global
+// writes are whole 64-byte row segments.  o may overwrite o': o' is read only
+// through TMA, before o of that tile is written, and only its own CTA
+// touches the tile.
 // ----------------------------------------------------------------------------
 template <int D>
 struct GT {
@@ -34,9 +37,12 @@ struct GT {
   static constexpr int OFF_WG = 0;
   static constexpr int OFF_A = OFF_WG + NCH * WG;
   static constexpr int OFF_SS = OFF_A + NSLOT * SLOT;  // [2 parity][2 half][BM] floats
-  static constexpr int OFF_BAR = OFF_SS + 2 * 2 * BM * 4;
+  static constexpr int OFF_OST = OFF_SS + 2 * 2 * BM * 4;  // per epilogue warp: 32 x 64 B
+  static constexpr int OST = 32 * 64;
+  static constexpr int OFF_BAR = OFF_OST + 8 * OST;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int EPI_WARPS = 8;       // two per TMEM lane quadrant
+  static_assert(SMEM <= 227 * 1024, "shared memory");
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr uint32_t TMEM_COLS = 2 * D <= 128 ? 128 : 2 * D;  // two accumulators
 };
@@ -44,7 +50,7 @@ struct GT {
 template <int D>
 __global__ void __launch_bounds__(GT<D>::THREADS, 1)
     gate_kernel(const __grid_constant__ CUtensorMap mWg, const __grid_constant__ CUtensorMap mA,
-                __nv_bfloat16* Oout, int64_t m, int H, float eps,
+                const __grid_constant__ CUtensorMap mO, int64_t m, int H, float eps,
                 int* err) {
   using L = GT<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -154,6 +160,7 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
     const int row = q * 32 + lane;
     const size_t ld = (size_t)H * D;
     float* ss_part = reinterpret_cast<float*>(smem + L::OFF_SS);
+    uint8_t* ost = smem + L::OFF_OST + (warp - 2) * L::OST;
     for (int64_t t = t0, i = 0; t < ntiles; t += tstride, ++i) {
       const int b = (int)(i & 1);
       const int64_t r = t * BM + row;
@@ -212,18 +219,26 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
           pk[e / 2] = pack_bf16x2(o.x * inv * g0 * sigmoid_fast(g0),
                                   o.y * inv * g1 * sigmoid_fast(g1));
         }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(Oout + r * ld + (size_t)head * D + half * HALF +
-                                                32 * g);
+        // this warp's [32 rows x 32 columns] of o through its staging buffer
+        // (64-byte swizzle: 16-byte unit c of row r at c ^ ((r / 2) % 4))
+        if (lane == 0) bulk_wait_group_read0();  // the previous box has been read
+        __syncwarp();
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(ost + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && t * BM + 32 * q < m) {  // rows past m are clipped by the store
+          tma_store_2d(&mO, ost, head * D + half * HALF + 32 * g, (int)(t * BM) + 32 * q);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
+    if (lane == 0) bulk_wait_group0();
   }
   tc_fence_before();
   __syncthreads();
@@ -240,7 +255,7 @@ cudaError_t tc_gate_impl(const Problem& p, const __nv_bfloat16* Wg, const void* 
   if (p.n == 0) return cudaSuccess;
   int* err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidDevice;
-  CUtensorMap mWg, mA;
+  CUtensorMap mWg, mA, mO;
   {
     const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * D}, str[1] = {(uint64_t)D * 2};
     const uint32_t box[2] = {CH, (uint32_t)D};
@@ -250,7 +265,10 @@ cudaError_t tc_gate_impl(const Problem& p, const __nv_bfloat16* Wg, const void* 
     const uint64_t ld = (uint64_t)p.H * D;
     const uint64_t dims[2] = {ld, (uint64_t)p.n}, str[1] = {ld * 2};
     const uint32_t box[2] = {CH, BM};
-    if (!make_map(&mA, Oin, 2, dims, str, box)) return cudaErrorInvalidValue;
+    const uint32_t obox[2] = {32, 32};
+    if (!make_map(&mA, Oin, 2, dims, str, box) ||
+        !make_map(&mO, Oout, 2, dims, str, obox, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
   }
   cudaError_t e = ensure_smem_attr(gate_kernel<D>, GT<D>::SMEM);
   if (e != cudaSuccess) return e;
@@ -261,7 +279,7 @@ cudaError_t tc_gate_impl(const Problem& p, const __nv_bfloat16* Wg, const void* 
   {
     TraceScope ts("tc_gate", st);
     gate_kernel<D><<<grid, GT<D>::THREADS, GT<D>::SMEM, st>>>(
-        mWg, mA, static_cast<__nv_bfloat16*>(Oout), p.n,
+        mWg, mA, mO, p.n,
         p.H, eps, err);
   }
   return cudaGetLastError();

@@ -33,12 +33,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 tensor of rank 2..5 with dims[0] contiguous; box inner dim is 64
-// elements (128 bytes) with the 128-byte swizzle.  Out-of-range rows read 0.
+// elements (128 bytes) with the 128-byte swizzle (or 32 elements with the
+// 64-byte swizzle).  Out-of-range rows read 0 and are not written.
 // The outer dimensions may be listed in any stride order: a "chunk" dimension
 // of stride 128 bytes placed after the row dimension makes one box land as
 // consecutive [rows x 128 B] blocks, the layout the MMA descriptors expect.
 bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-              const uint64_t* byte_strides, const uint32_t* box) {
+              const uint64_t* byte_strides, const uint32_t* box,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t gd[5], gs[4];
@@ -49,7 +51,7 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = byte_strides[i];
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                  gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
