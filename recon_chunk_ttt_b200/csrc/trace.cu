@@ -2,8 +2,11 @@
 // library is bracketed by two CUDA events recorded on the caller's stream, and
 // ttt_trace_read() turns them into launch counts and accumulated device time
 // per kernel name.  Disabled (the default), a TraceScope costs one branch.
+// Independently, every scope is an NVTX range named after the kernel, so a
+// profiler can select the library's launches by range (a no-op without one).
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstring>
 #include <mutex>
@@ -48,6 +51,7 @@ cudaEvent_t take_event() {
 bool trace_on() { return g_on; }
 
 TraceScope::TraceScope(const char* name, cudaStream_t st) : name_(name), st_(st), a_(nullptr) {
+  nvtxRangePushA(name);
   if (!g_on) return;
   std::lock_guard<std::mutex> lk(g_mu);
   a_ = take_event();
@@ -55,6 +59,7 @@ TraceScope::TraceScope(const char* name, cudaStream_t st) : name_(name), st_(st)
 }
 
 TraceScope::~TraceScope() {
+  nvtxRangePop();
   if (a_ == nullptr) return;
   std::lock_guard<std::mutex> lk(g_mu);
   cudaEvent_t b = take_event();
