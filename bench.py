@@ -53,6 +53,8 @@ def parse():
                     help="Newton-Schulz steps on the gradient in the timed step (0: off)")
     ap.add_argument("--no-gate-probe", action="store_true",
                     help="skip the gated-output-unit measurement")
+    ap.add_argument("--no-shard-probe", action="store_true",
+                    help="skip the token-sharded update measurement")
     ap.add_argument("--no-ns-probe", action="store_true",
                     help="skip the separate 5-step Newton-Schulz update measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -413,6 +415,10 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     if not args.no_ns_probe:
         line["ns_update"] = ns_probe(R, torch, dev, cfg_ns, K, V, eta, Win[0], Wout[0], shadow,
                                      ws_buf, stream, d, hid, H, pk, rank_max)
+    # -------------------------------------------------- token-sharded update
+    if not args.no_shard_probe:
+        line["sharded_update"] = shard_probe(R, torch, dev, cfg, K, V, eta, Win[0], Wout[0],
+                                             shadow, ws_buf, stream, T, world, rank, rank_max)
     # -------------------------------------------------- gated output unit
     if not args.no_gate_probe:
         line["gate"] = gate_probe(R, torch, dev, cfg, O, H, d, T, stream, pk, rank_max)
@@ -465,6 +471,41 @@ def ns_probe(R, torch, dev, cfg, K, V, eta, Win, Wout, shadow, ws, stream, d, hi
             "stages_ms": {k: tr[k][1] / reps for k in ns_names if k in tr},
             "note": "NS GEMMs issue 3 bf16 MMAs per product (hi/lo operand split); "
                     "achieved counts the algorithmic flops once"}
+
+
+def shard_probe(R, torch, dev, cfg, K, V, eta, Win, Wout, shadow, ws, stream, T, world, rank,
+                rank_max, reps: int = 5) -> dict:
+    """One layer's update of the whole scene split over the ranks: each rank
+    reduces its token shard (ttt_update_partial), the partials are exchanged
+    by one NCCL all-gather, and every rank finishes the same Ŵ
+    (ttt_update_finish).  Timed with events on the stream, max over ranks."""
+    from recon_chunk_ttt_b200.sharded import exchange_partials, shard_range
+    a, b = shard_range(T, rank, world)
+    Kr, Vr, er = K[a:b], V[a:b], eta[a:b]
+    partial = torch.empty(R.ttt_partial_floats(cfg), dtype=torch.float32, device=dev)
+    fin_ws = torch.empty(max(R.ttt_finish_workspace_bytes(cfg), 1), dtype=torch.uint8,
+                         device=dev)
+
+    def one():
+        R.ttt_update_partial(cfg, *Win, Kr, Vr, er, partial=partial, workspace=ws, stream=stream)
+        gathered = exchange_partials(partial) if world > 1 else partial.view(1, -1)
+        R.ttt_update_finish(cfg, *Win, gathered, *Wout, shadow=shadow, workspace=fin_ws,
+                            stream=stream)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    R.ttt_check_device_error()
+    ms = rank_max(e0.elapsed_time(e1) / reps)
+    return {"ranks": world, "tokens_per_rank": b - a, "tokens": T, "ms_per_layer_update": ms,
+            "update_tokens_per_s_one_scene": T / (ms / 1e3),
+            "exchange": "NCCL all-gather of one fp32 partial per rank" if world > 1 else "none"}
 
 
 def gate_probe(R, torch, dev, cfg, O, H, d, T, stream, pk, rank_max, reps: int = 5) -> dict:
