@@ -292,12 +292,9 @@ struct NsMaps {
                                // N3/64 column blocks}, landing as [block][row][128 B]
   CUtensorMap ah, al, bh, bl;  // A, B hi / lo, K-major: box {64 k, 128 rows}
 };
-// Global buffers of all matrices (matrix m at m * Rp * C or m * Rp * Rp).
+// fp32 iterates of all matrices (matrix m at m * Rp * C).
 struct NsBufs {
-  float* xf[2];
-  __nv_bfloat16 *xh[2], *xl[2];
-  float* af;
-  __nv_bfloat16 *ah, *al, *bh, *bl;
+  float* xf[2];  // fp32 iterates: X0 (read at start), the final X (written on the last step)
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -639,16 +636,7 @@ cudaError_t launch_ns_tc(const Problem& p, const NsWs& w, int* err, cudaStream_t
       return cudaErrorInvalidValue;
   }
   NsBufs buf;
-  for (int b = 0; b < 2; ++b) {
-    buf.xf[b] = w.X[b];
-    buf.xh[b] = w.Xh[b];
-    buf.xl[b] = w.Xl[b];
-  }
-  buf.af = w.A;
-  buf.ah = w.Ah;
-  buf.al = w.Al;
-  buf.bh = w.Bh;
-  buf.bl = w.Bl;
+  for (int b = 0; b < 2; ++b) buf.xf[b] = w.X[b];
   cudaError_t e = ensure_smem_attr(ns_tc_kernel<RP, C>, L::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
