@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("ttt_update", "ttt_apply", "ttt_stream_step", "ttt_update_workspace_bytes",
               "ttt_status_string", "ttt_shadow_bytes", "ttt_pack_shadow",
-              "ttt_check_device_error", "ttt_chunked"):
+              "ttt_check_device_error", "ttt_chunked", "ttt_gate", "ttt_update_partial",
+              "ttt_update_finish", "ttt_partial_floats", "ttt_finish_workspace_bytes"):
         assert n in names
 
 
@@ -162,3 +163,44 @@ def test_chunked_rejects_bad_arguments(B):
     f32 = _cfg(B, precision=B.PREC_FP32_CHECK)
     assert call(f32, n=0, shadow=None) == B.TTT_OK
     assert call(cfg, ws=None, mask=none, n=0) == B.TTT_OK
+
+
+def test_gate_partial_finish_reject_bad_arguments(B):
+    """Validation of ttt_gate, ttt_update_partial and ttt_update_finish happens
+    before any launch (FAKE pointers are never dereferenced)."""
+    L = B.lib()
+    cfg = _cfg(B)
+    c = ctypes.byref(cfg)
+    # gate
+    assert L.ttt_gate(None, FAKE, FAKE, 5, FAKE, None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_gate(c, None, FAKE, 5, FAKE, None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_gate(c, FAKE, None, 5, FAKE, None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_gate(c, FAKE, FAKE, -1, FAKE, None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_gate(c, FAKE + 8, FAKE, 5, FAKE, None) == B.TTT_ERR_ALIGNMENT
+    assert L.ttt_gate(c, FAKE, FAKE, 0, None, None) == B.TTT_OK  # nothing to do
+    assert L.ttt_gate(ctypes.byref(_cfg(B, d=128, hidden=256)), FAKE, FAKE, 5, FAKE,
+                      None) == B.TTT_ERR_UNSUPPORTED_SHAPE
+    # partial
+    assert B.ttt_partial_floats(cfg) == 3 * 4 * 256 * 512
+    assert L.ttt_update_partial(c, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, None, FAKE, 1 << 40,
+                                None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_update_partial(c, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, FAKE, FAKE, 1 << 40,
+                                None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_update_partial(c, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 10, FAKE, FAKE,
+                                1 << 40, None) == B.TTT_ERR_ALIGNMENT
+    assert L.ttt_update_partial(c, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, FAKE, FAKE, 100,
+                                None) == B.TTT_ERR_WORKSPACE
+    # finish
+    need = B.ttt_finish_workspace_bytes(cfg)
+    assert need > 0
+    ns5 = _cfg(B, ns_steps=5)
+    assert B.ttt_finish_workspace_bytes(ns5) > need  # the Newton-Schulz region
+    args = [FAKE, FAKE, FAKE, FAKE]
+    assert L.ttt_update_finish(c, *args, 0, FAKE, FAKE, FAKE, None, FAKE, need,
+                               None) == B.TTT_ERR_INVALID_ARG   # no ranks
+    assert L.ttt_update_finish(c, *args, 2, None, FAKE, FAKE, None, FAKE, need,
+                               None) == B.TTT_ERR_INVALID_ARG
+    assert L.ttt_update_finish(c, *args, 2, FAKE, FAKE, FAKE, None, FAKE, need - 1,
+                               None) == B.TTT_ERR_WORKSPACE
+    assert L.ttt_update_finish(c, *args, 2, FAKE, FAKE, FAKE, FAKE + 2, FAKE, need,
+                               None) == B.TTT_ERR_ALIGNMENT
