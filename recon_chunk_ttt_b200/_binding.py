@@ -14,7 +14,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libttt.so")
+# RECON_CHUNK_TTT_LIB may name another build of the same library (the debug
+# build, libttt_debug.so); it must exist, there is no fallback.
+LIB_PATH = os.environ.get("RECON_CHUNK_TTT_LIB") or os.path.join(_HERE, "libttt.so")
 
 TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED_SHAPE, TTT_ERR_ALIGNMENT, \
     TTT_ERR_WORKSPACE, TTT_ERR_CUDA, TTT_ERR_DEVICE = range(7)

@@ -1,9 +1,13 @@
 """Build libttt.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m recon_chunk_ttt_b200.build [--force] [--verbose]
+    python -m recon_chunk_ttt_b200.build [--force] [--verbose] [--debug]
 
 The library is compiled from csrc/*.cu into recon_chunk_ttt_b200/libttt.so;
-it is rebuilt when any source or header is newer than the library.
+it is rebuilt when any source or header is newer than the library.  --debug
+builds libttt_debug.so instead, with -DTTT_DEBUG: the kernels then check
+their TMA coordinates, TMEM columns and store indices and report a failed
+check in the device error word (ttt_check_device_error) rather than trapping.
+The binding loads it when RECON_CHUNK_TTT_LIB names its path.
 """
 from __future__ import annotations
 
@@ -18,6 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libttt.so")
+LIB_DEBUG = os.path.join(PKG, "libttt_debug.so")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
@@ -45,18 +50,20 @@ def _inputs():
         sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", tmp, *sources()]
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp"
+    flags = [*NVCC_FLAGS, *(["-DTTT_DEBUG"] if debug else [])]
+    cmd = [_nvcc(), *flags, *extra, "-I", INCLUDE, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -64,12 +71,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if verbose and (r.stdout or r.stderr):
         print(r.stdout, r.stderr, sep="\n")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     force = "--force" in sys.argv
     verbose = "--verbose" in sys.argv
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []
-    print(build(force=force or bool(extra), verbose=verbose or bool(extra), extra=extra))
+    print(build(force=force or bool(extra), verbose=verbose or bool(extra), extra=extra,
+                debug="--debug" in sys.argv))

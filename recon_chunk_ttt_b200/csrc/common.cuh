@@ -19,7 +19,25 @@ enum DeviceErr : int {
   kErrWaitAccFree = 4,   // MMA issuer gave up waiting for a drained accumulator
   kErrWaitOperand = 5,   // MMA issuer gave up waiting for an epilogue operand
   kErrWaitFinal = 6,     // final drain gave up
+  // debug builds only (TTT_DCHECK): a range check failed
+  kErrCheckTma = 16,     // a TMA coordinate outside its tensor
+  kErrCheckTmem = 17,    // a TMEM column outside the allocation
+  kErrCheckIndex = 18,   // a global or shared-memory index outside its buffer
 };
+
+// Debug builds (-DTTT_DEBUG, libttt_debug.so): device-side range checks that
+// record a code in the device error word and let the kernel go on (no trap);
+// release builds compile them out.
+#ifdef TTT_DEBUG
+#define TTT_DCHECK(cond, err, code)              \
+  do {                                           \
+    if (!(cond)) atomicExch((err), (int)(code)); \
+  } while (0)
+#else
+#define TTT_DCHECK(cond, err, code) \
+  do {                              \
+  } while (0)
+#endif
 
 // About 2^31 SM cycles: > 1 s at the B200 clock, far above any legitimate
 // wait (a stage load or an MMA batch takes microseconds).

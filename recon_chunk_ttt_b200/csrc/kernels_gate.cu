@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
           break;
         }
         mbar_arrive_expect_tx(&full[slot], L::SLOT);
+        TTT_DCHECK(t * BM < m && head * D + (c + 1) * CH <= H * D, err, kErrCheckTma);
         tma_load_2d(smem + L::OFF_A + slot * L::SLOT, &mA, &full[slot], head * D + c * CH,
                     (int)(t * BM));
         ++issued;
@@ -207,6 +208,7 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
 #pragma unroll
       for (int g = 0; g < HALF / 32; ++g) {
         uint32_t acc[32];
+        TTT_DCHECK(b * D + half * HALF + 32 * g + 32 <= (int)L::TMEM_COLS, err, kErrCheckTmem);
         tmem_ld_32x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * D + half * HALF + 32 * g),
                       acc);
         tmem_ld_wait();
@@ -229,6 +231,7 @@ __global__ void __launch_bounds__(GT<D>::THREADS, 1)
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         fence_proxy_async_smem();
         __syncwarp();
+        TTT_DCHECK(head * D + half * HALF + 32 * g + 32 <= H * D, err, kErrCheckTma);
         if (lane == 0 && t * BM + 32 * q < m) {  // rows past m are clipped by the store
           tma_store_2d(&mO, ost, head * D + half * HALF + 32 * g, (int)(t * BM) + 32 * q);
           bulk_commit_group();

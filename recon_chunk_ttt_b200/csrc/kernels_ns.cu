@@ -346,6 +346,7 @@ __device__ __forceinline__ void ns_epilogue(uint64_t* acc_full, uint32_t parity,
   const int q = warp & 3, half = (warp - 2) >> 2;
   const int row = 32 * q + lane;
   const uint32_t lanes = (uint32_t)(32 * q) << 16;
+  TTT_DCHECK(kXR + N <= kNsTmemCols && HALF % 32 == 0, err, kErrCheckTmem);
   uint8_t* hi = stage;
   uint8_t* lo = stage + N * 256;  // N/64 chunks of 16 KB
   mbar_wait(acc_full, parity, abort, err, kErrWaitAcc);
@@ -488,6 +489,8 @@ __global__ void __launch_bounds__(NSL<RP, C>::THREADS, 1)
             uint8_t* st = smem + s * L::STAGE;
             uint8_t* bst = st + 2 * L::A_T;
             const int k0 = j * 64;
+            TTT_DCHECK(mi * 128 + 128 <= RP && ni * 128 + 128 <= RP && k0 + 64 <= (p == 0 ? C : RP),
+                       err, kErrCheckTma);
             if (p == 0) {
               mbar_arrive_expect_tx(&full[s], 4 * L::A_T);
               tma_load_2d(st, &maps.xh[cur], &full[s], k0, mrow + mi * 128);

@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
         }
         mbar_arrive_expect_tx(wfull, L::NCH * (L::W13_CH + L::W2_CH));
         const int row = head * hid + slice * HS;
+        TTT_DCHECK(row >= 0 && row + HS <= H * hid, err, kErrCheckTma);
         for (int c = 0; c < L::NCH; ++c) {
           uint8_t* w13 = smem + L::OFF_W13 + c * L::W13_CH;
           tma_load_2d(w13, &mW1, wfull, c * CH, row);
@@ -194,6 +195,8 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], L::STAGE);
+          TTT_DCHECK(y >= 0 && (int64_t)y < n && head * L::NCH + (g + 1) * L::CPS <= H * L::NCH,
+                     err, kErrCheckTma);
           // one box = CPS chunks of [128 tokens x 64 d]
           tma_load_3d(smem + L::OFF_STAGE + stage * L::STAGE, m, &full[stage], 0, y,
                       head * L::NCH + g * L::CPS);
@@ -287,6 +290,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
       abits ^= 1u << buf;
       tc_fence_after();
       const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256 + ch * 32;
+      TTT_DCHECK(buf * 256 + ch * 32 + 128 + 32 <= (int)L::TMEM_COLS, err, kErrCheckTmem);
       uint32_t r1[32], r3[32], rd[32];
       tmem_ld_32x32(tl, r1);
       tmem_ld_32x32(tl + HS, r3);
@@ -319,6 +323,7 @@ __global__ void __launch_bounds__(FB<D>::THREADS, 1)
       // before refilling one, the store issued from it two stores ago must
       // have finished reading it.
       const int x = slice * HS, y = (int)(tile * BM);
+      TTT_DCHECK(x + HS <= hid && (int64_t)y < n, err, kErrCheckTma);
 #pragma unroll
       for (int o = 0; o < 3; ++o) {
         uint8_t* box = stage_out + (out_k & 1) * L::OUT_TILE;
@@ -480,6 +485,7 @@ __global__ void __launch_bounds__(GR<D>::THREADS, 1)
       const int blk = kind == 0 ? a : 2;  // P1, P3, P2
       float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat;
       const int j = (kind == 0 ? j_first : j_first + a * BM) + q * 32 + lane;
+      TTT_DCHECK(j < hid && a * 256 + D <= (int)L::TMEM_COLS, err, kErrCheckIndex);
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t rr[32];
         if (have) {
@@ -620,6 +626,7 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
           break;
         }
         mbar_arrive_expect_tx(&q_full[c], BM * 128);
+        TTT_DCHECK(qt * BM < m && head * D + (c + 1) * CH <= H * D, err, kErrCheckTma);
         tma_load_2d(smem + L::OFF_Q + c * BM * 128, &mQ, &q_full[c], head * D + c * CH,
                     (int)(qt * BM));
       }
@@ -630,6 +637,8 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
           if (!st) { ok = false; return; }
           mbar_arrive_expect_tx(&full[stage], L::CH_PER_STAGE * L::W13_CH);
           // one box: CH_PER_STAGE d-chunks x {W1s, W3s} x 64 rows
+          TTT_DCHECK(head * hid + (js + 1) * HS <= H * hid &&
+                         (g + 1) * L::CH_PER_STAGE <= L::NCH, err, kErrCheckTma);
           tma_load_4d(st, &mW13, &full[stage], 0, head * hid + js * HS, 0, g * L::CH_PER_STAGE);
           advance();
         }
@@ -638,6 +647,7 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
         uint8_t* st = next();
         if (!st) { ok = false; return; }
         mbar_arrive_expect_tx(&full[stage], D * 128);
+        TTT_DCHECK((js + 1) * HS <= hid && head < H, err, kErrCheckTma);
         tma_load_2d(st, &mW2, &full[stage], js * HS, head * D);
         advance();
       };
@@ -794,6 +804,7 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
         tmem_ld_32x32(to + c0, rr);
         tmem_ld_wait();
         if (qi < m) {
+          TTT_DCHECK(c0 + 32 <= D && head < H, err, kErrCheckIndex);
           uint4* dst = reinterpret_cast<uint4*>(O + qi * (int64_t)H * D + (int64_t)head * D + c0);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
