@@ -529,9 +529,16 @@ def gate_probe(R, torch, dev, cfg, O, H, d, T, stream, pk, rank_max, reps: int =
     ms = rank_max(e0.elapsed_time(e1) / reps)
     by = 4.0 * T * H * d
     gbs = by / (ms / 1e3) / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            ent = json.load(f).get("tc_gate")
+        if ent and ent.get("source_sha") == kernel_source_sha(ent.get("sources")):
+            traffic = ent["bytes_per_unit"] * T * H
     return {"ms_per_launch": ms, "rows": T, "achieved_gbs": gbs,
             "frac_of_hbm": gbs / pk["hbm_gbs"], "tflops": 2.0 * d * d * T * H / (ms / 1e3) / 1e12,
-            "bytes_per_launch": by}
+            "bytes_per_launch": by, "traffic": traffic}
 
 
 def stream_bench(R, torch, dev, rank_max, warm_frames: int = 8) -> dict:
