@@ -161,6 +161,18 @@ ttt_status ttt_stream_step(const ttt_config* cfg,
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code);
 
 /*
+ * Failure-detection self-test (no counterpart on the pages): launches one
+ * block whose thread waits, through the same bounded mbarrier wait the
+ * kernels use, on a barrier nothing completes.  After limit_cycles SM cycles
+ * (1 .. 2^31) the wait gives up, writes TTT_DEVICE_ERR_SELFTEST into the
+ * device error word and the kernel returns; the next ttt_check_device_error
+ * then returns TTT_ERR_DEVICE with that code, and the context stays usable.
+ * Nothing traps or hangs.
+ */
+enum { TTT_DEVICE_ERR_SELFTEST = 7 };
+ttt_status ttt_selftest_wait_timeout(int64_t limit_cycles, ttt_stream_t stream);
+
+/*
  * Gated output unit (kimjy99 review, section 2 "Feature Backbone", the last
  * equation): o = RMSNorm(o') ⊙ SiLU(W_g o'), applied per head to the layer
  * output o' (e.g. ttt_apply's O).  The page does not say whether the unit
@@ -247,7 +259,7 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
  * cudaMalloc after start-up).  The call allocates nothing.
  *  - Returns TTT_ERR_WORKSPACE, before launching anything, when
  *    ttt_update_workspace_bytes(cfg, n) exceeds TTT_STATIC_SCRATCH_BYTES
- *    (with 4 heads of d = 256, hidden 512 that is about 2,100 tokens per call;
+ *    (with 4 heads of d = 256, hidden 512 that is 2,560 tokens per call;
  *    one 518 x 518 frame is 1,374).
  *  - Every GPU that loads the library may hold the array until exit.
  *  - All calls on a device share the array and it keeps the last call's

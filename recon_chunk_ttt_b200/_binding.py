@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_chunked.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
                                   ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
         L.ttt_chunked.restype = ctypes.c_int
+        L.ttt_selftest_wait_timeout.argtypes = [_I64, _P]
+        L.ttt_selftest_wait_timeout.restype = ctypes.c_int
         L.ttt_check_device_error.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
         L.ttt_check_device_error.restype = ctypes.c_int
         L.ttt_trace_enable.argtypes = [ctypes.c_int32]
@@ -280,6 +282,16 @@ def ttt_chunked(cfg: ttt_config, W1, W2, W3, shadow, K, V, eta, Q, chunk: int,
                              mask, _ptr(O), _ptr(workspace), nbytes, _stream(stream)),
            "ttt_chunked")
     return O
+
+
+DEVICE_ERR_SELFTEST = 7  # TTT_DEVICE_ERR_SELFTEST
+
+
+def ttt_selftest_wait_timeout(limit_cycles: int = 1 << 24, stream=None) -> None:
+    """Launch the failure-detection self-test: a bounded wait that runs out
+    after limit_cycles and reports DEVICE_ERR_SELFTEST in the error word."""
+    _check(lib().ttt_selftest_wait_timeout(int(limit_cycles), _stream(stream)),
+           "ttt_selftest_wait_timeout")
 
 
 def ttt_check_device_error(stream=None) -> int:

@@ -19,6 +19,7 @@ enum DeviceErr : int {
   kErrWaitAccFree = 4,   // MMA issuer gave up waiting for a drained accumulator
   kErrWaitOperand = 5,   // MMA issuer gave up waiting for an epilogue operand
   kErrWaitFinal = 6,     // final drain gave up
+  kErrSelfTest = 7,      // ttt_selftest_wait_timeout: the wait ran out as intended
   // debug builds only (TTT_DCHECK): a range check failed
   kErrCheckTma = 16,     // a TMA coordinate outside its tensor
   kErrCheckTmem = 17,    // a TMEM column outside the allocation
@@ -81,13 +82,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // the device error word `err` and false is returned; the caller then leaves
 // its loop and goes to the CTA's common exit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err, int reason) {
+                                          int* err, int reason,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       atomicExch(err, reason);
       return false;

@@ -81,6 +81,9 @@ cudaError_t tc_gate(const Problem& p, const void* Wg, const void* Oin, void* Oou
 cudaError_t f32_gate(const Problem& p, const float* Wg, const float* Oin, float* Oout, float eps,
                      cudaStream_t st);
 
+// One block whose bounded mbarrier wait runs out after limit_cycles.
+cudaError_t selftest_wait_timeout(long long limit_cycles, cudaStream_t st);
+
 // The per-device error word (defined in kernels_common.cu).
 int* device_error_ptr();                       // device address, nullptr on failure
 cudaError_t read_and_clear_device_error(int* value);

@@ -172,6 +172,21 @@ __global__ void __launch_bounds__(256) sum_splits_kernel(const float* __restrict
       make_float4((float)acc[0], (float)acc[1], (float)acc[2], (float)acc[3]);
 }
 
+// Failure-detection self-test: thread 0 waits on an mbarrier nothing will
+// complete, through the same bounded wait the kernels use, with a short
+// limit; the wait gives up, records kErrSelfTest and the kernel returns.
+__global__ void selftest_timeout_kernel(long long limit, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, kErrSelfTest, limit);
+}
+
 }  // namespace
 
 cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const float* W1,
@@ -194,6 +209,13 @@ cudaError_t sum_splits(int S, size_t count, const float* partials, float* out, c
   const size_t threads = (count + 3) / 4;
   TraceScope ts("sum_splits", st);
   sum_splits_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(partials, S, count, out);
+  return cudaGetLastError();
+}
+
+cudaError_t selftest_wait_timeout(long long limit_cycles, cudaStream_t st) {
+  int* err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidDevice;
+  selftest_timeout_kernel<<<1, 32, 0, st>>>(limit_cycles, err);
   return cudaGetLastError();
 }
 

@@ -296,6 +296,12 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
   return TTT_OK;
 }
 
+ttt_status ttt_selftest_wait_timeout(int64_t limit_cycles, ttt_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > ((int64_t)1 << 31)) return TTT_ERR_INVALID_ARG;
+  return cuda_status(
+      ttt::selftest_wait_timeout((long long)limit_cycles, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ttt_status ttt_check_device_error(ttt_stream_t stream, int32_t* code) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return TTT_ERR_CUDA;

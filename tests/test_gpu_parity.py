@@ -259,3 +259,21 @@ def test_scene700_full_size_sampled():
         ref = O.ttt_apply(x.W1, x.W2, x.W3, wl.bits_to_f32(Qbits[idx]))
         got = Og[torch.from_numpy(idx).cuda()].float().cpu().double().numpy()
         assert O.rel_fro(got, ref) <= TOL_TC
+
+
+def test_bounded_wait_runs_out_and_reports():
+    """Failure detection on the GPU without a fault: a kernel's bounded
+    mbarrier wait on a barrier nothing completes gives up after ~2^24 cycles,
+    the error word carries the self-test code, reading it clears it, and the
+    context keeps working."""
+    R.ttt_selftest_wait_timeout(1 << 24)
+    with pytest.raises(R.TTTError) as e:
+        R.ttt_check_device_error()
+    assert e.value.status == R.TTT_ERR_DEVICE
+    assert f"device error word = {R.DEVICE_ERR_SELFTEST}" in str(e.value)
+    assert R.ttt_check_device_error() == 0
+    x = wl.make_inputs("tiny")
+    gpu = run_update_apply(x, R.PREC_BF16_TC, R.RENORM_ROW)
+    ref = oracle_update_apply(x, R.PREC_BF16_TC, R.RENORM_ROW)
+    assert max(rel_errors(gpu, ref, x)) <= TOL_TC
+    assert R.ttt_check_device_error() == 0
