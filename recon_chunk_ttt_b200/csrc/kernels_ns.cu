@@ -15,7 +15,8 @@
 // Stages (all on the caller's stream):
 //   ns_gather   sum the split-K partials in fixed order, transpose into the
 //               working layout, per-32x32-tile sums of squares (fp64)
-//   ns_scale    fixed-order Frobenius norm, X0 = G / ||G||_F, zero padding
+//   ns_scale    fixed-order Frobenius norm, X0 = G / ||G||_F in fp32 and as
+//               its bf16 pair (hi, lo), zero padding
 //   iterations  tensor cores: one clustered tcgen05 kernel for all steps;
 //               check mode: three fp32 CUDA-core GEMMs per step
 //   ns_finish   Delta back to the partials layout (S = 1) for reduce_renorm
@@ -23,7 +24,8 @@
 // Tensor-core precision: a bf16 MMA of plain operands loses too much through
 // five quintic steps, so every operand x is split as hi = bf16(x),
 // lo = bf16(x - hi) and each product is hi*hi + hi*lo + lo*hi with fp32
-// accumulation in TMEM; the iterate itself stays fp32.
+// accumulation in TMEM; each CTA keeps its own tiles of the iterate (and of
+// A between phases) in fp32 in TMEM, so only the bf16 pairs travel.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -250,8 +252,9 @@ __global__ void __launch_bounds__(256) ns_f32_gemm_kernel(
 
 // ----------------------------------------------------------------------------
 // Tensor-core iteration.  One cluster of (Rp/128)^2 CTAs per working matrix
-// runs every step.  Each GEMM's epilogue writes its result in fp32 (where a
-// later epilogue needs it) and as a bf16 pair hi = bf16(x), lo = bf16(x - hi);
+// runs every step.  Each GEMM's epilogue writes its result as a bf16 pair
+// hi = bf16(x), lo = bf16(x - hi) (TMA bulk stores; the fp32 value stays in
+// TMEM where a later epilogue of the same CTA needs it);
 // the next GEMM's operands are those pairs, loaded by TMA (128-byte swizzle)
 // into a two-stage ring, and each product is hi*hi + hi*lo + lo*hi with fp32
 // accumulation in TMEM.  Per CTA (cluster rank r, mi = r / RB, ni = r % RB,
