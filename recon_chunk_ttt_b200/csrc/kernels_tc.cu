@@ -35,6 +35,22 @@ namespace {
 constexpr int HS = 64;           // hidden slice per fb CTA / apply step
 constexpr int TK = 64;           // tokens per grad stage
 
+// A-operand-in-TMEM forms used by the apply: a 128-row x 16-element bf16
+// slice of a K-major 128-byte-swizzled shared-memory tile copied into 8 TMEM
+// columns (lane = row), and an MMA that reads its A operand from TMEM.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // Weight prologue: bf16 copies of W1, W3 ([H][hid][d]) and of W2^T ([H][hid][d])
 // ----------------------------------------------------------------------------
@@ -534,7 +550,8 @@ struct AP {
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int EPI_WARPS = 8;                    // 2 per TMEM lane quadrant
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr uint32_t TMEM_COLS = 512;             // F[0] 0, F[1] 128, O at 256
+  static constexpr uint32_t TMEM_COLS = 512;             // F at 0, q at 128, O at 256
+  static constexpr uint32_t TM_Q = 128;                  // the q tile (A of F) in TMEM
 };
 
 // Persistent: CTA b takes (query tile, head) items b, b + grid, ...  Per item
@@ -699,37 +716,47 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
     for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
       for (int js = 0; js < nsl && ok; ++js) {
         const int64_t g = i * nsl + js;
-        const int b = (int)(g & 1);
-        if (!mbar_wait(&f_empty[b], (uint32_t)((g >> 1) & 1) ^ 1, abort_flag, err,
-                       kErrWaitAccFree)) {
+        // one F buffer: wait until the epilogue has drained F(g - 1) (which
+        // also means every earlier F MMA, and so every read of the q tile in
+        // TMEM, has completed)
+        if (!mbar_wait(&f_empty[0], (uint32_t)(g & 1) ^ 1, abort_flag, err, kErrWaitAccFree)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int gs = 0; gs < w13_stages && ok; ++gs) {
-          if (!take()) { ok = false; break; }
-          const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
-          for (int cc = 0; cc < L::CH_PER_STAGE && ok; ++cc) {
-            const int c = gs * L::CH_PER_STAGE + cc;
-            if (js == 0) {
-              if (!mbar_wait(&q_full[c], (uint32_t)(i & 1), abort_flag, err, kErrWaitFull)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
+        if (js == 0) {
+          // this item's q tile into TMEM (16 copies of [128 rows x 16 d]);
+          // each shared-memory q chunk goes back to the producer once copied
+          for (int c = 0; c < L::NCH && ok; ++c) {
+            if (!mbar_wait(&q_full[c], (uint32_t)(i & 1), abort_flag, err, kErrWaitFull)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
             const uint32_t qa = sbase + L::OFF_Q + c * BM * 128;
 #pragma unroll
             for (int kk = 0; kk < CH / 16; ++kk)
-              umma_bf16(tmem + b * 128, sdesc_sw128(qa + kk * KSTEP_BYTES, 16, 1024),
-                        sdesc_sw128(st + cc * L::W13_CH + kk * KSTEP_BYTES, 16, 1024), idF,
-                        (c | kk) != 0);
-            if (js == nsl - 1) umma_commit(&q_empty[c]);  // q chunk c no longer needed
+              tmem_cp_128x256b(tmem + L::TM_Q + c * 32 + kk * 8,
+                               sdesc_sw128(qa + kk * KSTEP_BYTES, 16, 1024));
+            umma_commit(&q_empty[c]);
+          }
+          if (!ok) break;
+        }
+        for (int gs = 0; gs < w13_stages && ok; ++gs) {
+          if (!take()) { ok = false; break; }
+          const uint32_t st = sbase + L::OFF_STAGE + stage * L::STAGE;
+          for (int cc = 0; cc < L::CH_PER_STAGE; ++cc) {
+            const int c = gs * L::CH_PER_STAGE + cc;
+#pragma unroll
+            for (int kk = 0; kk < CH / 16; ++kk)
+              umma_bf16_ta(tmem, tmem + L::TM_Q + c * 32 + kk * 8,
+                           sdesc_sw128(st + cc * L::W13_CH + kk * KSTEP_BYTES, 16, 1024), idF,
+                           (c | kk) != 0);
           }
           release();
         }
         if (!ok) break;
-        umma_commit(&f_full[b]);
+        umma_commit(&f_full[0]);
         // O lags F by two slices, so the epilogue of slice js has the time of
         // two F MMAs to produce u before the tensor pipe needs it.
         if (js >= 2 && !do_o(g - 2, js - 2, i)) { ok = false; break; }
@@ -758,18 +785,18 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
         const int64_t g = i * nsl + js;
         const int b = (int)(g & 1);
         const uint32_t par = (uint32_t)((g >> 1) & 1);
-        const bool got = mbar_wait(&f_full[b], par, abort_flag, err, kErrWaitAcc);
+        const bool got = mbar_wait(&f_full[0], (uint32_t)(g & 1), abort_flag, err, kErrWaitAcc);
         __syncwarp();
         if (!got) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + b * 128 + ch * 32;
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + ch * 32;  // the one F buffer
         uint32_t r1[32], r3[32];
         tmem_ld_32x32(tl, r1);
         tmem_ld_32x32(tl + HS, r3);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&f_empty[b]);
+        if (lane == 0) mbar_arrive(&f_empty[0]);
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
