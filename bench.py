@@ -583,13 +583,29 @@ def stream_bench(R, torch, dev, rank_max, warm_frames: int = 8) -> dict:
     lat = sorted(ev[f].elapsed_time(ev[f + 1]) for f in range(w.frames))
     total_ms = rank_max(ev[0].elapsed_time(ev[-1]))
     flops = (12 + 6) * w.d * w.hidden * w.heads * p * w.frames
+    # Where a frame's time goes: a separate, untimed pass with every launch
+    # bracketed by events (the events add their own small cost).
+    nf = min(64, w.frames)
+    R.ttt_trace_enable(True)
+    R.ttt_trace_read(reset=True)
+    for f in range(nf):
+        frame(f)
+    torch.cuda.synchronize(dev)
+    R.ttt_trace_enable(False)
+    tr = R.ttt_trace_read(reset=True)
+    per_kernel_us = {k: v[1] * 1e3 / nf for k, v in tr.items()}
+    busy_us = sum(per_kernel_us.values())
+    p50 = lat[len(lat) // 2]
     return {"workload": f"stream256: {w.frames} frames x {p} tokens, {w.heads} heads x d={w.d}, "
                         f"hidden {w.hidden}, one ttt_stream_step per frame",
-            "frame_ms_p50": lat[len(lat) // 2], "frame_ms_p99": lat[min(len(lat) - 1,
-                                                                      int(0.99 * len(lat)))],
+            "frame_ms_p50": p50, "frame_ms_p99": lat[min(len(lat) - 1, int(0.99 * len(lat)))],
             "host_enqueue_ms_per_frame": host_ms,
             "tokens_per_s": w.frames * p / (total_ms / 1e3),
-            "achieved_tflops": flops / (total_ms / 1e3) / 1e12}
+            "achieved_tflops": flops / (total_ms / 1e3) / 1e12,
+            "kernel_us_per_frame": per_kernel_us,
+            "kernel_busy_us_per_frame": busy_us,
+            "launches_per_frame": sum(v[0] for v in tr.values()) / nf,
+            "between_kernels_us_per_frame": p50 * 1e3 - busy_us}
 
 
 def e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta, Win, Wout,
