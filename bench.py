@@ -101,8 +101,10 @@ class ClockSampler:
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
+        except OSError:  # no nvidia-smi on this machine
             self.proc = None
+            self.f.close()
+            os.unlink(self.path)
 
     def stop(self) -> dict:
         if self.proc is None:
