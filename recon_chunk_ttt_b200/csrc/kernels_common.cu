@@ -21,7 +21,6 @@ namespace {
 
 __device__ int g_device_error = 0;
 
-constexpr int kMaxRowPerLane = 16;  // rows up to 512 elements
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -53,7 +52,95 @@ __device__ __forceinline__ RowRef decode_row(int R, int d, int hid) {
   return r;
 }
 
-__global__ void __launch_bounds__(256) reduce_renorm_kernel(
+// V consecutive floats (V = 2 or 4) as one vector access.
+template <int V>
+__device__ __forceinline__ void load_vec(const float* p, float (&x)[V]) {
+  if constexpr (V == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    x[0] = t.x; x[1] = t.y;
+  }
+}
+
+// One row of one matrix, handled by one warp.  Lane l holds elements
+// 32*V*c + V*l .. +V-1 of the row, c < NC (row length 32*V*NC).  The split
+// sum, W' = W -/+ g and both norms are formed in fp64 so that the only
+// rounding left on Ŵ - W is the final fp32 store.  Each element sums the S
+// partials in increasing s; the row of W and a group of splits (four, or two
+// for the longest rows, to bound registers) are loaded before they are summed,
+// so a row costs about one memory round trip per group.
+template <int V, int NC>
+__device__ __forceinline__ void renorm_row(const float* __restrict__ P0, size_t sstride, int S,
+                                           const float* W, float* Wo, size_t base, double sign,
+                                           int mode, int warp, int lane, __nv_bfloat16_raw* shadow,
+                                           double* scratch) {
+  float wf[NC][V];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) load_vec<V>(W + base + 32 * V * c + V * lane, wf[c]);
+  double wn[NC][V];
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int e = 0; e < V; ++e) wn[c][e] = 0.0;
+  constexpr int G = NC >= 4 ? 2 : 4;
+  for (int s = 0; s < S; s += G) {
+    const int g = S - s < G ? S - s : G;
+    float x[G][NC][V];
+#pragma unroll
+    for (int u = 0; u < G; ++u)
+      if (u < g)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) load_vec<V>(P0 + (size_t)(s + u) * sstride + 32 * V * c, x[u][c]);
+#pragma unroll
+    for (int u = 0; u < G; ++u)
+      if (u < g)
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+          for (int e = 0; e < V; ++e) wn[c][e] += (double)x[u][c][e];
+  }
+  double s_old = 0.0, s_new = 0.0;
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      const double w = (double)wf[c][e];
+      const double wp = w + sign * wn[c][e];
+      wn[c][e] = wp;
+      s_old = fma(w, w, s_old);
+      s_new = fma(wp, wp, s_new);
+    }
+  s_old = warp_sum(s_old);
+  s_new = warp_sum(s_new);
+  double scale = 1.0;
+  if (mode == 1) scale = s_new > 0.0 ? sqrt(s_old) / sqrt(s_new) : 1.0;
+  if (mode == 2 && lane == 0) {
+    scratch[2 * (size_t)warp] = s_old;
+    scratch[2 * (size_t)warp + 1] = s_new;
+  }
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const size_t idx = base + 32 * V * c + V * lane;
+    float v[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) v[e] = (float)(wn[c][e] * scale);
+    uint32_t pk[V / 2];
+#pragma unroll
+    for (int e = 0; e < V; e += 2)
+      pk[e / 2] = (uint32_t)to_bf16_raw(v[e]).x | ((uint32_t)to_bf16_raw(v[e + 1]).x << 16);
+    if constexpr (V == 4) {
+      *reinterpret_cast<float4*>(Wo + idx) = make_float4(v[0], v[1], v[2], v[3]);
+      if (shadow != nullptr) *reinterpret_cast<uint2*>(shadow + idx) = make_uint2(pk[0], pk[1]);
+    } else {
+      *reinterpret_cast<float2*>(Wo + idx) = make_float2(v[0], v[1]);
+      if (shadow != nullptr) *reinterpret_cast<uint32_t*>(shadow + idx) = pk[0];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256, 2) reduce_renorm_kernel(
     const float* __restrict__ partials, int S, int H, int d, int hid, int mode,
     const float* W1, const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
     __nv_bfloat16_raw* __restrict__ shadow, double* __restrict__ scratch) {
@@ -65,51 +152,28 @@ __global__ void __launch_bounds__(256) reduce_renorm_kernel(
   const float* W = r.blk == 0 ? W1 : r.blk == 1 ? W3 : W2;
   float* Wo = r.blk == 0 ? W1o : r.blk == 1 ? W3o : W2o;
   const size_t base = (size_t)r.head * mat + (size_t)r.row * r.len;
-  // P1, P3 are G1, G3 (subtract); P2 is -G2 (add).
-  const float sign = r.blk == 2 ? 1.f : -1.f;
-  const int pblk = r.blk;  // partial block index equals blk
-  const int per_lane = r.len / 32;
-  // The split sum, W' = W -/+ g and both norms are formed in fp64 so that the
-  // only rounding left on Ŵ - W is the final fp32 store.
-  double wn[kMaxRowPerLane];
-  double s_old = 0.0, s_new = 0.0;
-  // Sum the S partials element by element in increasing s; the loads of one
-  // partial are issued together so the row's reads overlap.
-#pragma unroll
-  for (int k = 0; k < kMaxRowPerLane; ++k) wn[k] = 0.0;
-  for (int s = 0; s < S; ++s) {
-    const float* P = partials + (((size_t)s * H + r.head) * 3 + pblk) * mat + (size_t)r.row * r.len;
-#pragma unroll
-    for (int k = 0; k < kMaxRowPerLane; ++k)
-      if (k < per_lane) wn[k] += (double)P[lane + 32 * k];
-  }
-#pragma unroll
-  for (int k = 0; k < kMaxRowPerLane; ++k) {
-    if (k < per_lane) {
-      const double w = (double)W[base + lane + 32 * k];
-      const double wp = w + (double)sign * wn[k];
-      wn[k] = wp;
-      s_old = fma(w, w, s_old);
-      s_new = fma(wp, wp, s_new);
-    }
-  }
-  s_old = warp_sum(s_old);
-  s_new = warp_sum(s_new);
-  double scale = 1.0;
-  if (mode == 1) scale = s_new > 0.0 ? sqrt(s_old) / sqrt(s_new) : 1.0;
-  if (mode == 2 && lane == 0) {
-    scratch[2 * (size_t)warp] = s_old;
-    scratch[2 * (size_t)warp + 1] = s_new;
-  }
-  const size_t sh_off = (size_t)r.blk * H * mat;  // shadow blocks W1, W3, W2
-#pragma unroll
-  for (int k = 0; k < kMaxRowPerLane; ++k) {
-    if (k < per_lane) {
-      const int idx = lane + 32 * k;
-      const float v = (float)(wn[k] * scale);
-      Wo[base + idx] = v;
-      if (shadow != nullptr && mode != 2) shadow[sh_off + base + idx] = to_bf16_raw(v);
-    }
+  // P1, P3 are G1, G3 (subtract); P2 is -G2 (add).  Partial block = blk.
+  const double sign = r.blk == 2 ? 1.0 : -1.0;
+  const size_t sstride = (size_t)H * 3 * mat;  // one split
+  const float* P = partials + ((size_t)r.head * 3 + r.blk) * mat + (size_t)r.row * r.len;
+  // the shadow (W1 | W3 | W2 blocks) is written here unless the Frobenius
+  // scale still has to be applied
+  __nv_bfloat16_raw* sh = shadow != nullptr && mode != 2 ? shadow + (size_t)r.blk * H * mat
+                                                         : nullptr;
+  // row lengths: d or hidden of a supported shape (64, 128, 256, 512)
+  switch (r.len) {
+    case 64:
+      renorm_row<2, 1>(P + 2 * lane, sstride, S, W, Wo, base, sign, mode, warp, lane, sh, scratch);
+      break;
+    case 128:
+      renorm_row<4, 1>(P + 4 * lane, sstride, S, W, Wo, base, sign, mode, warp, lane, sh, scratch);
+      break;
+    case 256:
+      renorm_row<4, 2>(P + 4 * lane, sstride, S, W, Wo, base, sign, mode, warp, lane, sh, scratch);
+      break;
+    default:
+      renorm_row<4, 4>(P + 4 * lane, sstride, S, W, Wo, base, sign, mode, warp, lane, sh, scratch);
+      break;
   }
 }
 
