@@ -204,3 +204,21 @@ def test_gate_partial_finish_reject_bad_arguments(B):
                                None) == B.TTT_ERR_WORKSPACE
     assert L.ttt_update_finish(c, *args, 2, FAKE, FAKE, FAKE, FAKE + 2, FAKE, need,
                                None) == B.TTT_ERR_ALIGNMENT
+
+
+def test_static_stream_step_limit_and_rejection(B):
+    """ttt_stream_step_static's fixed 64 MiB scratch holds one call of up to
+    2,560 tokens for 4 heads of d = 256 (the limit the header states); a larger
+    call is rejected with TTT_ERR_WORKSPACE before anything touches a device."""
+    cfg = _cfg(B)
+    cap = 64 << 20
+    assert B.ttt_update_workspace_bytes(cfg, 2560) <= cap < B.ttt_update_workspace_bytes(cfg, 2561)
+    assert B.ttt_update_workspace_bytes(cfg, 1374) <= cap   # one 518 x 518 frame
+    L = B.lib()
+    f = L.ttt_stream_step_static
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    f.argtypes = [ctypes.POINTER(B.ttt_config), P, P, P, P, P, P, P, I64, P, I64, P, P]
+    f.restype = ctypes.c_int
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2561, FAKE, 5, FAKE, None]
+    assert f(ctypes.byref(cfg), *args) == B.TTT_ERR_WORKSPACE
+    assert f(None, *args) == B.TTT_ERR_INVALID_ARG
