@@ -342,7 +342,9 @@ cudaError_t f32_update(const Problem& p, const float* W1, const float* W2, const
                                          partials);
     }
   } else {
-    cudaMemsetAsync(partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * sizeof(float), st);
+    const cudaError_t m =
+        cudaMemsetAsync(partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * sizeof(float), st);
+    if (m != cudaSuccess) return m;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
