@@ -364,15 +364,8 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     per_launch = roof["achieved"] * (1e12 if roof["unit"] == "TFLOP/s" else 1e9) * (
         trace[dom][1] / 1e3) / max(launches, 1)
     roof["algorithmic_per_launch"] = per_launch
-    roof["traffic"] = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        with open(tp) as f:
-            tj = json.load(f)
-        ent = tj.get(dom)
-        if ent and ent.get("source_sha") == kernel_source_sha(ent.get("sources")):
-            units_per_launch = (T + M) * H / 2 if dom == "tc_apply" else T * H
-            roof["traffic"] = ent["bytes_per_unit"] * units_per_launch
+    # apply: image and ray launches alternate, so a launch averages (T + M) / 2 queries
+    roof["traffic"] = traffic_per_launch(dom, (T + M) * H / 2 if dom == "tc_apply" else T * H)
     gemm_upd_ms = trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1]
     upd_ms = gemm_upd_ms + trace.get("tc_convert_weights", (0, 0))[1] + \
         trace.get("reduce_renorm", (0, 0))[1]
@@ -531,13 +524,7 @@ def gate_probe(R, torch, dev, cfg, O, H, d, T, stream, pk, rank_max, reps: int =
     ms = rank_max(e0.elapsed_time(e1) / reps)
     by = 4.0 * T * H * d
     gbs = by / (ms / 1e3) / 1e9
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        with open(tp) as f:
-            ent = json.load(f).get("tc_gate")
-        if ent and ent.get("source_sha") == kernel_source_sha(ent.get("sources")):
-            traffic = ent["bytes_per_unit"] * T * H
+    traffic = traffic_per_launch("tc_gate", T * H)
     return {"ms_per_launch": ms, "rows": T, "achieved_gbs": gbs,
             "frac_of_hbm": gbs / pk["hbm_gbs"], "tflops": 2.0 * d * d * T * H / (ms / 1e3) / 1e12,
             "bytes_per_launch": by, "traffic": traffic}
@@ -677,6 +664,23 @@ def e2e(args, R, torch, dev, cfg, hK, hV, hQ, hQr, heta, hW, K, V, Q, Qr, eta, W
     return {"value": aggregate_value(world, T, layers, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": args.e2e_steps}
+
+
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def traffic_per_launch(kernel: str, units: float, path: str = TRAFFIC_JSON):
+    """DRAM bytes of one launch of `kernel` processing `units` token- or
+    query-heads, from the per-unit figure an ncu capture left in
+    profiles/traffic.json; None when there is no entry or the kernel sources
+    changed since the capture (their hash no longer matches)."""
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        ent = json.load(f).get(kernel)
+    if not ent or ent.get("source_sha") != kernel_source_sha(ent.get("sources")):
+        return None
+    return ent["bytes_per_unit"] * units
 
 
 def kernel_source_sha(files=None) -> str:
