@@ -156,6 +156,15 @@ def gradient_cols_w2(W1, W2, W3, K, V, eta, cols):
     return -(V * eta[:, None]).T @ u                 # [d, c]
 
 
+def gradient_rows_w2(W1, W2, W3, K, V, eta, rows):
+    """Selected rows c of G2 only (output coordinate c of the fast-weight MLP):
+    G2[c, :] = -sum_i eta_i v_i[c] u_i^T, with u_i over every hidden unit."""
+    W1, W3, K, V, eta = map(_f64, (W1, W3, K, V, eta))
+    rows = np.asarray(rows)
+    u = silu(K @ W1.T) * (K @ W3.T)                  # [n, hidden]
+    return -(V[:, rows] * eta[:, None]).T @ u        # [r, hidden]
+
+
 # --------------------------------------------------------------------------
 # Update and L2 renormalisation ([review] section 2, the two-line update after
 # Eq. 3; [survey] LaCT 架构 "L2 归一化"):

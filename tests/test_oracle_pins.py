@@ -133,6 +133,35 @@ def test_selected_rows_and_columns_match_full_gradient():
     cols = [1, 7, 14]
     np.testing.assert_allclose(O.gradient_cols_w2(W1, W2, W3, K, V, eta, cols),
                                G2[:, cols], rtol=1e-13)
+    r2 = [0, 3, 7]
+    np.testing.assert_allclose(O.gradient_rows_w2(W1, W2, W3, K, V, eta, r2), G2[r2],
+                               rtol=1e-13)
+
+
+# ------------------------------------------------------------ error measure
+def test_rel_fro_hand_computed():
+    """The parity measure ||x - ref||_F / ||ref||_F on values worked by hand:
+    the denominator is the reference's norm (not x's), both norms are square
+    roots of sums of squares over every entry, and an all-zero reference gives
+    the absolute error."""
+    # 3-4-5: x = 0 against ref = (3, 4): |x - ref| = 5, |ref| = 5
+    assert O.rel_fro([0.0, 0.0], [3.0, 4.0]) == 1.0
+    # (1, 1) vs (3, 4): sqrt(4 + 9) / 5 = sqrt(13) / 5 (a missing square root gives 13/25)
+    assert math.isclose(O.rel_fro([1.0, 1.0], [3.0, 4.0]), math.sqrt(13.0) / 5.0, rel_tol=1e-15)
+    # asymmetric: the reference's norm is the denominator
+    assert O.rel_fro([2.0, 0.0], [1.0, 0.0]) == 1.0
+    assert O.rel_fro([1.0, 0.0], [2.0, 0.0]) == 0.5
+    # matrices: the Frobenius norm runs over all entries
+    x = np.array([[1.0, 2.0], [3.0, 4.0]])
+    ref = np.array([[1.0, 2.0], [3.0, 2.0]])
+    assert math.isclose(O.rel_fro(x, ref), 2.0 / math.sqrt(18.0), rel_tol=1e-15)
+    # relative: scaling both by 1000 changes nothing
+    assert math.isclose(O.rel_fro(1e3 * x, 1e3 * ref), 2.0 / math.sqrt(18.0), rel_tol=1e-15)
+    # zero reference: the absolute error, sqrt(9 + 16)
+    assert O.rel_fro([3.0, -4.0], [0.0, 0.0]) == 5.0
+    assert O.rel_fro(np.zeros(3), np.zeros(3)) == 0.0
+    # identical inputs
+    assert O.rel_fro(x, x) == 0.0
 
 
 # ------------------------------------------------------------ invariants
