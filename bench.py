@@ -164,19 +164,49 @@ def aggregate_value(world: int, tokens: int, layers: int, ms: float) -> float:
     return world * tokens * layers / (ms / 1e3)
 
 
-def roofline_entry(name: str, flops: float, bytes_: float, ms: float, pk: dict) -> dict:
-    """Achieved rate of one kernel against the resource that bounds it: the
-    larger of flops / bf16 peak and bytes / HBM peak."""
-    t_tensor = flops / (pk["bf16_tflops_sustained"] * 1e12)
-    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
-    if t_hbm >= t_tensor:
+def kernel_work(d: int, hid: int) -> dict:
+    """Algorithmic work per unit (a token-head for the update, a query-head for
+    the apply) and the resource that bounds it.  Flops count the GEMMs (a GEMM
+    unit is 2 d hid): the update is 6 units (forward 2, backward 1, token
+    reduction 3), the apply 3.  Bytes are what the algorithm must move: the
+    update reads k, v (bf16) and eta (fp32) once, the apply reads q and writes o
+    (bf16); the intermediates (u, dh) are not algorithmic bytes.  Both are dense
+    contractions at hundreds of flop per byte, so the tensor pipe bounds them."""
+    unit = GEMM_UNIT(d, hid)
+    return {"tc_update_fused": {"bound": "tensor", "flops": 6 * unit, "bytes": 2 * d * 2 + 4},
+            "tc_apply": {"bound": "tensor", "flops": 3 * unit, "bytes": 2 * d * 2}}
+
+
+def renorm_bytes(H: int, d: int, hid: int, splits: int) -> float:
+    """Bytes one reduce + renorm launch must move: the split partials and W
+    read (fp32), W-hat written (fp32) and its bf16 shadow."""
+    mat = 3 * H * hid * d
+    return (splits + 1) * mat * 4 + mat * 4 + mat * 2
+
+
+def roofline_entry(flops: float, bytes_: float, ms: float, pk: dict, bound: str) -> dict:
+    """Achieved rate of one kernel (all its launches: `flops`, `bytes_` in `ms`)
+    against the resource its algorithm is bound by: the bf16 tensor pipe
+    (fraction of the sustained GEMM peak, the burst fraction beside it) or HBM
+    bandwidth.  A fraction above 1 means the timing or the work count is wrong:
+    it is reported as an error with frac = None, never as a rate."""
+    if bound == "tensor":
+        ach = flops / (ms / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        ent = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+               "frac": ach / peak, "peak_kind": "bf16_tflops_sustained",
+               "burst_frac": ach / pk["bf16_tflops"]}
+    else:
         ach = bytes_ / (ms / 1e3) / 1e9
-        return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "peak_kind": "hbm_gbs"}
-    ach = flops / (ms / 1e3) / 1e12
-    return {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
-            "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"],
-            "peak_kind": "bf16_tflops_sustained"}
+        peak = pk["hbm_gbs"]
+        ent = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+               "frac": ach / peak, "peak_kind": "hbm_gbs"}
+    if ent["frac"] > 1.0:
+        ent["error"] = (f"achieved {ach:.1f} {ent['unit']} is above the measured peak "
+                        f"({ent['frac']:.3f}): timing or work count wrong")
+        ent["frac"] = None
+        ent.pop("burst_frac", None)
+    return ent
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -343,45 +373,53 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
 
     # -------------------------------------------------- roofline
     pk, pk_kind = peaks()
-    unit = GEMM_UNIT(d, hid)
     reps = layers * args.steps
-    # algorithmic flops and bytes of all launches of each kernel in the timed region
-    work = {
-        "tc_fwd_bwd": (3 * unit * T * H * reps, (2 * d * 2 + 4 + 3 * hid * 2) * T * H * reps),
-        "tc_grad": (3 * unit * T * H * reps, (3 * hid * 2 + 2 * d * 2) * T * H * reps),
-        "tc_apply": (3 * unit * (T + M) * H * reps, 2 * d * 2 * (T + M) * H * reps),
-    }
+    kw = kernel_work(d, hid)
+    units = {"tc_update_fused": T * H * reps, "tc_apply": (T + M) * H * reps}
+    splits = R.ttt_update_splits(cfg, T)
     per_kernel = {k: {"launches": v[0], "ms_total": v[1], "ms_avg": v[1] / max(v[0], 1)}
                   for k, v in trace.items()}
-    for k, (fl, by) in work.items():
+    for k, ent in kw.items():
         if k in trace:
-            per_kernel[k]["roofline"] = roofline_entry(k, fl, by, trace[k][1], pk)
-    dom = max((k for k in work if k in trace), key=lambda k: trace[k][1])
+            per_kernel[k]["roofline"] = roofline_entry(ent["flops"] * units[k],
+                                                       ent["bytes"] * units[k], trace[k][1], pk,
+                                                       ent["bound"])
+    if "reduce_renorm" in trace:
+        by = renorm_bytes(H, d, hid, splits) * trace["reduce_renorm"][0]
+        per_kernel["reduce_renorm"]["roofline"] = roofline_entry(0.0, by,
+                                                                 trace["reduce_renorm"][1], pk,
+                                                                 "hbm")
+        per_kernel["reduce_renorm"]["splits"] = splits
+    dom = max((k for k in kw if k in trace), key=lambda k: trace[k][1])
     launches = trace[dom][0]
-    roof = dict(roofline_entry(dom, work[dom][0], work[dom][1], trace[dom][1], pk))
+    roof = dict(per_kernel[dom]["roofline"])
     roof["peak_kind"] += f" ({pk_kind})"
     roof["kernel"] = dom
-    per_launch = roof["achieved"] * (1e12 if roof["unit"] == "TFLOP/s" else 1e9) * (
-        trace[dom][1] / 1e3) / max(launches, 1)
-    roof["algorithmic_per_launch"] = per_launch
-    # apply: image and ray launches alternate, so a launch averages (T + M) / 2 queries
+    roof["algorithmic_per_launch"] = kw[dom]["flops"] * units[dom] / max(launches, 1)
+    roof["algorithmic_bytes_per_launch"] = kw[dom]["bytes"] * units[dom] / max(launches, 1)
+    # DRAM bytes per launch from the committed ncu capture (None if its
+    # kernel sources changed since); apply launches alternate image and ray
+    # queries, so one averages (T + M) / 2 queries
     roof["traffic"] = traffic_per_launch(dom, (T + M) * H / 2 if dom == "tc_apply" else T * H)
-    gemm_upd_ms = trace.get("tc_fwd_bwd", (0, 0))[1] + trace.get("tc_grad", (0, 0))[1]
-    upd_ms = gemm_upd_ms + trace.get("tc_convert_weights", (0, 0))[1] + \
-        trace.get("reduce_renorm", (0, 0))[1]
-    upd_flops = 6 * unit * T * H * reps
-    peak = pk["bf16_tflops_sustained"]
+    roof["traffic_over_algorithmic_bytes"] = (roof["traffic"] / roof["algorithmic_bytes_per_launch"]
+                                              if roof["traffic"] else None)
+    upd_ms = trace.get("tc_update_fused", (0, 0.0))[1]
+    upd_all_ms = upd_ms + trace.get("tc_convert_weights", (0, 0.0))[1] + \
+        trace.get("reduce_renorm", (0, 0.0))[1]
+    upd_flops = kw["tc_update_fused"]["flops"] * T * H * reps
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal q/k/v, L2-normalised per head; no dataset)",
             "config": workload_config(w, layers), "roofline": roof,
             "update_gemm_tensor_frac": {
-                "value": upd_flops / (gemm_upd_ms / 1e3) / 1e12 / peak if gemm_upd_ms else None,
+                "value": upd_flops / (upd_ms / 1e3) / 1e12 / pk["bf16_tflops_sustained"]
+                if upd_ms else None,
                 "of": "bf16_tflops_sustained",
-                "burst_frac": (upd_flops / (gemm_upd_ms / 1e3) / 1e12 / pk["bf16_tflops"]
-                               if gemm_upd_ms else None),
-                "update_ms_per_layer": upd_ms / (layers * args.steps)},
+                "burst_frac": (upd_flops / (upd_ms / 1e3) / 1e12 / pk["bf16_tflops"]
+                               if upd_ms else None),
+                "update_gemm_ms_per_layer": upd_ms / reps,
+                "update_ms_per_layer": upd_all_ms / reps},
             "kernels": per_kernel, "clocks": clk,
             "gpu_launches": int(sum(v[0] for v in trace.values()))}
     if args.ns_steps:

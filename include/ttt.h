@@ -102,6 +102,12 @@ size_t ttt_update_workspace_bytes(const ttt_config* cfg, int64_t n_tokens);
 /* Bytes of the bf16 weight shadow (3 * H * d * hidden * 2). */
 size_t ttt_shadow_bytes(const ttt_config* cfg);
 
+/* Number of token splits S the update of n tokens reduces: the gradient is
+ * accumulated as S fp32 partials over contiguous token ranges (a function of
+ * cfg and n only), summed in increasing split order before the
+ * renormalisation.  The workspace holds them.  0 if the config is invalid. */
+int32_t ttt_update_splits(const ttt_config* cfg, int64_t n_tokens);
+
 /*
  * One TTT update of all heads (Eq. 1–3 and the renormalisation above):
  *   g = ∇_W Σ_{i<n} η_i (−f_W(k_i)^T v_i),  Ŵ = renorm(W − Δ),
@@ -258,15 +264,25 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
  * frame arrives (fixed memory budgets, allocator owned by another runtime, no
  * cudaMalloc after start-up).  The call allocates nothing.
  *  - Returns TTT_ERR_WORKSPACE, before launching anything, when
- *    ttt_update_workspace_bytes(cfg, n) exceeds TTT_STATIC_SCRATCH_BYTES
- *    (with 4 heads of d = 256, hidden 512 that is 2,560 tokens per call;
- *    one 518 x 518 frame is 1,374).
+ *    ttt_update_workspace_bytes(cfg, n) exceeds TTT_STATIC_SCRATCH_BYTES.
+ *    The limit depends on the configuration.  BF16_TC keeps the update's
+ *    intermediates on chip, so its workspace stops growing with n: with 4
+ *    heads of d = 256, hidden 512 every n fits (19.0 MB with ns_steps = 0,
+ *    63.0 MB with ns_steps > 0); for every n, up to 42 such heads fit with
+ *    ns_steps = 0 and 4 with ns_steps > 0.  FP32_CHECK keeps per-token
+ *    intermediates: 4 heads of d = 256 fit up to 2,471 tokens per call with
+ *    ns_steps = 0 and 678 with ns_steps > 0 (one 518 x 518 frame is 1,374
+ *    tokens).
  *  - Every GPU that loads the library may hold the array until exit.
  *  - All calls on a device share the array and it keeps the last call's
  *    contents (nothing in it has to start at zero); calls that can overlap on
  *    the GPU race on it and must be serialised by the caller.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    (cudaGetSymbolAddress) and caches it with the id of the device's current
+ *    context; a call after the context changed (cudaDeviceReset, or the
+ *    primary context released and created again) looks it up anew.  Make
+ *    such a call (the first on each device, and the first after a reset)
+ *    before any stream capture.
  */
 #define TTT_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
 ttt_status ttt_stream_step_static(const ttt_config* cfg,

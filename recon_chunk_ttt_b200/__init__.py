@@ -20,7 +20,7 @@ _EXPORTS = {
     "PREC_FP32_CHECK", "LIB_PATH", "ttt_trace_enable", "ttt_trace_read",
     "ttt_stream_step_static", "MAX_NS_STEPS", "ttt_chunked", "ORDER_UPDATE_THEN_APPLY",
     "ORDER_APPLY_THEN_UPDATE", "ttt_partial_floats", "ttt_finish_workspace_bytes",
-    "ttt_update_partial", "ttt_update_finish", "ttt_gate", "GATE_EPS",
+    "ttt_update_partial", "ttt_update_finish", "ttt_gate", "GATE_EPS", "ttt_update_splits",
     "ttt_selftest_wait_timeout", "DEVICE_ERR_SELFTEST", "TTT_OK", "TTT_ERR_INVALID_ARG",
     "TTT_ERR_UNSUPPORTED_SHAPE", "TTT_ERR_ALIGNMENT", "TTT_ERR_WORKSPACE", "TTT_ERR_CUDA",
     "TTT_ERR_DEVICE",

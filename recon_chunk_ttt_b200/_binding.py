@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_gate.restype = ctypes.c_int
         L.ttt_partial_floats.argtypes = [_CFG]
         L.ttt_partial_floats.restype = ctypes.c_size_t
+        L.ttt_update_splits.argtypes = [_CFG, _I64]
+        L.ttt_update_splits.restype = ctypes.c_int32
         L.ttt_finish_workspace_bytes.argtypes = [_CFG]
         L.ttt_finish_workspace_bytes.restype = ctypes.c_size_t
         L.ttt_update_partial.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _I64, _P, _P,
@@ -219,6 +221,10 @@ def ttt_gate(cfg: ttt_config, Wg, O_prime, O=None, stream=None):
 
 def ttt_partial_floats(cfg: ttt_config) -> int:
     return int(lib().ttt_partial_floats(ctypes.byref(cfg)))
+
+
+def ttt_update_splits(cfg: ttt_config, n_tokens: int) -> int:
+    return int(lib().ttt_update_splits(ctypes.byref(cfg), n_tokens))
 
 
 def ttt_finish_workspace_bytes(cfg: ttt_config) -> int:

@@ -73,6 +73,14 @@ cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const 
                       float* partial_out = nullptr);
 cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,
                      cudaStream_t st);
+// Fused update kernel (kernels_fused.cu): fp32 weights W1, W3 [H][hid][d],
+// W2 [H][d][hid] in (rounded to bf16 inside); the S split partials of the
+// plan out.
+cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, const float* W3,
+                         const void* K, const void* V, const float* eta, int S, int64_t chunk,
+                         float* partials, int* err, cudaStream_t st);
+// Clusters of the fused update that fill one wave of the GPU.
+int fused_clusters_per_wave();
 
 // ---- gated output unit: o = RMSNorm(o') * SiLU(W_g o') per head ------------
 // p.n = rows.  W_g [H][d][d] (row = output); bf16 (tc) or float (f32).

@@ -1,0 +1,706 @@
+// Fused TTT update on sm_100a: forward, backward and token-reduction GEMMs of
+// one gradient step in one clustered kernel, with the η-scaled intermediates
+// kept on chip (kimjy99 ZipMap review, section 2 "Feature Backbone", Eq. 1-3):
+//
+//   h1 = W1 k, h3 = W3 k, u = SiLU(h1) ⊙ h3, du = -W2^T v,
+//   dh3 = du ⊙ SiLU(h1), dh1 = du ⊙ h3 ⊙ SiLU'(h1),
+//   G1 = Σ_i η_i dh1_i k_i^T,  G3 = Σ_i η_i dh3_i k_i^T,  P2 = Σ_i η_i u_i v_i^T (= -G2^T).
+//
+// A cluster of three CTAs (one per SM) owns one head, one group of 128 hidden
+// units and one contiguous token range (a split).  Per 128-token tile:
+//   ranks 0 and 1 ("F", hidden units 64r .. 64r+63 of the group)
+//     F    = K [W1s; W3s]^T            M = 128 tokens, N = 128, into TMEM (2 buffers)
+//     epilogue: with du from rank 2, η·u (bf16) goes to rank 2, η·dh1 and η·dh3
+//     (bf16) to this CTA's shared memory
+//     G13 += [η·dh1 | η·dh3]^T K       M = 128 (64 dh1 rows, 64 dh3 rows), N = d, in TMEM
+//   rank 2 ("D", all 128 hidden units of the group)
+//     DU   = V W2s^T                   M = 128 tokens, N = 128, into TMEM (2 buffers)
+//     epilogue: du (bf16) to ranks 0 and 1
+//     P2  += (η·u)^T V                 M = 128 hidden, N = d, in TMEM
+// The gradient MMAs of tile i run after the forward MMAs of tile i+1, so the
+// epilogues and exchanges of a tile overlap the next tile's MMAs.  At the end
+// each CTA writes its slice of the split's fp32 partial ([S][H][3][hid*d],
+// blocks G1, G3, P2 as [d][hid]); a fixed-order reduction over the splits
+// follows in another kernel, so results are bitwise reproducible.
+//
+// The exchanges are bulk copies (cp.async.bulk shared::cta -> shared::cluster)
+// from a staging buffer of the sender into the receiver's operand buffer,
+// completing on the receiver's mbarrier; the receiver frees the buffer by a
+// remote mbarrier arrive (rank 2's MMA by a tcgen05.commit to ranks 0 and 1).
+// No TMA load uses multicast.  Every wait is bounded; a CTA that gives up sets
+// the abort flag of all three CTAs and the device error word.
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_util.cuh"
+
+namespace ttt {
+
+namespace {
+
+template <int D>
+struct FU {
+  static constexpr int NCH = D / CH;            // 64-wide d chunks
+  static constexpr int GH = 128;                // hidden units per cluster
+  static constexpr int FH = 64;                 // hidden units per F CTA
+  static constexpr int TKG = 32;                // tokens per gradient stage
+  static constexpr int NKF = 3;                 // forward ring: [128 tokens x 64 d] stages
+  static constexpr int NKG = 3;                 // gradient ring: [32 tokens x d] stages
+  static constexpr int CHUNK = BM * 128;        // 16 KB
+  static constexpr int KG_STAGE = TKG * D * 2;
+  static constexpr int XB = BM * 128;           // exchange block: 128 tokens x 64 bf16 (16 KB)
+  static constexpr int W2BLK = D * 128;         // D: one block of 64 hidden units x d rows
+  // F: NCH K-major chunks of [128 rows (64 of W1, 64 of W3) x 64 d];
+  // D: 2 MN-major blocks of [d rows x 64 hidden units] of W2 (same bytes)
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_KF = OFF_W + NCH * CHUNK;
+  static constexpr int OFF_KG = OFF_KF + NKF * CHUNK;
+  static constexpr int OFF_GA = OFF_KG + NKG * KG_STAGE;  // A of the gradient MMA: 2 blocks
+  static constexpr int OFF_EX = OFF_GA + 2 * XB;          // F: du in | η·u out; D: du out x 2
+  static constexpr int OFF_BAR = OFF_EX + 2 * XB;
+  static constexpr int NBAR = 2 * NKF + 2 * NKG + 16;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + tmem slot, abort, alignment
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static constexpr int EPI_WARPS = 16;          // four per TMEM lane quadrant
+  static constexpr int EPI_THREADS = 32 * EPI_WARPS;
+  // kf producer, MMA, kg producer, epilogue warps, then one signalling warp
+  static constexpr int THREADS = 96 + EPI_THREADS + 32;
+  static constexpr int SIGNAL_WARP = 3 + EPI_WARPS;
+  static constexpr uint32_t TMEM_COLS = 512;    // forward buffers at 0 and 128, gradient at 256
+  static constexpr uint32_t TM_G = 256;
+};
+
+// Barrier slots (same offsets in every CTA of the cluster, so a multicast
+// commit and the remote arrives find them).
+template <int D>
+struct Bars {
+  uint64_t* base;
+  __device__ uint64_t* kf_full(int s) { return base + s; }
+  __device__ uint64_t* kf_empty(int s) { return base + FU<D>::NKF + s; }
+  __device__ uint64_t* kg_full(int s) { return base + 2 * FU<D>::NKF + s; }
+  __device__ uint64_t* kg_empty(int s) { return base + 2 * FU<D>::NKF + FU<D>::NKG + s; }
+  __device__ uint64_t* x(int i) { return base + 2 * FU<D>::NKF + 2 * FU<D>::NKG + i; }
+  __device__ uint64_t* w_full() { return x(0); }
+  __device__ uint64_t* acc_full(int b) { return x(1 + b); }
+  __device__ uint64_t* acc_empty(int b) { return x(3 + b); }
+  __device__ uint64_t* ga_full() { return x(5); }     // F: η·dh1|η·dh3 written; D: η·u arrived
+  __device__ uint64_t* ga_empty() { return x(6); }    // F: G13 of the tile done
+  __device__ uint64_t* g_full() { return x(7); }      // last gradient MMA done
+  __device__ uint64_t* done() { return x(8); }
+  __device__ uint64_t* au_empty() { return x(9); }    // F: rank 2's P2 read the η·u block
+  __device__ uint64_t* du_full() { return x(10); }    // F: du of the tile arrived
+  __device__ uint64_t* du_empty(int f) { return x(11 + f); }  // D: rank f read its du
+  __device__ uint64_t* du_read() { return x(13); }    // F: every epilogue warp read du
+};
+
+// Give up: device error word, and the abort flag of every CTA of the cluster.
+__device__ __forceinline__ void cluster_abort(volatile int* abort, int* err, int reason) {
+  atomicExch(err, reason);
+  const uint32_t a = smem_u32(const_cast<int*>(abort));
+#pragma unroll
+  for (uint32_t r = 0; r < 3; ++r)
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(a, r)), "r"(1) : "memory");
+}
+
+// Bounded wait on a local mbarrier.  On a time-out the reason goes to the
+// device error word and the abort flag of every CTA of the cluster is set, so
+// the others leave their waits at once.  kCluster: arrivals may come from
+// other CTAs (acquire at cluster scope).
+template <bool kCluster>
+__device__ __forceinline__ bool cwait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                      int* err, int reason) {
+  auto probe = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (probe()) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (probe()) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      cluster_abort(abort, err, reason);
+      return false;
+    }
+  }
+}
+
+// Final waits before the CTA may leave: bounded, not cut short by the abort
+// flag, so no asynchronous arrival can still be on its way here.
+__device__ __forceinline__ void final_wait(uint64_t* bar, uint32_t parity, int* err) {
+  volatile int never = 0;
+  cwait<true>(bar, parity, &never, err, kErrWaitFinal);
+}
+
+template <int D>
+__global__ void __launch_bounds__(FU<D>::THREADS, 1)
+    fused_update_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+                        const __grid_constant__ CUtensorMap mKg,
+                        const __grid_constant__ CUtensorMap mVg,
+                        const float* __restrict__ W1, const float* __restrict__ W2,
+                        const float* __restrict__ W3, const float* __restrict__ eta,
+                        int64_t n, int H, int hid, int S, int64_t chunk,
+                        float* __restrict__ partials, int* err) {
+  using L = FU<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Bars<D> bar{reinterpret_cast<uint64_t*>(smem + L::OFF_BAR)};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_BAR + L::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int rank = (int)cluster_ctarank();
+  const bool isF = rank < 2;
+  // Work item: (head, hidden group, split)
+  const int groups = hid / L::GH;
+  const int item = blockIdx.x / 3;
+  const int g = item / S, s = item % S;
+  const int head = g / groups, grp = g % groups;
+  const int64_t ntiles_all = (n + BM - 1) / BM;
+  const int64_t t0 = (int64_t)s * chunk / BM;
+  int64_t t1 = ((int64_t)s + 1) * chunk / BM;
+  if (t1 > ntiles_all) t1 = ntiles_all;
+  const int nt = t1 > t0 ? (int)(t1 - t0) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NKF; ++i) {
+      mbar_init(bar.kf_full(i), 1);
+      mbar_init(bar.kf_empty(i), 1);
+    }
+    for (int i = 0; i < L::NKG; ++i) {
+      mbar_init(bar.kg_full(i), 1);
+      mbar_init(bar.kg_empty(i), 1);
+    }
+    mbar_init(bar.w_full(), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar.acc_full(b), 1);
+      mbar_init(bar.acc_empty(b), L::EPI_WARPS);
+    }
+    mbar_init(bar.ga_full(), 1);
+    mbar_init(bar.ga_empty(), 1);
+    mbar_init(bar.g_full(), 1);
+    mbar_init(bar.done(), 1);
+    mbar_init(bar.au_empty(), 1);
+    mbar_init(bar.du_full(), 1);
+    mbar_init(bar.du_empty(0), 1);
+    mbar_init(bar.du_empty(1), 1);
+    mbar_init(bar.du_read(), L::EPI_WARPS);
+    *abort_flag = 0;
+    fence_mbar_init();
+    // Receivers arm their own exchange barriers (the senders' bulk copies
+    // only complete bytes): F expects its du block, D both η·u blocks.
+    if (nt > 0) {
+      if (isF)
+        mbar_arrive_expect_tx(bar.du_full(), L::XB);
+      else
+        mbar_arrive_expect_tx(bar.ga_full(), 2 * L::XB);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  // every CTA's barriers exist before any remote arrive or copy targets them
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ weights + forward ring
+    const CUtensorMap* m = isF ? &mK : &mV;
+    tma_prefetch_desc(m);
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i) {
+      const int y = (int)((t0 + i) * BM);
+      for (int c = 0; c < L::NCH; ++c) {
+        if (!cwait<false>(bar.kf_empty(stage), phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar.kf_full(stage), L::CHUNK);
+        TTT_DCHECK((int64_t)y < n && head * L::NCH + c < H * L::NCH, err, kErrCheckTma);
+        tma_load_3d(smem + L::OFF_KF + stage * L::CHUNK, m, bar.kf_full(stage), 0, y,
+                    head * L::NCH + c);
+        ++issued;
+        if (++stage == L::NKF) { stage = 0; phase ^= 1; }
+      }
+    }
+    drain_ring(bar.kf_full(0), L::NKF, issued, err);
+  } else if (warp == 2 && lane == 0) {
+    // ------------------------------------------------ gradient ring
+    const CUtensorMap* m = isF ? &mKg : &mVg;
+    tma_prefetch_desc(m);
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i) {
+      const int y = (int)((t0 + i) * BM);
+      for (int st = 0; st < BM / L::TKG; ++st) {
+        if (!cwait<false>(bar.kg_empty(stage), phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar.kg_full(stage), L::KG_STAGE);
+        TTT_DCHECK((int64_t)(y + st * L::TKG) < n + BM && head < H, err, kErrCheckTma);
+        // one box: NCH d-chunks x [TKG tokens x 64 d]
+        tma_load_3d(smem + L::OFF_KG + stage * L::KG_STAGE, m, bar.kg_full(stage), 0,
+                    y + st * L::TKG, head * L::NCH);
+        ++issued;
+        if (++stage == L::NKG) { stage = 0; phase ^= 1; }
+      }
+    }
+    drain_ring(bar.kg_full(0), L::NKG, issued, err);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    // F: B = [W1s; W3s] rows, K-major; D: B = W2 columns of the group,
+    // MN-major (two blocks of 64 hidden units x d rows)
+    const uint32_t idF = idesc_bf16_f32(BM, 128, false, !isF);
+    const uint32_t idG = idesc_bf16_f32(BM, D, true, true);
+    const uint32_t sbase = smem_u32(smem);
+    bool ok = nt == 0 || cwait<false>(bar.w_full(), 0, abort_flag, err, kErrWaitFull);
+    // Forward MMAs of tile fi (one 64-d chunk per issue) and gradient MMAs of
+    // tile gj (one TKG-token stage per issue) are interleaved as their operands
+    // arrive, alternating when both are ready, so both operand rings drain at
+    // an even rate.  Each accumulator still receives its MMAs in one fixed
+    // order (chunks, stages and tiles ascending): the result does not depend
+    // on the interleaving.  Barriers are polled without blocking; the whole
+    // loop gives up after kWaitLimitCycles without progress.
+    int fi = 0, fc = 0, gj = 0, gst = 0;
+    bool f_open = false, g_open = false, prefer_g = true;
+    int fs = 0, gs = 0;
+    uint32_t fph = 0, gph = 0;
+    long long last = clock64();
+    const uint32_t ga = sbase + L::OFF_GA;
+    while (ok && gj < nt) {
+      bool issued = false;
+      for (int pass = 0; pass < 2 && !issued; ++pass) {
+        const bool try_g = (pass == 0) == prefer_g;
+        if (try_g) {
+          if (gj >= fi) continue;  // tile gj's forward MMAs are not all issued yet
+          if (!g_open) {
+            const bool r = isF ? mbar_test_wait(bar.ga_full(), (uint32_t)(gj & 1))
+                               : mbar_test_wait_cluster(bar.ga_full(), (uint32_t)(gj & 1));
+            if (!r) continue;
+            g_open = true;
+            if (!isF && gj + 1 < nt) mbar_arrive_expect_tx(bar.ga_full(), 2 * L::XB);
+          }
+          if (!mbar_test_wait(bar.kg_full(gs), gph)) continue;
+          tc_fence_after();
+          const uint32_t kg = sbase + L::OFF_KG + gs * L::KG_STAGE;
+#pragma unroll
+          for (int kk = 0; kk < L::TKG / 16; ++kk) {
+            // A: MN-major, 2 blocks of 64 rows (LBO), 16 tokens per K step;
+            // B: MN-major, NCH blocks of 64 d (LBO = TKG rows x 128 B)
+            const uint64_t da = sdesc_sw128(ga + (gst * L::TKG + kk * 16) * 128, L::XB, 1024);
+            const uint64_t db = sdesc_sw128(kg + kk * 16 * 128, L::TKG * 128, 1024);
+            umma_bf16(tmem + L::TM_G, da, db, idG, (gj | gst | kk) != 0);
+          }
+          umma_commit(bar.kg_empty(gs));
+          if (++gs == L::NKG) { gs = 0; gph ^= 1; }
+          if (++gst == BM / L::TKG) {
+            if (isF)
+              umma_commit(bar.ga_empty());
+            else
+              umma_commit_cluster(bar.au_empty(), (uint16_t)0x3);  // ranks 0 and 1 may refill
+            gst = 0;
+            ++gj;
+            g_open = false;
+          }
+          issued = true;
+          prefer_g = false;
+        } else {
+          if (fi >= nt) continue;
+          if (!f_open) {
+            if (!mbar_test_wait(bar.acc_empty(fi & 1), (uint32_t)(((fi >> 1) & 1) ^ 1))) continue;
+            f_open = true;
+          }
+          if (!mbar_test_wait(bar.kf_full(fs), fph)) continue;
+          tc_fence_after();
+          const uint32_t a = sbase + L::OFF_KF + fs * L::CHUNK;
+          const uint32_t dF = tmem + (fi & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < CH / 16; ++kk) {
+            const uint64_t db =
+                isF ? sdesc_sw128(sbase + L::OFF_W + fc * L::CHUNK + kk * KSTEP_BYTES, 16, 1024)
+                    : sdesc_sw128(sbase + L::OFF_W + (fc * CH + kk * 16) * 128, L::W2BLK, 1024);
+            umma_bf16(dF, sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024), db, idF, (fc | kk) != 0);
+          }
+          umma_commit(bar.kf_empty(fs));
+          if (++fs == L::NKF) { fs = 0; fph ^= 1; }
+          if (++fc == L::NCH) {
+            umma_commit(bar.acc_full(fi & 1));
+            fc = 0;
+            ++fi;
+            f_open = false;
+          }
+          issued = true;
+          prefer_g = true;
+        }
+      }
+      if (issued) {
+        last = clock64();
+      } else if (*abort_flag) {
+        ok = false;
+      } else if (clock64() - last > kWaitLimitCycles) {
+        cluster_abort(abort_flag, err, kErrWaitOperand);
+        ok = false;
+      }
+    }
+    umma_commit(bar.g_full());
+    umma_commit(bar.done());
+    volatile int never = 0;
+    mbar_wait(bar.done(), 0, &never, err, kErrWaitFinal);
+  } else if (warp == L::SIGNAL_WARP) {
+    // ------------------------------------------------ F: du consumed -> rank 2
+    // A remote arrive with cluster-scope release costs about a microsecond on
+    // the issuing thread; this warp pays it so the epilogue does not.
+    if (isF && lane == 0) {
+      const uint32_t c_du_empty = mapa_shared(smem_u32(bar.du_empty(rank)), 2);
+      for (int i = 0; i < nt; ++i) {
+        if (!cwait<false>(bar.du_read(), (uint32_t)(i & 1), abort_flag, err, kErrWaitOperand))
+          break;
+        mbar_arrive_remote(c_du_empty);
+      }
+    }
+  } else if (warp >= 3) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;              // TMEM lane quadrant of this warp
+    const int h = (warp - 3) >> 2;       // column quarter
+    const int row = q * 32 + lane;       // token row (tiles) / accumulator row (gradient)
+    const bool leader = warp == 3 && lane == 0;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint8_t* ga = smem + L::OFF_GA;
+    uint8_t* ex = smem + L::OFF_EX;
+    bool ok = true;
+    if (nt > 0) {
+      // This CTA's weights, fp32 -> bf16 (round to nearest) into the swizzled
+      // operand layout; 16-byte granule g of a 128-byte row r sits at g ^ (r % 8).
+      const int et = threadIdx.x - 96;
+      const size_t mat = (size_t)hid * D;
+      if (isF) {
+        // rows 0..63: W1, 64..127: W3 (hidden units of this CTA); a warp reads
+        // one d-row of 32 granules (D = 256) at a time
+        constexpr int GPR = D / 8;  // granules per weight row
+        for (int i = et; i < 2 * L::FH * GPR; i += L::EPI_THREADS) {
+          const int r = i / GPR, gg = i % GPR, c = gg / 8, g = gg % 8;
+          const float* src = (r < L::FH ? W1 : W3) + (size_t)head * mat +
+                             (size_t)(grp * L::GH + rank * L::FH + (r % L::FH)) * D + gg * 8;
+          const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+          const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+          *reinterpret_cast<uint4*>(smem + L::OFF_W + c * L::CHUNK + r * 128 + ((g ^ (r & 7)) * 16)) =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                         pack_bf16x2(b.z, b.w));
+        }
+      } else {
+        // W2[head][c][grp*128 + j]: d-row c, hidden units j of the group, as
+        // two blocks of 64 units; a half-warp reads one d-row (512 bytes)
+        for (int i = et; i < D * (L::GH / 8); i += L::EPI_THREADS) {
+          const int c = i / (L::GH / 8), gg = i % (L::GH / 8), blk = gg / 8, g = gg % 8;
+          const float* src = W2 + (size_t)head * mat + (size_t)c * hid + grp * L::GH + gg * 8;
+          const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+          const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+          *reinterpret_cast<uint4*>(smem + L::OFF_W + blk * L::W2BLK + c * 128 + ((g ^ (c & 7)) * 16)) =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                         pack_bf16x2(b.z, b.w));
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, L::EPI_THREADS);
+      if (leader) mbar_arrive(bar.w_full());
+    }
+    if (isF) {
+      // remote addresses in rank 2
+      const uint32_t c_au_full = mapa_shared(smem_u32(bar.ga_full()), 2);
+      const uint32_t c_au_dst = mapa_shared(smem_u32(ga + rank * L::XB), 2);
+      uint8_t* du_in = ex;
+      uint8_t* au_out = ex + L::XB;
+      // η of this thread's token row, one tile ahead (its load latency is not
+      // on the per-tile path)
+      auto eta_of = [&](int i) -> float {
+        const int64_t tok = (t0 + i) * BM + row;
+        return i < nt && tok < n ? __ldg(&eta[tok * H + head]) : 0.f;
+      };
+      float eta_next = eta_of(0);
+      for (int i = 0; i < nt; ++i) {
+        const int b = i & 1;
+        const float ne = -eta_next;  // -η (du = -W2^T v)
+        eta_next = eta_of(i + 1);
+        bool got = cwait<false>(bar.acc_full(b), (uint32_t)((i >> 1) & 1), abort_flag, err,
+                                kErrWaitAcc);
+        __syncwarp();
+        if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
+        tc_fence_after();
+        // h1, h3 of this row for hidden units [16h, 16h + 16) of this CTA
+        uint32_t r1[16], r3[16];
+        const uint32_t tl = tmem + lane_base + b * 128 + h * 16;
+        tmem_ld_16x(tl, r1);
+        tmem_ld_16x(tl + L::FH, r3);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar.acc_empty(b));
+        // η·u needs no du: form it, keep SiLU(h1) and h3·SiLU'(h1) for later
+        float sa[16], shd[16];
+        uint32_t pu[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float o_u[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const float h1 = __uint_as_float(r1[e + t]);
+            const float h3 = __uint_as_float(r3[e + t]);
+            const float sg = sigmoid_fast(h1);
+            const float a = h1 * sg;                         // SiLU(h1)
+            sa[e + t] = a;
+            shd[e + t] = h3 * fmaf(-a, sg, a + sg);          // h3·SiLU'(h1), SiLU' = s + a(1 - s)
+            o_u[t] = -ne * (a * h3);
+          }
+          pu[e / 2] = pack_bf16x2(o_u[0], o_u[1]);
+        }
+        // η·u to rank 2, once the previous copy has read the staging buffer
+        if (leader) bulk_wait_group_read0();
+        named_bar_sync(1, L::EPI_THREADS);
+        {
+          uint8_t* r_u = au_out + row * 128;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            *reinterpret_cast<uint4*>(r_u + (((2 * h + c) ^ (row & 7)) * 16)) =
+                make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, L::EPI_THREADS);
+        if (leader) {
+          // rank 2's P2 of the previous tile has read its η·u block
+          if (i >= 1 && !cwait<true>(bar.au_empty(), (uint32_t)((i - 1) & 1), abort_flag, err,
+                                     kErrWaitOperand)) {
+            ok = false;
+          } else {
+            bulk_copy_to_cluster(c_au_dst, au_out, L::XB, c_au_full);
+            bulk_commit_group();
+          }
+        }
+        // du of this tile from rank 2
+        got = cwait<true>(bar.du_full(), (uint32_t)(i & 1), abort_flag, err, kErrWaitOperand);
+        __syncwarp();
+        if (named_bar_any(1, L::EPI_THREADS, !got || !ok)) { ok = false; break; }
+        // every epilogue thread is past this phase: arm the next tile's du
+        if (leader && i + 1 < nt) mbar_arrive_expect_tx(bar.du_full(), L::XB);
+        uint32_t dv[8];
+        {
+          const uint8_t* rp = du_in + row * 128;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 t = *reinterpret_cast<const uint4*>(rp + (((2 * h + c) ^ (row & 7)) * 16));
+            dv[4 * c] = t.x; dv[4 * c + 1] = t.y; dv[4 * c + 2] = t.z; dv[4 * c + 3] = t.w;
+          }
+        }
+        uint32_t p1[8], p3[8];  // η·dh1, η·dh3 as packed bf16 pairs
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(&dv[e / 2]);
+          const float e0 = ne * __low2float(d2), e1 = ne * __high2float(d2);  // η du
+          p1[e / 2] = pack_bf16x2(e0 * shd[e], e1 * shd[e + 1]);
+          p3[e / 2] = pack_bf16x2(e0 * sa[e], e1 * sa[e + 1]);
+        }
+        // du consumed (its values are in registers): the signalling warp
+        // tells rank 2, off this path
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar.du_read());
+        // G13 of the previous tile has read the operand buffer
+        if (i >= 1) {
+          got = cwait<false>(bar.ga_empty(), (uint32_t)((i - 1) & 1), abort_flag, err,
+                             kErrWaitOperand);
+          __syncwarp();
+          if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
+        }
+        {
+          uint8_t* r_1 = ga + row * 128;
+          uint8_t* r_3 = ga + L::XB + row * 128;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int pos = ((2 * h + c) ^ (row & 7)) * 16;
+            *reinterpret_cast<uint4*>(r_1 + pos) =
+                make_uint4(p1[4 * c], p1[4 * c + 1], p1[4 * c + 2], p1[4 * c + 3]);
+            *reinterpret_cast<uint4*>(r_3 + pos) =
+                make_uint4(p3[4 * c], p3[4 * c + 1], p3[4 * c + 2], p3[4 * c + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, L::EPI_THREADS);
+        if (leader) mbar_arrive(bar.ga_full());
+      }
+      if (leader) {
+        bulk_wait_group0();
+        // the last multicast arrive from rank 2 has landed before this CTA may go
+        if (ok && nt > 0) final_wait(bar.au_empty(), (uint32_t)((nt - 1) & 1), err);
+      }
+    } else {
+      // rank 2: du of each tile to ranks 0 and 1
+      const uint32_t c_du_full[2] = {mapa_shared(smem_u32(bar.du_full()), 0),
+                                     mapa_shared(smem_u32(bar.du_full()), 1)};
+      const uint32_t c_du_dst[2] = {mapa_shared(smem_u32(ex), 0), mapa_shared(smem_u32(ex), 1)};
+      for (int i = 0; i < nt; ++i) {
+        const int b = i & 1;
+        bool got = cwait<false>(bar.acc_full(b), (uint32_t)((i >> 1) & 1), abort_flag, err,
+                                kErrWaitAcc);
+        __syncwarp();
+        if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
+        tc_fence_after();
+        // DU of this row for hidden units [32h, 32h + 32) of the group: rank h / 2's
+        // units [32(h % 2), 32(h % 2) + 32)
+        uint32_t r0[32];
+        tmem_ld_32x32(tmem + lane_base + b * 128 + h * 32, r0);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar.acc_empty(b));
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+        if (leader) bulk_wait_group_read0();
+        named_bar_sync(1, L::EPI_THREADS);
+        {
+          uint8_t* rp = ex + (h >> 1) * L::XB + row * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(rp + (((4 * (h & 1) + c) ^ (row & 7)) * 16)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, L::EPI_THREADS);
+        if (leader) {
+          for (int f = 0; f < 2 && ok; ++f) {
+            // rank f has read its previous du block
+            if (i >= 1 && !cwait<true>(bar.du_empty(f), (uint32_t)((i - 1) & 1), abort_flag, err,
+                                       kErrWaitOperand)) {
+              ok = false;
+              break;
+            }
+            bulk_copy_to_cluster(c_du_dst[f], ex + f * L::XB, L::XB, c_du_full[f]);
+          }
+          bulk_commit_group();
+        }
+        if (named_bar_any(1, L::EPI_THREADS, !ok)) { ok = false; break; }
+      }
+      if (leader) bulk_wait_group0();
+    }
+    // ---------------------------------------------- gradient partial
+    const bool have = ok && nt > 0 &&
+                      cwait<false>(bar.g_full(), 0, abort_flag, err, kErrWaitAcc);
+    __syncwarp();
+    tc_fence_after();
+    const size_t mat = (size_t)hid * D;
+    if (ok) {
+      if (isF) {
+        // lanes 0..63: G1 rows, 64..127: G3 rows of this CTA's 64 hidden units
+        const int blk = q < 2 ? 0 : 1;
+        const int hrow = grp * L::GH + rank * L::FH + (q & 1) * 32 + lane;
+        float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat + (size_t)hrow * D;
+        TTT_DCHECK(hrow < hid, err, kErrCheckIndex);
+        for (int c0 = h * (D / 4); c0 < (h + 1) * (D / 4); c0 += 16) {
+          uint32_t rr[16];
+          if (have) {
+            tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) rr[e] = 0u;
+          }
+          float4* dst = reinterpret_cast<float4*>(P + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
+                                 __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
+        }
+      } else {
+        // P2 rows = hidden units of the group, stored transposed as [d][hid]
+        const int j = grp * L::GH + row;
+        float* P = partials + (((size_t)s * H + head) * 3 + 2) * mat;
+        TTT_DCHECK(j < hid, err, kErrCheckIndex);
+        for (int c0 = h * (D / 4); c0 < (h + 1) * (D / 4); c0 += 16) {
+          uint32_t rr[16];
+          if (have) {
+            tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) rr[e] = 0u;
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) P[(size_t)(c0 + e) * hid + j] = __uint_as_float(rr[e]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // no CTA leaves while another may still copy into or arrive on it
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2,
+                              const float* W3, const void* K, const void* V, const float* eta,
+                              int S, int64_t chunk, float* partials, int* err, cudaStream_t st) {
+  using L = FU<D>;
+  CUtensorMap mK, mV, mKg, mVg;
+  const uint64_t ld = (uint64_t)p.H * D;
+  {
+    // {64 d, tokens, d-chunks of all heads}
+    const uint64_t dims[3] = {(uint64_t)CH, (uint64_t)p.n, ld / CH};
+    const uint64_t str[2] = {ld * 2, CH * 2};
+    const uint32_t boxf[3] = {CH, BM, 1};
+    const uint32_t boxg[3] = {CH, L::TKG, (uint32_t)L::NCH};
+    if (!make_map(&mK, K, 3, dims, str, boxf) || !make_map(&mV, V, 3, dims, str, boxf) ||
+        !make_map(&mKg, K, 3, dims, str, boxg) || !make_map(&mVg, V, 3, dims, str, boxg))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = ensure_smem_attr(fused_update_kernel<D>, L::SMEM);
+  if (e != cudaSuccess) return e;
+  const int G = p.H * (p.hid / L::GH);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(3 * G * S));
+  cfg.blockDim = dim3(L::THREADS);
+  cfg.dynamicSmemBytes = L::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 3;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TraceScope ts("tc_update_fused", st);
+  return cudaLaunchKernelEx(&cfg, fused_update_kernel<D>, mK, mV, mKg, mVg, W1, W2, W3, eta,
+                            p.n, p.H, p.hid, S, chunk, partials, err);
+}
+
+}  // namespace
+
+cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, const float* W3,
+                         const void* K, const void* V, const float* eta, int S, int64_t chunk,
+                         float* partials, int* err, cudaStream_t st) {
+  if (p.d == 256)
+    return fused_update_impl<256>(p, W1, W2, W3, K, V, eta, S, chunk, partials, err, st);
+  return fused_update_impl<64>(p, W1, W2, W3, K, V, eta, S, chunk, partials, err, st);
+}
+
+// 3-CTA clusters of this kernel's size that are resident at once on a B200
+// (148 SMs in clusters of GPCs): 45, measured with
+// cudaOccupancyMaxActiveClusters; more clusters would run in a second wave.
+int fused_clusters_per_wave() { return 45; }
+
+}  // namespace ttt

@@ -1,18 +1,12 @@
 // bf16 tensor-core path of the TTT update and apply on sm_100a: tcgen05 MMAs
 // with fp32 accumulators in tensor memory (TMEM), operands staged in shared
 // memory by TMA (cp.async.bulk.tensor, 128-byte swizzle, each CTA loads its own tiles), warp
-// specialised (one TMA producer thread, one MMA issuer thread, epilogue
-// warps), every wait bounded.
+// specialised (TMA producer, MMA issuer, epilogue warps), every wait bounded.
 //
-// Update of one head (kimjy99 ZipMap review, section 2, Eq. 1-3):
-//   fb kernel   h1 = W1 k, h3 = W3 k (one N=128 MMA over [W1s; W3s]),
-//               du = -W2^T v (N=64 MMA), then in the epilogue
-//               η·u, η·dh1, η·dh3 (u = SiLU(h1) ⊙ h3, dh3 = du ⊙ SiLU(h1),
-//               dh1 = du ⊙ h3 ⊙ SiLU'(h1)) stored as bf16 [H][n][hid].
-//   grad kernel split-K token reduction on MN-major operands:
-//               P1 = Σ η dh1 k^T, P3 = Σ η dh3 k^T, P2 = Σ η u v^T (= -G2^T,
-//               stored transposed as [d][hid]); fixed token ranges.
-//   then the shared fixed-order reduce + renorm kernel.
+// Update (kimjy99 ZipMap review, section 2, Eq. 1-3): the fused forward /
+// backward / token-reduction kernel (kernels_fused.cu, which rounds the fp32
+// weights to bf16 on chip) writing one fp32 partial per token split, then the
+// shared fixed-order reduce + renorm kernel.
 // Apply:        per 128-query tile, for each 64-wide hidden slice:
 //               F = Q [W1s; W3s]^T (TMEM), u = SiLU(h1) ⊙ h3 -> bf16 in shared
 //               memory, O += u W2s^T (TMEM); hidden activations never leave
@@ -32,8 +26,7 @@ size_t tc_main_bytes(const Problem& p);
 
 namespace {
 
-constexpr int HS = 64;           // hidden slice per fb CTA / apply step
-constexpr int TK = 64;           // tokens per grad stage
+constexpr int HS = 64;           // hidden slice per apply step
 
 // A-operand-in-TMEM forms used by the apply: a 128-row x 16-element bf16
 // slice of a K-major 128-byte-swizzled shared-memory tile copied into 8 TMEM
@@ -49,488 +42,6 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, u
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-// ----------------------------------------------------------------------------
-// Weight prologue: bf16 copies of W1, W3 ([H][hid][d]) and of W2^T ([H][hid][d])
-// ----------------------------------------------------------------------------
-__global__ void convert_weights_kernel(int H, int d, int hid, const float* __restrict__ W1,
-                                       const float* __restrict__ W2, const float* __restrict__ W3,
-                                       __nv_bfloat16* __restrict__ b1, __nv_bfloat16* __restrict__ b3,
-                                       __nv_bfloat16* __restrict__ b2t) {
-  // One block per 32 x 32 tile (hidden rows j0.., d columns c0..) of one head;
-  // the W2 tile is transposed through shared memory so that both its read and
-  // its write are coalesced.
-  __shared__ float tile[32][33];
-  const int tiles_c = d / 32, tiles_j = hid / 32;
-  const int h = blockIdx.x / (tiles_c * tiles_j);
-  const int t = blockIdx.x % (tiles_c * tiles_j);
-  const int j0 = (t / tiles_c) * 32, c0 = (t % tiles_c) * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const size_t mat = (size_t)h * hid * d;
-  for (int r = ty; r < 32; r += 8) {
-    const size_t i = mat + (size_t)(j0 + r) * d + c0 + tx;
-    b1[i] = __float2bfloat16_rn(W1[i]);
-    b3[i] = __float2bfloat16_rn(W3[i]);
-    tile[r][tx] = W2[mat + (size_t)(c0 + r) * hid + j0 + tx];
-  }
-  __syncthreads();
-  for (int r = ty; r < 32; r += 8)
-    b2t[mat + (size_t)(j0 + r) * d + c0 + tx] = __float2bfloat16_rn(tile[tx][r]);
-}
-
-// ----------------------------------------------------------------------------
-// fb kernel: forward dual GEMM + backward GEMM + gated epilogue
-// ----------------------------------------------------------------------------
-template <int D>
-struct FB {
-  static constexpr int NCH = D / CH;
-  static constexpr int CPS = NCH >= 2 ? 2 : 1;            // d-chunks per stage (one TMA box)
-  static constexpr int NSTAGE = 6 / CPS;
-  static constexpr int CHUNK = BM * CH * 2;               // 16 KB: 128 tokens x 64 d
-  static constexpr int STAGE = CPS * CHUNK;
-  static constexpr int W13_CH = 2 * HS * CH * 2;          // 16 KB: W1s rows then W3s rows
-  static constexpr int W2_CH = HS * CH * 2;               // 8 KB
-  static constexpr int OUT_TILE = BM * HS * 2;            // 16 KB: one output [128 x 64] bf16
-  static constexpr int OFF_W13 = 0;
-  static constexpr int OFF_W2 = OFF_W13 + NCH * W13_CH;
-  static constexpr int OFF_STAGE = OFF_W2 + NCH * W2_CH;
-  static constexpr int OFF_OUT = OFF_STAGE + NSTAGE * STAGE;  // 2 rotating output boxes
-  static constexpr int OFF_BAR = OFF_OUT + 2 * OUT_TILE;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;       // + alignment slack
-  static constexpr int EPI_WARPS = 8;                     // 2 per TMEM lane quadrant
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;     // producer, MMA, epilogue
-  static constexpr uint32_t TMEM_COLS = 512;              // 2 x (F13 128 + DU 64), at 0 / 256
-};
-
-// Work items are (head*nslices + slice, token tile) pairs.  With reps > 0 the
-// grid is groups*reps CTAs: CTA b owns group b / reps and the token tiles
-// [r*ntiles/reps, (r+1)*ntiles/reps), r = b % reps, so the hidden slices of one
-// head walk the same k/v tiles in lockstep and share them through L2.  With
-// reps == 0 (more groups than CTAs) each CTA takes a contiguous range of the
-// flattened item space.
-__device__ __forceinline__ void fb_item_range(int64_t ntiles, int groups, int reps,
-                                              int64_t& it0, int64_t& it1) {
-  if (reps > 0) {
-    const int64_t g = blockIdx.x / reps, r = blockIdx.x % reps;
-    it0 = g * ntiles + r * ntiles / reps;
-    it1 = g * ntiles + (r + 1) * ntiles / reps;
-  } else {
-    const int64_t total = (int64_t)groups * ntiles;
-    it0 = total * blockIdx.x / gridDim.x;
-    it1 = total * (blockIdx.x + 1) / gridDim.x;
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(FB<D>::THREADS, 1)
-    fb_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
-              const __grid_constant__ CUtensorMap mW1, const __grid_constant__ CUtensorMap mW3,
-              const __grid_constant__ CUtensorMap mW2t, const __grid_constant__ CUtensorMap mUs,
-              const __grid_constant__ CUtensorMap mD1s, const __grid_constant__ CUtensorMap mD3s,
-              const float* __restrict__ eta, int64_t n, int H, int hid, int reps, int* err) {
-  using L = FB<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* empty = full + L::NSTAGE;
-  uint64_t* wfull = empty + L::NSTAGE;
-  uint64_t* wempty = wfull + 1;
-  uint64_t* acc_full = wempty + 1;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* done = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int nslices = hid / HS;
-  const int64_t ntiles = (n + BM - 1) / BM;
-  int64_t it0, it1;
-  fb_item_range(ntiles, H * nslices, reps, it0, it1);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < L::NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(wfull, 1);
-    mbar_init(wempty, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], L::EPI_WARPS);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, L::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&mK);
-    tma_prefetch_desc(&mV);
-    int stage = 0;
-    uint32_t phase = 0, wphase = 0;
-    int cur_hs = -1;
-    int64_t issued = 0, wloads = 0;
-    bool ok = true;
-    for (int64_t it = it0; it < it1 && ok; ++it) {
-      const int hs = (int)(it / ntiles);
-      const int64_t tile = it % ntiles;
-      const int head = hs / nslices, slice = hs % nslices;
-      if (hs != cur_hs) {
-        if (cur_hs >= 0) {
-          if (!mbar_wait(wempty, wphase, abort_flag, err, kErrWaitEmpty)) { ok = false; break; }
-          wphase ^= 1;
-        }
-        mbar_arrive_expect_tx(wfull, L::NCH * (L::W13_CH + L::W2_CH));
-        const int row = head * hid + slice * HS;
-        TTT_DCHECK(row >= 0 && row + HS <= H * hid, err, kErrCheckTma);
-        for (int c = 0; c < L::NCH; ++c) {
-          uint8_t* w13 = smem + L::OFF_W13 + c * L::W13_CH;
-          tma_load_2d(w13, &mW1, wfull, c * CH, row);
-          tma_load_2d(w13 + HS * 128, &mW3, wfull, c * CH, row);
-          tma_load_2d(smem + L::OFF_W2 + c * L::W2_CH, &mW2t, wfull, c * CH, row);
-        }
-        ++wloads;
-        cur_hs = hs;
-      }
-      const int y = (int)(tile * BM);
-      for (int pass = 0; pass < 2 && ok; ++pass) {
-        const CUtensorMap* m = pass == 0 ? &mK : &mV;
-        for (int g = 0; g < L::NCH / L::CPS; ++g) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], L::STAGE);
-          TTT_DCHECK(y >= 0 && (int64_t)y < n && head * L::NCH + (g + 1) * L::CPS <= H * L::NCH,
-                     err, kErrCheckTma);
-          // one box = CPS chunks of [128 tokens x 64 d]
-          tma_load_3d(smem + L::OFF_STAGE + stage * L::STAGE, m, &full[stage], 0, y,
-                      head * L::NCH + g * L::CPS);
-          ++issued;
-          if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
-        }
-      }
-    }
-    drain_ring(full, L::NSTAGE, issued, err);
-    drain_ring(wfull, 1, wloads, err);
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idF = idesc_bf16_f32(BM, 2 * HS, false, false);
-    const uint32_t idU = idesc_bf16_f32(BM, HS, false, false);
-    int stage = 0;
-    uint32_t phase = 0, wphase = 0;
-    uint32_t abits = 0;  // bit b: phase parity of accumulator buffer b
-    int cur_hs = -1, buf = 0;
-    bool ok = true;
-    const uint32_t sbase = smem_u32(smem);
-    for (int64_t it = it0; it < it1 && ok; ++it) {
-      const int hs = (int)(it / ntiles);
-      if (hs != cur_hs) {
-        if (cur_hs >= 0) umma_commit(wempty);  // old weights free once prior MMAs finish
-        if (!mbar_wait(wfull, wphase, abort_flag, err, kErrWaitFull)) { ok = false; break; }
-        wphase ^= 1;
-        cur_hs = hs;
-      }
-      if (!mbar_wait(&acc_empty[buf], ((abits >> buf) & 1) ^ 1, abort_flag, err,
-                     kErrWaitAccFree)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t dF = tmem + buf * 256, dU = tmem + buf * 256 + 128;
-      for (int pass = 0; pass < 2 && ok; ++pass) {
-        for (int g = 0; g < L::NCH / L::CPS; ++g) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          for (int cc = 0; cc < L::CPS; ++cc) {
-            const int c = g * L::CPS + cc;
-            const uint32_t a = sbase + L::OFF_STAGE + stage * L::STAGE + cc * L::CHUNK;
-            const uint32_t b = pass == 0 ? sbase + L::OFF_W13 + c * L::W13_CH
-                                         : sbase + L::OFF_W2 + c * L::W2_CH;
-#pragma unroll
-            for (int kk = 0; kk < CH / 16; ++kk) {
-              const uint64_t da = sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024);
-              const uint64_t db = sdesc_sw128(b + kk * KSTEP_BYTES, 16, 1024);
-              umma_bf16(pass == 0 ? dF : dU, da, db, pass == 0 ? idF : idU, (c | kk) != 0);
-            }
-          }
-          umma_commit(&empty[stage]);
-          if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
-        }
-      }
-      umma_commit(&acc_full[buf]);
-      abits ^= 1u << buf;
-      buf ^= 1;
-    }
-    // Wait for every MMA issued by this thread before TMEM is released.
-    umma_commit(done);
-    volatile int never = 0;
-    mbar_wait(done, 0, &never, err, kErrWaitFinal);
-  } else if (warp >= 2) {
-    // ------------------------------------------------------------ epilogue
-    // Two warps per TMEM lane quadrant; warp half `ch` takes hidden columns
-    // [32*ch, 32*ch+32) of the slice.  Outputs are staged in shared memory in
-    // the 128-byte-swizzled box layout and written by TMA bulk stores.
-    const int q = warp & 3;
-    const int ch = (warp - 2) / 4;
-    const int row = q * 32 + lane;
-    const bool leader = warp == 2 && lane == 0;
-    uint8_t* stage_out = smem + L::OFF_OUT;
-    uint32_t out_k = 0;  // stores issued so far (selects the staging buffer)
-    uint32_t abits = 0;
-    int buf = 0;
-    for (int64_t it = it0; it < it1; ++it) {
-      const int hs = (int)(it / ntiles);
-      const int64_t tile = it % ntiles;
-      const int head = hs / nslices, slice = hs % nslices;
-      const int64_t tok = tile * BM + row;
-      const bool live = tok < n;
-      const float ne = live ? -__ldg(&eta[tok * H + head]) : 0.f;  // -η: du = -(W2^T v)
-      const bool got =
-          mbar_wait(&acc_full[buf], (abits >> buf) & 1, abort_flag, err, kErrWaitAcc);
-      __syncwarp();
-      if (named_bar_any(1, 32 * L::EPI_WARPS, !got)) break;
-      abits ^= 1u << buf;
-      tc_fence_after();
-      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + buf * 256 + ch * 32;
-      TTT_DCHECK(buf * 256 + ch * 32 + 128 + 32 <= (int)L::TMEM_COLS, err, kErrCheckTmem);
-      uint32_t r1[32], r3[32], rd[32];
-      tmem_ld_32x32(tl, r1);
-      tmem_ld_32x32(tl + HS, r3);
-      tmem_ld_32x32(tl + 128, rd);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      uint32_t pk[3][16];  // η·u, η·dh1, η·dh3 as packed bf16 pairs
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float o_u[2], o_1[2], o_3[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float h1 = __uint_as_float(r1[i + e]);
-          const float h3 = __uint_as_float(r3[i + e]);
-          const float edu = ne * __uint_as_float(rd[i + e]);  // η du
-          const float s = sigmoid_fast(h1);
-          const float a = h1 * s;                             // SiLU(h1)
-          const float dsl = fmaf(-a, s, a + s);               // SiLU'(h1) = s + a(1-s)
-          o_u[e] = -ne * (a * h3);
-          o_3[e] = edu * a;
-          o_1[e] = edu * h3 * dsl;
-        }
-        pk[0][i / 2] = pack_bf16x2(o_u[0], o_u[1]);
-        pk[1][i / 2] = pack_bf16x2(o_1[0], o_1[1]);
-        pk[2][i / 2] = pack_bf16x2(o_3[0], o_3[1]);
-      }
-      // Three [128 x 64] boxes go out through two rotating staging buffers;
-      // before refilling one, the store issued from it two stores ago must
-      // have finished reading it.
-      const int x = slice * HS, y = (int)(tile * BM);
-      TTT_DCHECK(x + HS <= hid && (int64_t)y < n, err, kErrCheckTma);
-#pragma unroll
-      for (int o = 0; o < 3; ++o) {
-        uint8_t* box = stage_out + (out_k & 1) * L::OUT_TILE;
-        if (leader) bulk_wait_group_read1();
-        named_bar_sync(1, 32 * L::EPI_WARPS);
-        uint8_t* r = box + (row / 8) * 1024 + (row % 8) * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(r + (((ch * 4 + c) ^ (row % 8)) * 16)) =
-              make_uint4(pk[o][4 * c], pk[o][4 * c + 1], pk[o][4 * c + 2], pk[o][4 * c + 3]);
-        fence_proxy_async_smem();
-        named_bar_sync(1, 32 * L::EPI_WARPS);
-        if (leader) {
-          tma_store_3d(o == 0 ? &mUs : o == 1 ? &mD1s : &mD3s, box, x, y, head);
-          bulk_commit_group();
-        }
-        ++out_k;
-      }
-      buf ^= 1;
-    }
-    if (leader) bulk_wait_group0();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc(tmem, L::TMEM_COLS);
-  }
-}
-
-// ----------------------------------------------------------------------------
-// grad kernel: split-K token reduction with MN-major operands
-//   kind 0: acc0 = Σ_t DH1[t, tile]^T K[t, :], acc1 = Σ_t DH3[t, tile]^T K[t, :]
-//   kind 1: acc_a = Σ_t U[t, tile_a]^T V[t, :] for two hidden tiles (one if
-//           hid = 128)
-// Each CTA = (kind, head, hidden tile group, split s); split s owns tokens
-// [s*chunk, min(n, (s+1)*chunk)), chunk a multiple of TK.
-// ----------------------------------------------------------------------------
-template <int D>
-struct GR {
-  static constexpr int NSTAGE = 3;
-  static constexpr int A_TILE = BM * TK * 2;              // 16 KB: 2 boxes [64 tok x 64 hid]
-  static constexpr int B_TILE = D * TK * 2;               // D/64 boxes [64 tok x 64 d]
-  static constexpr int STAGE = 2 * A_TILE + B_TILE;
-  static constexpr int OFF_BAR = NSTAGE * STAGE;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr int THREADS = 192;
-  static constexpr uint32_t TMEM_COLS = 512;              // acc a at column a*256
-};
-
-template <int D>
-__global__ void __launch_bounds__(GR<D>::THREADS, 1)
-    grad_kernel(const __grid_constant__ CUtensorMap mDH1, const __grid_constant__ CUtensorMap mDH3,
-                const __grid_constant__ CUtensorMap mU, const __grid_constant__ CUtensorMap mK,
-                const __grid_constant__ CUtensorMap mV, int64_t n, int H, int hid, int64_t chunk,
-                int ctas_kind0, int ctas_kind1, float* __restrict__ partials, int* err) {
-  using L = GR<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* empty = full + L::NSTAGE;
-  uint64_t* acc_full = empty + L::NSTAGE;
-  uint64_t* done = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // Decode (split, kind, head, tile group).
-  const int per_split = ctas_kind0 + ctas_kind1;
-  const int s = blockIdx.x / per_split;
-  int r = blockIdx.x % per_split;
-  const int kind = r < ctas_kind0 ? 0 : 1;
-  if (kind == 1) r -= ctas_kind0;
-  const int groups_per_head = kind == 0 ? hid / BM : (hid / BM + 1) / 2;
-  const int head = r / groups_per_head, grp = r % groups_per_head;
-  const int j_first = kind == 0 ? grp * BM : grp * 2 * BM;
-  const int nacc = kind == 0 ? 2 : (j_first + BM < hid ? 2 : 1);
-  const int64_t ts = (int64_t)s * chunk;
-  const int64_t te = ts + chunk < n ? ts + chunk : n;
-  const int nsteps = te > ts ? (int)((te - ts + TK - 1) / TK) : 0;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < L::NSTAGE; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    mbar_init(acc_full, 1);
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, L::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    int64_t issued = 0;
-    const uint32_t bytes = (uint32_t)(nacc * L::A_TILE + L::B_TILE);
-    for (int k = 0; k < nsteps; ++k) {
-      if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err, kErrWaitEmpty)) break;
-      uint8_t* st = smem + stage * L::STAGE;
-      mbar_arrive_expect_tx(&full[stage], bytes);
-      const int y = (int)(ts + (int64_t)k * TK);
-      for (int a = 0; a < nacc; ++a) {
-        const CUtensorMap* m = kind == 0 ? (a == 0 ? &mDH1 : &mDH3) : &mU;
-        const int j = kind == 0 ? j_first : j_first + a * BM;
-        // one box: 2 hidden chunks x [64 tokens x 64 hidden]
-        tma_load_4d(st + a * L::A_TILE, m, &full[stage], 0, y, j / CH, head);
-      }
-      // one box: D/64 d-chunks x [64 tokens x 64 d]
-      tma_load_3d(st + 2 * L::A_TILE, kind == 0 ? &mK : &mV, &full[stage], 0, y, head * (D / CH));
-      ++issued;
-      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
-    }
-    drain_ring(full, L::NSTAGE, issued, err);
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc = idesc_bf16_f32(BM, D, true, true);
-    const uint32_t sbase = smem_u32(smem);
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int k = 0; k < nsteps; ++k) {
-      if (!mbar_wait(&full[stage], phase, abort_flag, err, kErrWaitFull)) break;
-      tc_fence_after();
-      const uint32_t st = sbase + stage * L::STAGE;
-#pragma unroll
-      for (int kk = 0; kk < TK / 16; ++kk) {
-        // 16 tokens = two 8-row groups of 1024 bytes.
-        const uint64_t db = sdesc_sw128(st + 2 * L::A_TILE + kk * 2048, TK * 128, 1024);
-        for (int a = 0; a < nacc; ++a) {
-          const uint64_t da = sdesc_sw128(st + a * L::A_TILE + kk * 2048, TK * 128, 1024);
-          umma_bf16(tmem + a * 256, da, db, idesc, (k | kk) != 0);
-        }
-      }
-      umma_commit(&empty[stage]);
-      if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
-    }
-    umma_commit(acc_full);
-    umma_commit(done);
-    volatile int never = 0;
-    mbar_wait(done, 0, &never, err, kErrWaitFinal);
-  } else if (warp >= 2) {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const bool have = nsteps > 0 && mbar_wait(acc_full, 0, abort_flag, err, kErrWaitAcc);
-    __syncwarp();
-    tc_fence_after();
-    const size_t mat = (size_t)hid * D;
-    for (int a = 0; a < nacc; ++a) {
-      const int blk = kind == 0 ? a : 2;  // P1, P3, P2
-      float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat;
-      const int j = (kind == 0 ? j_first : j_first + a * BM) + q * 32 + lane;
-      TTT_DCHECK(j < hid && a * 256 + D <= (int)L::TMEM_COLS, err, kErrCheckIndex);
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t rr[32];
-        if (have) {
-          tmem_ld_32x32(tmem + ((uint32_t)(q * 32) << 16) + a * 256 + c0, rr);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) rr[i] = 0u;
-        }
-        if (kind == 0) {
-          float4* dst = reinterpret_cast<float4*>(P + (size_t)j * D + c0);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
-                                 __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) P[(size_t)(c0 + i) * hid + j] = __uint_as_float(rr[i]);
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc(tmem, L::TMEM_COLS);
-  }
 }
 
 // ----------------------------------------------------------------------------
@@ -860,36 +371,19 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
 // Host side
 // ----------------------------------------------------------------------------
 struct TcWs {
-  __nv_bfloat16 *b1, *b3, *b2t, *U, *DH1, *DH3;
   float *partials, *scratch;
 };
 
+// Workspace: the split partials [S][H][3][hid*d] fp32, then the renorm
+// scratch.
 TcWs carve(const Problem& p, void* ws, int S) {
   TcWs w;
   char* c = static_cast<char*>(ws);
-  const size_t wsz = (size_t)p.H * p.hid * p.d;
-  w.b1 = reinterpret_cast<__nv_bfloat16*>(c);
-  w.b3 = w.b1 + wsz;
-  w.b2t = w.b3 + wsz;
-  c += align_up(3 * wsz * 2, 1024);
-  const size_t inter = (size_t)p.H * p.n * p.hid;
-  w.U = reinterpret_cast<__nv_bfloat16*>(c);
-  c += align_up(inter * 2, 1024);
-  w.DH1 = reinterpret_cast<__nv_bfloat16*>(c);
-  c += align_up(inter * 2, 1024);
-  w.DH3 = reinterpret_cast<__nv_bfloat16*>(c);
-  c += align_up(inter * 2, 1024);
   w.partials = reinterpret_cast<float*>(c);
   c += align_up((size_t)S * p.H * 3 * p.hid * p.d * 4, 1024);
   w.scratch = reinterpret_cast<float*>(c);
   return w;
 }
-
-int grad_ctas_per_split(const Problem& p) {
-  const int tiles = p.hid / BM;
-  return p.H * tiles + p.H * ((tiles + 1) / 2);
-}
-
 
 template <int D>
 cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, const float* W3,
@@ -900,76 +394,14 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   TcWs w = carve(p, ws, sp.S);
   int* err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidDevice;
-  const size_t wsz = (size_t)p.H * p.hid * p.d;
   if (p.n > 0) {
-    {
-      TraceScope ts("tc_convert_weights", st);
-      const int cb = p.H * (p.hid / 32) * (p.d / 32);
-      convert_weights_kernel<<<cb, 256, 0, st>>>(p.H, p.d, p.hid, W1, W2, W3, w.b1, w.b3, w.b2t);
-    }
-    CUtensorMap mK, mV, mW1, mW3, mW2t, mDH1, mDH3, mU, mKg, mVg, mUs, mD1s, mD3s;
-    const uint64_t ld = (uint64_t)p.H * D;
-    {
-      // {64 d, tokens, d-chunks of all heads}: fb boxes are FB::CPS chunks of 128
-      // tokens, grad boxes all D/64 chunks of one head for 64 tokens.
-      const uint64_t dims3[3] = {(uint64_t)CH, (uint64_t)p.n, ld / CH};
-      const uint64_t str3[2] = {ld * 2, CH * 2};
-      const uint32_t box3[3] = {CH, BM, (uint32_t)FB<D>::CPS};
-      const uint32_t boxg[3] = {CH, TK, (uint32_t)(D / CH)};
-      if (!make_map(&mK, K, 3, dims3, str3, box3) || !make_map(&mV, V, 3, dims3, str3, box3) ||
-          !make_map(&mKg, K, 3, dims3, str3, boxg) || !make_map(&mVg, V, 3, dims3, str3, boxg))
-        return cudaErrorInvalidValue;
-    }
-    {
-      const uint64_t dims[2] = {(uint64_t)D, (uint64_t)p.H * p.hid}, str[1] = {(uint64_t)D * 2};
-      const uint32_t box[2] = {CH, HS};
-      if (!make_map(&mW1, w.b1, 2, dims, str, box) || !make_map(&mW3, w.b3, 2, dims, str, box) ||
-          !make_map(&mW2t, w.b2t, 2, dims, str, box))
-        return cudaErrorInvalidValue;
-    }
-    {
-      // stores (fb): {hidden, tokens, heads}, box [128 tokens x 64 hidden]
-      const uint64_t dims[3] = {(uint64_t)p.hid, (uint64_t)p.n, (uint64_t)p.H};
-      const uint64_t str[2] = {(uint64_t)p.hid * 2, (uint64_t)p.n * p.hid * 2};
-      const uint32_t boxs[3] = {CH, BM, 1};
-      // loads (grad): {64 hidden, tokens, hidden chunks, heads}, box = 2 chunks x 64 tokens
-      const uint64_t dims4[4] = {(uint64_t)CH, (uint64_t)p.n, (uint64_t)(p.hid / CH),
-                                 (uint64_t)p.H};
-      const uint64_t str4[3] = {(uint64_t)p.hid * 2, CH * 2, (uint64_t)p.n * p.hid * 2};
-      const uint32_t box4[4] = {CH, TK, 2, 1};
-      if (!make_map(&mDH1, w.DH1, 4, dims4, str4, box4) ||
-          !make_map(&mDH3, w.DH3, 4, dims4, str4, box4) ||
-          !make_map(&mU, w.U, 4, dims4, str4, box4) || !make_map(&mUs, w.U, 3, dims, str, boxs) ||
-          !make_map(&mD1s, w.DH1, 3, dims, str, boxs) || !make_map(&mD3s, w.DH3, 3, dims, str, boxs))
-        return cudaErrorInvalidValue;
-    }
-    // fb: (head, slice) groups x token-range replicas, see fb_item_range.
-    const int sms = num_sms();
-    const int groups = p.H * (p.hid / HS);
-    const int reps = groups <= sms ? sms / groups : 0;
-    const int grid_fb = reps > 0 ? groups * reps : sms;
-    cudaError_t e = ensure_smem_attr(fb_kernel<D>, FB<D>::SMEM);
-    if (e != cudaSuccess) return e;
-    {
-      TraceScope ts("tc_fwd_bwd", st);
-      fb_kernel<D><<<grid_fb, FB<D>::THREADS, FB<D>::SMEM, st>>>(
-          mK, mV, mW1, mW3, mW2t, mUs, mD1s, mD3s, eta, p.n, p.H, p.hid, reps, err);
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const int tiles = p.hid / BM;
-    const int k0 = p.H * tiles, k1 = p.H * ((tiles + 1) / 2);
-    e = ensure_smem_attr(grad_kernel<D>, GR<D>::SMEM);
-    if (e != cudaSuccess) return e;
-    {
-      TraceScope ts("tc_grad", st);
-      grad_kernel<D><<<sp.S * (k0 + k1), GR<D>::THREADS, GR<D>::SMEM, st>>>(
-          mDH1, mDH3, mU, mKg, mVg, p.n, p.H, p.hid, sp.chunk, k0, k1, w.partials, err);
-    }
-    e = cudaGetLastError();
+    const cudaError_t e =
+        fused_update(p, W1, W2, W3, K, V, eta, sp.S, sp.chunk, w.partials, err, st);
     if (e != cudaSuccess) return e;
   } else {
-    cudaMemsetAsync(w.partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * 4, st);
+    const cudaError_t e =
+        cudaMemsetAsync(w.partials, 0, (size_t)sp.S * p.H * 3 * p.hid * p.d * 4, st);
+    if (e != cudaSuccess) return e;
   }
   if (partial_out != nullptr)
     return sum_splits(sp.S, (size_t)p.H * 3 * p.hid * p.d, w.partials, partial_out, st);
@@ -1023,26 +455,26 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
 }  // namespace
 
 SplitPlan tc_split_plan(const Problem& p) {
-  const int per = grad_ctas_per_split(p);
-  int S = 148 / per;
+  // The fused update runs one 3-CTA cluster per (head, 128 hidden units,
+  // split); S splits of each group fill at most one wave of clusters,
+  // with at least 512 tokens per split (below that the fp32 partials, 6.3 MB
+  // per split for 4 heads of d 256, cost more than the parallelism gains).
+  // Every split is a whole number of 128-token tiles and none is empty.
+  const int groups = p.H * (p.hid / 128);
+  int S = fused_clusters_per_wave() / groups;
   if (S < 1) S = 1;
-  // at least 512 tokens per split: below that the fp32 partials (6.3 MB per
-  // split for 4 heads of d 256) cost more than the parallelism gains
   const int64_t max_s = (p.n + 511) / 512;
   if (S > max_s) S = (int)(max_s < 1 ? 1 : max_s);
   int64_t chunk = (p.n + S - 1) / S;
-  chunk = (chunk + TK - 1) / TK * TK;
-  if (chunk < TK) chunk = TK;
+  chunk = (chunk + BM - 1) / BM * BM;
+  if (chunk < BM) chunk = BM;
+  if (p.n > 0) S = (int)((p.n + chunk - 1) / chunk);
   return {S, chunk};
 }
 
 size_t tc_main_bytes(const Problem& p) {
   const SplitPlan sp = tc_split_plan(p);
-  const size_t wsz = (size_t)p.H * p.hid * p.d;
-  const size_t inter = (size_t)p.H * p.n * p.hid;
-  size_t b = align_up(3 * wsz * 2, 1024);
-  b += 3 * align_up(inter * 2, 1024);
-  b += align_up((size_t)sp.S * p.H * 3 * p.hid * p.d * 4, 1024);
+  size_t b = align_up((size_t)sp.S * p.H * 3 * p.hid * p.d * 4, 1024);
   b += align_up((size_t)p.H * (2 * p.hid + p.d) * 2 * 8, 1024);
   return b;
 }

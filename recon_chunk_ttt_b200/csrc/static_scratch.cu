@@ -17,10 +17,17 @@
 // ordering) race on it: serialise them.
 //
 // Host code cannot pass the array's name to a kernel (on the host it is only a
-// stand-in symbol), so the device address is looked up once per device with
-// cudaGetSymbolAddress() on the first call made while that device is current.
-// That first call should happen before any stream capture begins.
+// stand-in symbol), so the device address is looked up with
+// cudaGetSymbolAddress() on the first call made while a device is current, and
+// cached together with the unique id of that device's current CUDA context.
+// When the context changes (after cudaDeviceReset, or when the primary context
+// was released and created again, the module is loaded anew and the array may
+// move) the id no longer matches and the address is looked up again.  A call
+// that looks the address up should happen before any stream capture begins:
+// the first call on each device, and the first call after such a reset.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -33,21 +40,68 @@ constexpr size_t kScratchBytes = TTT_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_static_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
+struct CachedAddress {
+  void* addr;
+  unsigned long long ctx_id;
+};
+CachedAddress g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of g_static_scratch on the current device (looked up once).
+// The driver's cuCtxGetCurrent / cuCtxGetId, found through the runtime (no
+// link-time dependency on the driver library).
+PFN_cuCtxGetCurrent_v4000 ctx_get_current() {
+  static PFN_cuCtxGetCurrent_v4000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess
+               ? reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p)
+               : nullptr;
+  }();
+  return fn;
+}
+PFN_cuCtxGetId_v12000 ctx_get_id() {
+  static PFN_cuCtxGetId_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess
+               ? reinterpret_cast<PFN_cuCtxGetId_v12000>(p)
+               : nullptr;
+  }();
+  return fn;
+}
+
+// Unique id of the calling thread's current context (0 if there is none or
+// the driver cannot tell).
+unsigned long long current_context_id() {
+  auto get_current = ctx_get_current();
+  auto get_id = ctx_get_id();
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_static_scratch in the current device's context.
 ttt_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTT_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  CachedAddress& c = g_scratch[dev];
+  unsigned long long id = current_context_id();
+  if (c.addr == nullptr || id == 0 || id != c.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
       return TTT_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    // the lookup makes the device's primary context current if it was not
+    if (id == 0) id = current_context_id();
+    c.addr = p;
+    c.ctx_id = id;  // 0: unknown, looked up again on the next call
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return TTT_OK;
 }
 

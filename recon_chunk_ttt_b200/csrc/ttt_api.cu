@@ -173,6 +173,13 @@ ttt_status ttt_gate(const ttt_config* cfg, const void* Wg, const void* O_prime, 
   return cuda_status(ttt::tc_gate(p, Wg, O_prime, O, TTT_GATE_EPS, st));
 }
 
+int32_t ttt_update_splits(const ttt_config* cfg, int64_t n_tokens) {
+  if (check_cfg(cfg) != TTT_OK || n_tokens < 0 || n_tokens > kMaxTokens) return 0;
+  const Problem p = make_problem(cfg, n_tokens);
+  return cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_split_plan(p).S
+                                               : ttt::tc_split_plan(p).S;
+}
+
 size_t ttt_partial_floats(const ttt_config* cfg) {
   if (check_cfg(cfg) != TTT_OK) return 0;
   return (size_t)3 * cfg->heads * cfg->d * cfg->hidden;

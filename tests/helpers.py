@@ -76,9 +76,24 @@ def as_output_type(W_ref):
     return np.asarray(W_ref, dtype=np.float32).astype(np.float64)
 
 
+def rel_fro_heads(x, ref, heads, token_major=False):
+    """The relative Frobenius error over all heads and of every single head,
+    the largest of them: one wrong head cannot hide among correct ones.
+    Weights are [H, ...]; token-major outputs are [m, H*d]."""
+    x, ref = np.asarray(x, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+    if token_major:
+        per = [(x.reshape(x.shape[0], heads, -1)[:, h], ref.reshape(ref.shape[0], heads, -1)[:, h])
+               for h in range(heads)]
+    else:
+        per = [(x[h], ref[h]) for h in range(heads)]
+    return max([O.rel_fro(x, ref)] + [O.rel_fro(a, b) for a, b in per])
+
+
 def rel_errors(gpu, ref, x):
-    """Relative Frobenius errors on Ŵ - W (per matrix) and on O."""
+    """Relative Frobenius errors on Ŵ - W (per matrix) and on O, each the
+    maximum over the whole tensor and every head."""
     W = (x.W1, x.W2, x.W3)
-    errs = [O.rel_fro(g - w, as_output_type(r) - w) for g, r, w in zip(gpu[:3], ref[0], W)]
-    errs.append(O.rel_fro(gpu[3], ref[1]))
+    H = x.W1.shape[0]
+    errs = [rel_fro_heads(g - w, as_output_type(r) - w, H) for g, r, w in zip(gpu[:3], ref[0], W)]
+    errs.append(rel_fro_heads(gpu[3], ref[1], H, token_major=True))
     return errs

@@ -57,14 +57,37 @@ def test_workspace_sizes(B):
     cfg = _cfg(B)
     n = 961800
     ws = B.ttt_update_workspace_bytes(cfg, n)
-    inter = 3 * 4 * n * 512 * 2          # bf16 η·u, η·dh1, η·dh3
-    assert inter < ws < inter + 64 * 2**20
+    # the fused update keeps η·u, η·dh1, η·dh3 on chip: the workspace is the
+    # S fp32 gradient partials and the renorm scratch, independent of n once
+    # S stops growing
+    S = B.ttt_update_splits(cfg, n)
+    mat = 3 * 4 * 256 * 512
+    assert 1 <= S <= 16
+    assert S * mat * 4 <= ws < S * mat * 4 + 2**20
+    assert ws < 64 * 2**20
+    assert B.ttt_update_workspace_bytes(cfg, 10 * n) == ws
     assert B.ttt_update_workspace_bytes(cfg, 0) > 0
     f32 = B.ttt_update_workspace_bytes(_cfg(B, precision=B.PREC_FP32_CHECK), 1000)
     assert f32 >= 3 * 4 * 1000 * 512 * 4
     assert B.ttt_shadow_bytes(cfg) == 3 * 4 * 256 * 512 * 2
     assert B.ttt_update_workspace_bytes(_cfg(B, d=100), 10) == 0
     assert B.ttt_update_workspace_bytes(cfg, -1) == 0
+    assert B.ttt_update_splits(_cfg(B, d=100), 10) == 0
+
+
+def test_split_plan(B):
+    """The token splits of the update: whole 128-token tiles, at least 512
+    tokens each, none empty, at most one wave of 3-CTA clusters (45 resident
+    on a B200) over all (head, 128-hidden-unit) groups, one split for small n."""
+    cfg = _cfg(B)
+    assert B.ttt_update_splits(cfg, 0) == 1
+    assert B.ttt_update_splits(cfg, 1) == 1
+    assert B.ttt_update_splits(cfg, 512) == 1
+    assert B.ttt_update_splits(cfg, 1374) == 2       # one 518 x 518 frame
+    assert B.ttt_update_splits(cfg, 961800) == 2     # 16 groups x 2 splits = 32 clusters
+    assert B.ttt_update_splits(_cfg(B, heads=1), 961800) == 11
+    assert B.ttt_update_splits(_cfg(B, heads=1, d=64, hidden=128), 108) == 1
+    assert B.ttt_update_splits(_cfg(B, heads=64), 961800) == 1
     # Newton-Schulz: two d x hidden iterates, two d x d products and Delta per
     # matrix, on top of the update's own workspace (both precisions)
     for prec in (B.PREC_BF16_TC, B.PREC_FP32_CHECK):
@@ -207,18 +230,30 @@ def test_gate_partial_finish_reject_bad_arguments(B):
 
 
 def test_static_stream_step_limit_and_rejection(B):
-    """ttt_stream_step_static's fixed 64 MiB scratch holds one call of up to
-    2,560 tokens for 4 heads of d = 256 (the limit the header states); a larger
-    call is rejected with TTT_ERR_WORKSPACE before anything touches a device."""
-    cfg = _cfg(B)
+    """ttt_stream_step_static's fixed 64 MiB scratch, per configuration (the
+    limits the header states): BF16_TC keeps its intermediates on chip, so 4
+    heads of d = 256 fit for every n with and without Newton-Schulz, and for
+    every n up to 42 (ns_steps = 0) or 4 (ns_steps > 0) such heads fit; FP32_CHECK fits 2,471
+    tokens (678 with Newton-Schulz).  A call over the limit is rejected with
+    TTT_ERR_WORKSPACE before anything touches a device."""
     cap = 64 << 20
-    assert B.ttt_update_workspace_bytes(cfg, 2560) <= cap < B.ttt_update_workspace_bytes(cfg, 2561)
-    assert B.ttt_update_workspace_bytes(cfg, 1374) <= cap   # one 518 x 518 frame
+    ws = B.ttt_update_workspace_bytes
+    for ns in (0, 5):
+        cfg = _cfg(B, ns_steps=ns)
+        assert ws(cfg, 1374) <= cap and ws(cfg, 10**9) <= cap
+    assert ws(_cfg(B, heads=42), 10**9) <= cap < ws(_cfg(B, heads=43), 1)
+    assert ws(_cfg(B, heads=4, ns_steps=5), 10**9) <= cap < ws(_cfg(B, heads=5, ns_steps=5), 10**9)
+    f32 = _cfg(B, precision=B.PREC_FP32_CHECK)
+    f32ns = _cfg(B, precision=B.PREC_FP32_CHECK, ns_steps=5)
+    assert ws(f32, 2471) <= cap < ws(f32, 2472)
+    assert ws(f32ns, 678) <= cap < ws(f32ns, 679)
+    assert ws(f32, 1374) <= cap < ws(f32ns, 1374)   # one frame: fits without Newton-Schulz
     L = B.lib()
     f = L.ttt_stream_step_static
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f.argtypes = [ctypes.POINTER(B.ttt_config), P, P, P, P, P, P, P, I64, P, I64, P, P]
     f.restype = ctypes.c_int
-    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2561, FAKE, 5, FAKE, None]
-    assert f(ctypes.byref(cfg), *args) == B.TTT_ERR_WORKSPACE
-    assert f(None, *args) == B.TTT_ERR_INVALID_ARG
+    for cfg, n in ((f32, 2472), (f32ns, 1374), (_cfg(B, heads=43), 10)):
+        args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n, FAKE, 5, FAKE, None]
+        assert f(ctypes.byref(cfg), *args) == B.TTT_ERR_WORKSPACE
+    assert f(None, *[FAKE] * 7, 5, FAKE, 5, FAKE, None) == B.TTT_ERR_INVALID_ARG

@@ -47,8 +47,9 @@ def test_layer8(precision, tol):
 
 
 @pytest.mark.slow
-def test_scale100_bf16():
-    _check(wl.make_inputs("scale100"), R.PREC_BF16_TC, TOL_TC)
+@pytest.mark.parametrize("precision,tol", PRECS)
+def test_scale100(precision, tol):
+    _check(wl.make_inputs("scale100"), precision, tol)
 
 
 # ------------------------------------------------------- ragged / edge sizes
@@ -212,53 +213,76 @@ def test_stream_renorm_off_equals_sum_of_frame_updates():
 
 
 # --------------------------------------------- full-size headline (scene700)
+def _w2_rows(W1, W2, W3, Kh, Vh, eta, rows, chunk=131072):
+    """Rows of G2 over all tokens, summed over token chunks (bounded memory)."""
+    g = 0.0
+    for s in range(0, Kh.shape[0], chunk):
+        g = g + O.gradient_rows_w2(W1, W2, W3, Kh[s:s + chunk], Vh[s:s + chunk],
+                                   eta[s:s + chunk], rows)
+    return g
+
+
 @pytest.mark.slow
 def test_scene700_full_size_sampled():
-    """T = 961,800 tokens, 4 heads: the update in the launch configuration of
-    the benchmark, checked on sampled rows of Ŵ1, Ŵ3 (renorm row), the row
-    norms of Ŵ2, and sampled columns of G2 (renorm off); the apply on all
-    961,800 image queries + 21,984 ray queries checked on sampled rows."""
+    """T = 961,800 tokens, 4 heads, in the launch configuration of the
+    benchmark, for the first and the last (24th) layer's seeded weights:
+    sampled rows of all three updated matrices under the row renorm (Ŵ1, Ŵ3
+    rows need only their hidden units; Ŵ2 rows need u of every hidden unit),
+    sampled columns of G2 with the renorm off (first layer), and the apply of
+    the updated weights to all 961,800 image and 21,984 ray queries, checked
+    on sampled rows against the oracle's apply of the same bf16 weights."""
     w = wl.WORKLOADS["scene700"]
     x = wl.make_inputs(w, bits=True)
     H, hid, d = x.W1.shape
     dev = lambda b: torch.from_numpy(b.view(np.int16)).to("cuda").view(torch.bfloat16)  # noqa
     K, V, Q, Qr = dev(x.K), dev(x.V), dev(x.Q), dev(x.Qray)
-    W1, W2, W3 = (to_dev(a, torch.float32) for a in (x.W1, x.W2, x.W3))
     eta = to_dev(x.eta, torch.float32)
-    res = {}
-    for renorm in (R.RENORM_ROW, R.RENORM_OFF):
-        cfg = R.make_config(H, d, hid, renorm=renorm)
-        res[renorm] = [t.cpu().double().numpy()
-                       for t in R.ttt_update(cfg, W1, W2, W3, K, V, eta)]
-    R.ttt_check_device_error()
-    rows, cols = [0, 137, 300, 511], [5, 256, 509]
-    errs = []
-    for h in range(H):
-        sl = slice(h * d, (h + 1) * d)
-        Kh = wl.bits_to_f32(x.K[:, sl])
-        Vh = wl.bits_to_f32(x.V[:, sl])
-        g1, g3 = O.gradient_rows_w13(x.W1[h], x.W2[h], x.W3[h], Kh, Vh, x.eta[:, h], rows)
-        for Wm, g, gi in ((x.W1[h], g1, 0), (x.W3[h], g3, 2)):
-            ref = O.renorm(Wm[rows], Wm[rows].astype(np.float64) - g, O.RENORM_ROW)
-            errs.append(O.rel_fro(res[R.RENORM_ROW][gi][h][rows] - Wm[rows], ref - Wm[rows]))
-        g2 = O.gradient_cols_w2(x.W1[h], x.W2[h], x.W3[h], Kh, Vh, x.eta[:, h], cols)
-        errs.append(O.rel_fro(res[R.RENORM_OFF][1][h][:, cols] - x.W2[h][:, cols], -g2))
-        np.testing.assert_allclose(np.linalg.norm(res[R.RENORM_ROW][1][h], axis=1),
-                                   np.linalg.norm(x.W2[h].astype(np.float64), axis=1), rtol=1e-5)
-    assert max(errs) <= TOL_TC, errs
-    # Apply at full size on the pre-update weights (an oracle-known state).
-    cfg = R.make_config(H, d, hid)
-    shadow = R.ttt_pack_shadow(cfg, W1, W2, W3)
-    Oi = R.ttt_apply(cfg, Q, shadow=shadow)
-    Orr = R.ttt_apply(cfg, Qr, shadow=shadow)
-    R.ttt_check_device_error()
+    rows, rows2, cols = [0, 137, 300, 511], [0, 101, 255], [5, 256, 509]
     rng = np.random.default_rng(0)
-    for Qbits, Og in ((x.Q, Oi), (x.Qray, Orr)):
-        m = Qbits.shape[0]
-        idx = np.unique(np.concatenate([rng.integers(0, m, 96), [0, m - 1, m - 2]]))
-        ref = O.ttt_apply(x.W1, x.W2, x.W3, wl.bits_to_f32(Qbits[idx]))
-        got = Og[torch.from_numpy(idx).cuda()].float().cpu().double().numpy()
-        assert O.rel_fro(got, ref) <= TOL_TC
+    errs = {}
+    for layer, heads in ((0, range(H)), (w.layers - 1, (0, H - 1))):
+        if layer == 0:
+            Wh = (x.W1, x.W2, x.W3)
+        else:
+            W1_, W2_, W3_ = wl.draw_weights(np.random.default_rng([w.seed, layer]), H, d, hid,
+                                            1.0 / d, 1.0 / hid)
+            Wh = (W1_, W2_, W3_)
+        W1, W2, W3 = (to_dev(a, torch.float32) for a in Wh)
+        res = {}
+        for renorm in ((R.RENORM_ROW, R.RENORM_OFF) if layer == 0 else (R.RENORM_ROW,)):
+            cfg = R.make_config(H, d, hid, renorm=renorm)
+            shadow = R.alloc_shadow(cfg)
+            res[renorm] = [t_.cpu().double().numpy()
+                           for t_ in R.ttt_update(cfg, W1, W2, W3, K, V, eta, shadow=shadow)]
+            if renorm == R.RENORM_ROW:
+                Oi = R.ttt_apply(cfg, Q, shadow=shadow)
+                Orr = R.ttt_apply(cfg, Qr, shadow=shadow)
+        R.ttt_check_device_error()
+        got_row = res[R.RENORM_ROW]
+        for h in heads:
+            sl = slice(h * d, (h + 1) * d)
+            Kh = wl.bits_to_f32(x.K[:, sl])
+            Vh = wl.bits_to_f32(x.V[:, sl])
+            W1h, W2h, W3h = Wh[0][h], Wh[1][h], Wh[2][h]
+            g1, g3 = O.gradient_rows_w13(W1h, W2h, W3h, Kh, Vh, x.eta[:, h], rows)
+            g2 = _w2_rows(W1h, W2h, W3h, Kh, Vh, x.eta[:, h], rows2)
+            for Wm, g, gi, rr in ((W1h, g1, 0, rows), (W3h, g3, 2, rows), (W2h, g2, 1, rows2)):
+                ref = O.renorm(Wm[rr], Wm[rr].astype(np.float64) - g, O.RENORM_ROW)
+                errs[(layer, h, gi)] = O.rel_fro(got_row[gi][h][rr] - Wm[rr], ref - Wm[rr])
+            if layer == 0:
+                gc = O.gradient_cols_w2(W1h, W2h, W3h, Kh, Vh, x.eta[:, h], cols)
+                errs[(layer, h, "g2cols")] = O.rel_fro(
+                    res[R.RENORM_OFF][1][h][:, cols] - W2h[:, cols], -gc)
+        # the apply reads the bf16 shadow of the updated weights
+        Wb = [wl.bf16_round(a.astype(np.float32)) for a in got_row]
+        for name, Qbits, Og in (("image", x.Q, Oi), ("ray", x.Qray, Orr)):
+            m = Qbits.shape[0]
+            idx = np.unique(np.concatenate([rng.integers(0, m, 96), [0, m - 1, m - 2]]))
+            ref = O.ttt_apply(*Wb, wl.bits_to_f32(Qbits[idx]))
+            got = Og[torch.from_numpy(idx).cuda()].float().cpu().double().numpy()
+            errs[(layer, name)] = O.rel_fro(got, ref)
+    bad = {k: v for k, v in errs.items() if not v <= TOL_TC}
+    assert not bad, (bad, max(errs.values()))
 
 
 def test_bounded_wait_runs_out_and_reports():
