@@ -267,11 +267,11 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
  *    ttt_update_workspace_bytes(cfg, n) exceeds TTT_STATIC_SCRATCH_BYTES.
  *    The limit depends on the configuration.  BF16_TC keeps the update's
  *    intermediates on chip, so its workspace stops growing with n: with 4
- *    heads of d = 256, hidden 512 every n fits (19.0 MB with ns_steps = 0,
- *    63.0 MB with ns_steps > 0); for every n, up to 42 such heads fit with
- *    ns_steps = 0 and 4 with ns_steps > 0.  FP32_CHECK keeps per-token
- *    intermediates: 4 heads of d = 256 fit up to 2,471 tokens per call with
- *    ns_steps = 0 and 678 with ns_steps > 0 (one 518 x 518 frame is 1,374
+ *    heads of d = 256, hidden 512 every n fits (25.2 MB with ns_steps = 0,
+ *    69.3 MB with ns_steps > 0); for every n, up to 31 such heads fit with
+ *    ns_steps = 0 and 6 with ns_steps > 0.  FP32_CHECK keeps per-token
+ *    intermediates: 4 heads of d = 256 fit up to 3,836 tokens per call with
+ *    ns_steps = 0 and 2,044 with ns_steps > 0 (one 518 x 518 frame is 1,374
  *    tokens).
  *  - Every GPU that loads the library may hold the array until exit.
  *  - All calls on a device share the array and it keeps the last call's
@@ -284,7 +284,7 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
  *    such a call (the first on each device, and the first after a reset)
  *    before any stream capture.
  */
-#define TTT_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+#define TTT_STATIC_SCRATCH_BYTES ((size_t)96 << 20)
 ttt_status ttt_stream_step_static(const ttt_config* cfg,
                                   float* W1, float* W2, float* W3, void* shadow,
                                   const void* K, const void* V, const float* eta, int64_t n,

@@ -74,10 +74,17 @@ cudaError_t tc_update(const Problem& p, const float* W1, const float* W2, const 
 cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q, void* O,
                      cudaStream_t st);
 // Fused update kernel (kernels_fused.cu): fp32 weights W1, W3 [H][hid][d],
-// W2 [H][d][hid] in (rounded to bf16 inside); the S split partials of the
-// plan out.
+// W2 [H][d][hid] in (rounded to bf16 inside); the S partial slots of the
+// plan out ([S][H][3][hid*d]).  The head-major tile space is split evenly
+// over `sets` sets of hid/128 3-CTA clusters (one per group of 128 hidden
+// units); a head's gradient arrives in at most `splits` pieces (slots),
+// unused slots are zero.
+struct FusedPlan {
+  int sets, splits;
+};
+FusedPlan fused_plan(const Problem& p);
 cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, const float* W3,
-                         const void* K, const void* V, const float* eta, int S, int64_t chunk,
+                         const void* K, const void* V, const float* eta, int NS, int S,
                          float* partials, int* err, cudaStream_t st);
 // Clusters of the fused update that fill one wave of the GPU.
 int fused_clusters_per_wave();

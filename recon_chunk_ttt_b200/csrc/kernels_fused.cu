@@ -47,10 +47,18 @@ struct FU {
   static constexpr int NCH = D / CH;            // 64-wide d chunks
   static constexpr int GH = 128;                // hidden units per cluster
   static constexpr int FH = 64;                 // hidden units per F CTA
+  // Ring shapes (measured at scene700 size): the forward ring holds one whole
+  // k (or v) tile in one 64 KB TMA box, the gradient ring two 16 KB stages.
+  // A thread's TMA boxes complete one after another, so fewer, larger boxes
+  // deliver more bytes per unit of time.
   static constexpr int TKG = 32;                // tokens per gradient stage
-  static constexpr int NKF = 3;                 // forward ring: [128 tokens x 64 d] stages
-  static constexpr int NKG = 3;                 // gradient ring: [32 tokens x d] stages
-  static constexpr int CHUNK = BM * 128;        // 16 KB
+  static constexpr int NKF = 1;                 // forward ring stages
+  static constexpr int NKG = 2;                 // gradient ring: [TKG tokens x d] stages
+  static constexpr int CPS_ = 4;                // d-chunks per forward stage (one TMA box)
+  static constexpr int CPS = CPS_ < NCH ? CPS_ : NCH;
+  static_assert(NCH % CPS == 0, "chunks per stage");
+  static constexpr int CHUNK = BM * 128;        // 16 KB: 128 rows x 64 bf16
+  static constexpr int KF_STAGE = CPS * CHUNK;
   static constexpr int KG_STAGE = TKG * D * 2;
   static constexpr int XB = BM * 128;           // exchange block: 128 tokens x 64 bf16 (16 KB)
   static constexpr int W2BLK = D * 128;         // D: one block of 64 hidden units x d rows
@@ -58,7 +66,7 @@ struct FU {
   // D: 2 MN-major blocks of [d rows x 64 hidden units] of W2 (same bytes)
   static constexpr int OFF_W = 0;
   static constexpr int OFF_KF = OFF_W + NCH * CHUNK;
-  static constexpr int OFF_KG = OFF_KF + NKF * CHUNK;
+  static constexpr int OFF_KG = OFF_KF + NKF * KF_STAGE;
   static constexpr int OFF_GA = OFF_KG + NKG * KG_STAGE;  // A of the gradient MMA: 2 blocks
   static constexpr int OFF_EX = OFF_GA + 2 * XB;          // F: du in | η·u out; D: du out x 2
   static constexpr int OFF_BAR = OFF_EX + 2 * XB;
@@ -95,6 +103,7 @@ struct Bars {
   __device__ uint64_t* du_full() { return x(10); }    // F: du of the tile arrived
   __device__ uint64_t* du_empty(int f) { return x(11 + f); }  // D: rank f read its du
   __device__ uint64_t* du_read() { return x(13); }    // F: every epilogue warp read du
+  __device__ uint64_t* g_empty() { return x(14); }    // gradient accumulator drained
 };
 
 // Give up: device error word, and the abort flag of every CTA of the cluster.
@@ -133,6 +142,51 @@ __device__ __forceinline__ void final_wait(uint64_t* bar, uint32_t parity, int* 
   cwait<true>(bar, parity, &never, err, kErrWaitFinal);
 }
 
+// Work split.  Clusters come in sets of `groups` (the hidden units of a head
+// in groups of 128), cluster `grp` of a set taking hidden group grp.  The
+// head-major tile space (H heads x ntg tiles of 128 tokens) is cut into NS
+// equal contiguous ranges, one per set, so the clusters of a set walk the
+// same k/v tiles at the same pace (one read from HBM, the rest from L2).  The
+// part of a range inside one head is a segment; a range holds one segment, or
+// the end of one head and the start of the next.  Piece p of a (head, group)
+// is the segment of the p-th set whose range meets the head, and its gradient
+// goes to partial slot p; slots a head has no piece for are written as zeros
+// by the set holding its last piece.  All of it is a function of (n, shape,
+// NS), so the split sums are fixed.
+struct Seg {
+  int head, grp;     // group of the segment
+  int64_t ta;        // first tile of the segment within its group
+  int nts;           // tiles in the segment
+  int base;          // index of its first tile among the cluster's tiles
+  int p;             // piece (partial slot) of the group
+  bool last;         // the group's last piece
+};
+__host__ __device__ __forceinline__ int64_t range_lo(int c, int NC, int64_t T) {
+  return (int64_t)c * T / NC;
+}
+// The set whose range holds tile index x of the head-major space.
+__host__ __device__ __forceinline__ int cluster_of(int64_t x, int NC, int64_t T) {
+  int c = (int)(x * NC / T);
+  while (c > 0 && range_lo(c, NC, T) > x) --c;
+  while (c + 1 < NC && range_lo(c + 1, NC, T) <= x) ++c;
+  return c;
+}
+__device__ __forceinline__ Seg make_seg(int c, int NC, int64_t T, int64_t ntg, int grp, int sg) {
+  const int64_t lo = range_lo(c, NC, T), hi = range_lo(c + 1, NC, T);
+  const int64_t g = lo / ntg + sg;  // head
+  const int64_t a = g * ntg > lo ? g * ntg : lo;
+  const int64_t b = (g + 1) * ntg < hi ? (g + 1) * ntg : hi;
+  Seg s;
+  s.head = (int)g;
+  s.grp = grp;
+  s.ta = a - g * ntg;
+  s.nts = (int)(b - a);
+  s.base = (int)(a - lo);
+  s.p = c - cluster_of(g * ntg, NC, T);
+  s.last = c == cluster_of((g + 1) * ntg - 1, NC, T);
+  return s;
+}
+
 template <int D>
 __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     fused_update_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
@@ -140,7 +194,7 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
                         const __grid_constant__ CUtensorMap mVg,
                         const float* __restrict__ W1, const float* __restrict__ W2,
                         const float* __restrict__ W3, const float* __restrict__ eta,
-                        int64_t n, int H, int hid, int S, int64_t chunk,
+                        int64_t n, int H, int hid, int NS, int S,
                         float* __restrict__ partials, int* err) {
   using L = FU<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -152,16 +206,14 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int rank = (int)cluster_ctarank();
   const bool isF = rank < 2;
-  // Work item: (head, hidden group, split)
   const int groups = hid / L::GH;
-  const int item = blockIdx.x / 3;
-  const int g = item / S, s = item % S;
-  const int head = g / groups, grp = g % groups;
-  const int64_t ntiles_all = (n + BM - 1) / BM;
-  const int64_t t0 = (int64_t)s * chunk / BM;
-  int64_t t1 = ((int64_t)s + 1) * chunk / BM;
-  if (t1 > ntiles_all) t1 = ntiles_all;
-  const int nt = t1 > t0 ? (int)(t1 - t0) : 0;
+  const int set = blockIdx.x / 3 / groups, grp = blockIdx.x / 3 % groups;
+  const int64_t ntg = (n + BM - 1) / BM;
+  const int64_t T = (int64_t)H * ntg;
+  const int64_t lo = range_lo(set, NS, T), hi = range_lo(set + 1, NS, T);
+  const int NT = (int)(hi - lo);                        // tiles of this cluster
+  const int nseg = NT > 0 ? (int)((hi - 1) / ntg - lo / ntg + 1) : 0;
+  auto seg = [&](int sg) { return make_seg(set, NS, T, ntg, grp, sg); };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NKF; ++i) {
@@ -180,6 +232,7 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     mbar_init(bar.ga_full(), 1);
     mbar_init(bar.ga_empty(), 1);
     mbar_init(bar.g_full(), 1);
+    mbar_init(bar.g_empty(), 1);
     mbar_init(bar.done(), 1);
     mbar_init(bar.au_empty(), 1);
     mbar_init(bar.du_full(), 1);
@@ -190,7 +243,7 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     fence_mbar_init();
     // Receivers arm their own exchange barriers (the senders' bulk copies
     // only complete bytes): F expects its du block, D both η·u blocks.
-    if (nt > 0) {
+    if (NT > 0) {
       if (isF)
         mbar_arrive_expect_tx(bar.du_full(), L::XB);
       else
@@ -209,26 +262,31 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------ weights + forward ring
+    // ------------------------------------------------ forward ring
     const CUtensorMap* m = isF ? &mK : &mV;
     tma_prefetch_desc(m);
     int stage = 0;
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
-    for (int i = 0; i < nt && ok; ++i) {
-      const int y = (int)((t0 + i) * BM);
-      for (int c = 0; c < L::NCH; ++c) {
-        if (!cwait<false>(bar.kf_empty(stage), phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
-          ok = false;
-          break;
+    for (int sg = 0; sg < nseg && ok; ++sg) {
+      const Seg S_ = seg(sg);
+      for (int i = 0; i < S_.nts && ok; ++i) {
+        const int y = (int)((S_.ta + i) * BM);
+        for (int c = 0; c < L::NCH; c += L::CPS) {
+          if (!cwait<false>(bar.kf_empty(stage), phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar.kf_full(stage), L::KF_STAGE);
+          TTT_DCHECK((int64_t)y < n && S_.head * L::NCH + c + L::CPS <= H * L::NCH, err,
+                     kErrCheckTma);
+          // one box: CPS chunks of [128 tokens x 64 d]
+          tma_load_3d(smem + L::OFF_KF + stage * L::KF_STAGE, m, bar.kf_full(stage), 0, y,
+                      S_.head * L::NCH + c);
+          ++issued;
+          if (++stage == L::NKF) { stage = 0; phase ^= 1; }
         }
-        mbar_arrive_expect_tx(bar.kf_full(stage), L::CHUNK);
-        TTT_DCHECK((int64_t)y < n && head * L::NCH + c < H * L::NCH, err, kErrCheckTma);
-        tma_load_3d(smem + L::OFF_KF + stage * L::CHUNK, m, bar.kf_full(stage), 0, y,
-                    head * L::NCH + c);
-        ++issued;
-        if (++stage == L::NKF) { stage = 0; phase ^= 1; }
       }
     }
     drain_ring(bar.kf_full(0), L::NKF, issued, err);
@@ -240,20 +298,23 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
-    for (int i = 0; i < nt && ok; ++i) {
-      const int y = (int)((t0 + i) * BM);
-      for (int st = 0; st < BM / L::TKG; ++st) {
-        if (!cwait<false>(bar.kg_empty(stage), phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
-          ok = false;
-          break;
+    for (int sg = 0; sg < nseg && ok; ++sg) {
+      const Seg S_ = seg(sg);
+      for (int i = 0; i < S_.nts && ok; ++i) {
+        const int y = (int)((S_.ta + i) * BM);
+        for (int st = 0; st < BM / L::TKG; ++st) {
+          if (!cwait<false>(bar.kg_empty(stage), phase ^ 1, abort_flag, err, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar.kg_full(stage), L::KG_STAGE);
+          TTT_DCHECK((int64_t)(y + st * L::TKG) < n + BM && S_.head < H, err, kErrCheckTma);
+          // one box: NCH d-chunks x [TKG tokens x 64 d]
+          tma_load_3d(smem + L::OFF_KG + stage * L::KG_STAGE, m, bar.kg_full(stage), 0,
+                      y + st * L::TKG, S_.head * L::NCH);
+          ++issued;
+          if (++stage == L::NKG) { stage = 0; phase ^= 1; }
         }
-        mbar_arrive_expect_tx(bar.kg_full(stage), L::KG_STAGE);
-        TTT_DCHECK((int64_t)(y + st * L::TKG) < n + BM && head < H, err, kErrCheckTma);
-        // one box: NCH d-chunks x [TKG tokens x 64 d]
-        tma_load_3d(smem + L::OFF_KG + stage * L::KG_STAGE, m, bar.kg_full(stage), 0,
-                    y + st * L::TKG, head * L::NCH);
-        ++issued;
-        if (++stage == L::NKG) { stage = 0; phase ^= 1; }
       }
     }
     drain_ring(bar.kg_full(0), L::NKG, issued, err);
@@ -264,96 +325,91 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     const uint32_t idF = idesc_bf16_f32(BM, 128, false, !isF);
     const uint32_t idG = idesc_bf16_f32(BM, D, true, true);
     const uint32_t sbase = smem_u32(smem);
-    bool ok = nt == 0 || cwait<false>(bar.w_full(), 0, abort_flag, err, kErrWaitFull);
-    // Forward MMAs of tile fi (one 64-d chunk per issue) and gradient MMAs of
-    // tile gj (one TKG-token stage per issue) are interleaved as their operands
-    // arrive, alternating when both are ready, so both operand rings drain at
-    // an even rate.  Each accumulator still receives its MMAs in one fixed
-    // order (chunks, stages and tiles ascending): the result does not depend
-    // on the interleaving.  Barriers are polled without blocking; the whole
-    // loop gives up after kWaitLimitCycles without progress.
-    int fi = 0, fc = 0, gj = 0, gst = 0;
-    bool f_open = false, g_open = false, prefer_g = true;
+    const uint32_t ga = sbase + L::OFF_GA;
     int fs = 0, gs = 0;
     uint32_t fph = 0, gph = 0;
-    long long last = clock64();
-    const uint32_t ga = sbase + L::OFF_GA;
-    while (ok && gj < nt) {
-      bool issued = false;
-      for (int pass = 0; pass < 2 && !issued; ++pass) {
-        const bool try_g = (pass == 0) == prefer_g;
-        if (try_g) {
-          if (gj >= fi) continue;  // tile gj's forward MMAs are not all issued yet
-          if (!g_open) {
-            const bool r = isF ? mbar_test_wait(bar.ga_full(), (uint32_t)(gj & 1))
-                               : mbar_test_wait_cluster(bar.ga_full(), (uint32_t)(gj & 1));
-            if (!r) continue;
-            g_open = true;
-            if (!isF && gj + 1 < nt) mbar_arrive_expect_tx(bar.ga_full(), 2 * L::XB);
+    bool ok = true;
+    for (int sg = 0; sg < nseg && ok; ++sg) {
+      const Seg S_ = seg(sg);
+      // this segment's weights are staged; the previous gradient is drained
+      if (!cwait<false>(bar.w_full(), (uint32_t)(sg & 1), abort_flag, err, kErrWaitFull) ||
+          (sg >= 1 && !cwait<false>(bar.g_empty(), (uint32_t)((sg - 1) & 1), abort_flag, err,
+                                    kErrWaitAccFree))) {
+        ok = false;
+        break;
+      }
+      // Per tile i: the forward MMAs of tile i, then the gradient MMAs of
+      // tile i - 1 (whose operand the epilogue has been forming meanwhile).
+      for (int i = 0; i <= S_.nts && ok; ++i) {
+        if (i < S_.nts) {
+          const int gi = S_.base + i;
+          const int b = gi & 1;
+          if (!cwait<false>(bar.acc_empty(b), ((gi >> 1) & 1) ^ 1, abort_flag, err,
+                            kErrWaitAccFree)) {
+            ok = false;
+            break;
           }
-          if (!mbar_test_wait(bar.kg_full(gs), gph)) continue;
           tc_fence_after();
-          const uint32_t kg = sbase + L::OFF_KG + gs * L::KG_STAGE;
+          const uint32_t dF = tmem + b * 128;
+          for (int c0 = 0; c0 < L::NCH && ok; c0 += L::CPS) {
+            if (!cwait<false>(bar.kf_full(fs), fph, abort_flag, err, kErrWaitFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int cc = 0; cc < L::CPS; ++cc) {
+              const int c = c0 + cc;
+              const uint32_t a = sbase + L::OFF_KF + fs * L::KF_STAGE + cc * L::CHUNK;
 #pragma unroll
-          for (int kk = 0; kk < L::TKG / 16; ++kk) {
-            // A: MN-major, 2 blocks of 64 rows (LBO), 16 tokens per K step;
-            // B: MN-major, NCH blocks of 64 d (LBO = TKG rows x 128 B)
-            const uint64_t da = sdesc_sw128(ga + (gst * L::TKG + kk * 16) * 128, L::XB, 1024);
-            const uint64_t db = sdesc_sw128(kg + kk * 16 * 128, L::TKG * 128, 1024);
-            umma_bf16(tmem + L::TM_G, da, db, idG, (gj | gst | kk) != 0);
+              for (int kk = 0; kk < CH / 16; ++kk) {
+                const uint64_t db =
+                    isF ? sdesc_sw128(sbase + L::OFF_W + c * L::CHUNK + kk * KSTEP_BYTES, 16, 1024)
+                        : sdesc_sw128(sbase + L::OFF_W + (c * CH + kk * 16) * 128, L::W2BLK, 1024);
+                umma_bf16(dF, sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024), db, idF,
+                          (c | kk) != 0);
+              }
+            }
+            umma_commit(bar.kf_empty(fs));
+            if (++fs == L::NKF) { fs = 0; fph ^= 1; }
           }
-          umma_commit(bar.kg_empty(gs));
-          if (++gs == L::NKG) { gs = 0; gph ^= 1; }
-          if (++gst == BM / L::TKG) {
-            if (isF)
-              umma_commit(bar.ga_empty());
-            else
-              umma_commit_cluster(bar.au_empty(), (uint16_t)0x3);  // ranks 0 and 1 may refill
-            gst = 0;
-            ++gj;
-            g_open = false;
-          }
-          issued = true;
-          prefer_g = false;
-        } else {
-          if (fi >= nt) continue;
-          if (!f_open) {
-            if (!mbar_test_wait(bar.acc_empty(fi & 1), (uint32_t)(((fi >> 1) & 1) ^ 1))) continue;
-            f_open = true;
-          }
-          if (!mbar_test_wait(bar.kf_full(fs), fph)) continue;
+          if (!ok) break;
+          umma_commit(bar.acc_full(b));
+        }
+        if (i >= 1) {
+          const int j = S_.base + i - 1;
+          const bool got =
+              isF ? cwait<false>(bar.ga_full(), (uint32_t)(j & 1), abort_flag, err, kErrWaitOperand)
+                  : cwait<true>(bar.ga_full(), (uint32_t)(j & 1), abort_flag, err, kErrWaitOperand);
+          if (!got) { ok = false; break; }
+          if (!isF && j + 1 < NT) mbar_arrive_expect_tx(bar.ga_full(), 2 * L::XB);
           tc_fence_after();
-          const uint32_t a = sbase + L::OFF_KF + fs * L::CHUNK;
-          const uint32_t dF = tmem + (fi & 1) * 128;
+          for (int st = 0; st < BM / L::TKG && ok; ++st) {
+            if (!cwait<false>(bar.kg_full(gs), gph, abort_flag, err, kErrWaitFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kg = sbase + L::OFF_KG + gs * L::KG_STAGE;
 #pragma unroll
-          for (int kk = 0; kk < CH / 16; ++kk) {
-            const uint64_t db =
-                isF ? sdesc_sw128(sbase + L::OFF_W + fc * L::CHUNK + kk * KSTEP_BYTES, 16, 1024)
-                    : sdesc_sw128(sbase + L::OFF_W + (fc * CH + kk * 16) * 128, L::W2BLK, 1024);
-            umma_bf16(dF, sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024), db, idF, (fc | kk) != 0);
+            for (int kk = 0; kk < L::TKG / 16; ++kk) {
+              // A: MN-major, 2 blocks of 64 rows (LBO), 16 tokens per K step;
+              // B: MN-major, NCH blocks of 64 d (LBO = TKG rows x 128 B)
+              const uint64_t da = sdesc_sw128(ga + (st * L::TKG + kk * 16) * 128, L::XB, 1024);
+              const uint64_t db = sdesc_sw128(kg + kk * 16 * 128, L::TKG * 128, 1024);
+              umma_bf16(tmem + L::TM_G, da, db, idG, ((i - 1) | st | kk) != 0);
+            }
+            umma_commit(bar.kg_empty(gs));
+            if (++gs == L::NKG) { gs = 0; gph ^= 1; }
           }
-          umma_commit(bar.kf_empty(fs));
-          if (++fs == L::NKF) { fs = 0; fph ^= 1; }
-          if (++fc == L::NCH) {
-            umma_commit(bar.acc_full(fi & 1));
-            fc = 0;
-            ++fi;
-            f_open = false;
-          }
-          issued = true;
-          prefer_g = true;
+          if (!ok) break;
+          if (isF)
+            umma_commit(bar.ga_empty());
+          else
+            umma_commit_cluster(bar.au_empty(), (uint16_t)0x3);  // ranks 0 and 1 may refill
         }
       }
-      if (issued) {
-        last = clock64();
-      } else if (*abort_flag) {
-        ok = false;
-      } else if (clock64() - last > kWaitLimitCycles) {
-        cluster_abort(abort_flag, err, kErrWaitOperand);
-        ok = false;
-      }
+      if (ok) umma_commit(bar.g_full());
     }
-    umma_commit(bar.g_full());
     umma_commit(bar.done());
     volatile int never = 0;
     mbar_wait(bar.done(), 0, &never, err, kErrWaitFinal);
@@ -363,8 +419,8 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     // the issuing thread; this warp pays it so the epilogue does not.
     if (isF && lane == 0) {
       const uint32_t c_du_empty = mapa_shared(smem_u32(bar.du_empty(rank)), 2);
-      for (int i = 0; i < nt; ++i) {
-        if (!cwait<false>(bar.du_read(), (uint32_t)(i & 1), abort_flag, err, kErrWaitOperand))
+      for (int gi = 0; gi < NT; ++gi) {
+        if (!cwait<false>(bar.du_read(), (uint32_t)(gi & 1), abort_flag, err, kErrWaitOperand))
           break;
         mbar_arrive_remote(c_du_empty);
       }
@@ -376,268 +432,282 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     const int row = q * 32 + lane;       // token row (tiles) / accumulator row (gradient)
     const bool leader = warp == 3 && lane == 0;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const int et = threadIdx.x - 96;
+    const size_t mat = (size_t)hid * D;
     uint8_t* ga = smem + L::OFF_GA;
     uint8_t* ex = smem + L::OFF_EX;
     bool ok = true;
-    if (nt > 0) {
-      // This CTA's weights, fp32 -> bf16 (round to nearest) into the swizzled
-      // operand layout; 16-byte granule g of a 128-byte row r sits at g ^ (r % 8).
-      const int et = threadIdx.x - 96;
-      const size_t mat = (size_t)hid * D;
-      if (isF) {
-        // rows 0..63: W1, 64..127: W3 (hidden units of this CTA); a warp reads
-        // one d-row of 32 granules (D = 256) at a time
-        constexpr int GPR = D / 8;  // granules per weight row
-        for (int i = et; i < 2 * L::FH * GPR; i += L::EPI_THREADS) {
-          const int r = i / GPR, gg = i % GPR, c = gg / 8, g = gg % 8;
-          const float* src = (r < L::FH ? W1 : W3) + (size_t)head * mat +
-                             (size_t)(grp * L::GH + rank * L::FH + (r % L::FH)) * D + gg * 8;
-          const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-          const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
-          *reinterpret_cast<uint4*>(smem + L::OFF_W + c * L::CHUNK + r * 128 + ((g ^ (r & 7)) * 16)) =
-              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                         pack_bf16x2(b.z, b.w));
-        }
-      } else {
-        // W2[head][c][grp*128 + j]: d-row c, hidden units j of the group, as
-        // two blocks of 64 units; a half-warp reads one d-row (512 bytes)
-        for (int i = et; i < D * (L::GH / 8); i += L::EPI_THREADS) {
-          const int c = i / (L::GH / 8), gg = i % (L::GH / 8), blk = gg / 8, g = gg % 8;
-          const float* src = W2 + (size_t)head * mat + (size_t)c * hid + grp * L::GH + gg * 8;
-          const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-          const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
-          *reinterpret_cast<uint4*>(smem + L::OFF_W + blk * L::W2BLK + c * 128 + ((g ^ (c & 7)) * 16)) =
-              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                         pack_bf16x2(b.z, b.w));
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, L::EPI_THREADS);
-      if (leader) mbar_arrive(bar.w_full());
-    }
-    if (isF) {
-      // remote addresses in rank 2
-      const uint32_t c_au_full = mapa_shared(smem_u32(bar.ga_full()), 2);
-      const uint32_t c_au_dst = mapa_shared(smem_u32(ga + rank * L::XB), 2);
-      uint8_t* du_in = ex;
-      uint8_t* au_out = ex + L::XB;
-      // η of this thread's token row, one tile ahead (its load latency is not
-      // on the per-tile path)
-      auto eta_of = [&](int i) -> float {
-        const int64_t tok = (t0 + i) * BM + row;
-        return i < nt && tok < n ? __ldg(&eta[tok * H + head]) : 0.f;
-      };
-      float eta_next = eta_of(0);
-      for (int i = 0; i < nt; ++i) {
-        const int b = i & 1;
-        const float ne = -eta_next;  // -η (du = -W2^T v)
-        eta_next = eta_of(i + 1);
-        bool got = cwait<false>(bar.acc_full(b), (uint32_t)((i >> 1) & 1), abort_flag, err,
-                                kErrWaitAcc);
-        __syncwarp();
-        if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
-        tc_fence_after();
-        // h1, h3 of this row for hidden units [16h, 16h + 16) of this CTA
-        uint32_t r1[16], r3[16];
-        const uint32_t tl = tmem + lane_base + b * 128 + h * 16;
-        tmem_ld_16x(tl, r1);
-        tmem_ld_16x(tl + L::FH, r3);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar.acc_empty(b));
-        // η·u needs no du: form it, keep SiLU(h1) and h3·SiLU'(h1) for later
-        float sa[16], shd[16];
-        uint32_t pu[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float o_u[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const float h1 = __uint_as_float(r1[e + t]);
-            const float h3 = __uint_as_float(r3[e + t]);
-            const float sg = sigmoid_fast(h1);
-            const float a = h1 * sg;                         // SiLU(h1)
-            sa[e + t] = a;
-            shd[e + t] = h3 * fmaf(-a, sg, a + sg);          // h3·SiLU'(h1), SiLU' = s + a(1 - s)
-            o_u[t] = -ne * (a * h3);
+    // remote addresses
+    const uint32_t c_au_full = mapa_shared(smem_u32(bar.ga_full()), 2);
+    const uint32_t c_au_dst = mapa_shared(smem_u32(ga + rank * L::XB), 2);
+    const uint32_t c_du_full0 = mapa_shared(smem_u32(bar.du_full()), 0);
+    const uint32_t c_du_full1 = mapa_shared(smem_u32(bar.du_full()), 1);
+    const uint32_t c_du_dst0 = mapa_shared(smem_u32(ex), 0);
+    const uint32_t c_du_dst1 = mapa_shared(smem_u32(ex), 1);
+    uint8_t* du_in = ex;
+    uint8_t* au_out = ex + L::XB;
+    for (int sg = 0; sg < nseg && ok; ++sg) {
+      const Seg S_ = seg(sg);
+      {
+        // This segment's weights, fp32 -> bf16 (round to nearest) into the
+        // swizzled operand layout; 16-byte granule g of a 128-byte row r sits
+        // at g ^ (r % 8).  Every MMA that read the previous weights is done
+        // (the previous segment's gradient was drained after g_full).
+        if (isF) {
+          // rows 0..63: W1, 64..127: W3 (hidden units of this CTA); a warp
+          // reads one d-row of 32 granules (D = 256) at a time
+          constexpr int GPR = D / 8;  // granules per weight row
+          for (int x = et; x < 2 * L::FH * GPR; x += L::EPI_THREADS) {
+            const int r = x / GPR, gg = x % GPR, c = gg / 8, g = gg % 8;
+            const float* src = (r < L::FH ? W1 : W3) + (size_t)S_.head * mat +
+                               (size_t)(S_.grp * L::GH + rank * L::FH + (r % L::FH)) * D + gg * 8;
+            const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+            *reinterpret_cast<uint4*>(smem + L::OFF_W + c * L::CHUNK + r * 128 +
+                                      ((g ^ (r & 7)) * 16)) =
+                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                           pack_bf16x2(b.z, b.w));
           }
-          pu[e / 2] = pack_bf16x2(o_u[0], o_u[1]);
-        }
-        // η·u to rank 2, once the previous copy has read the staging buffer
-        if (leader) bulk_wait_group_read0();
-        named_bar_sync(1, L::EPI_THREADS);
-        {
-          uint8_t* r_u = au_out + row * 128;
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            *reinterpret_cast<uint4*>(r_u + (((2 * h + c) ^ (row & 7)) * 16)) =
-                make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
+        } else {
+          // W2[head][c][grp*128 + j]: d-row c, hidden units j of the group, as
+          // two blocks of 64 units; a half-warp reads one d-row (512 bytes)
+          for (int x = et; x < D * (L::GH / 8); x += L::EPI_THREADS) {
+            const int c = x / (L::GH / 8), gg = x % (L::GH / 8), blk = gg / 8, g = gg % 8;
+            const float* src =
+                W2 + (size_t)S_.head * mat + (size_t)c * hid + S_.grp * L::GH + gg * 8;
+            const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+            *reinterpret_cast<uint4*>(smem + L::OFF_W + blk * L::W2BLK + c * 128 +
+                                      ((g ^ (c & 7)) * 16)) =
+                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                           pack_bf16x2(b.z, b.w));
+          }
         }
         fence_proxy_async_smem();
         named_bar_sync(1, L::EPI_THREADS);
-        if (leader) {
-          // rank 2's P2 of the previous tile has read its η·u block
-          if (i >= 1 && !cwait<true>(bar.au_empty(), (uint32_t)((i - 1) & 1), abort_flag, err,
-                                     kErrWaitOperand)) {
-            ok = false;
-          } else {
-            bulk_copy_to_cluster(c_au_dst, au_out, L::XB, c_au_full);
-            bulk_commit_group();
-          }
-        }
-        // du of this tile from rank 2
-        got = cwait<true>(bar.du_full(), (uint32_t)(i & 1), abort_flag, err, kErrWaitOperand);
-        __syncwarp();
-        if (named_bar_any(1, L::EPI_THREADS, !got || !ok)) { ok = false; break; }
-        // every epilogue thread is past this phase: arm the next tile's du
-        if (leader && i + 1 < nt) mbar_arrive_expect_tx(bar.du_full(), L::XB);
-        uint32_t dv[8];
-        {
-          const uint8_t* rp = du_in + row * 128;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint4 t = *reinterpret_cast<const uint4*>(rp + (((2 * h + c) ^ (row & 7)) * 16));
-            dv[4 * c] = t.x; dv[4 * c + 1] = t.y; dv[4 * c + 2] = t.z; dv[4 * c + 3] = t.w;
-          }
-        }
-        uint32_t p1[8], p3[8];  // η·dh1, η·dh3 as packed bf16 pairs
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(&dv[e / 2]);
-          const float e0 = ne * __low2float(d2), e1 = ne * __high2float(d2);  // η du
-          p1[e / 2] = pack_bf16x2(e0 * shd[e], e1 * shd[e + 1]);
-          p3[e / 2] = pack_bf16x2(e0 * sa[e], e1 * sa[e + 1]);
-        }
-        // du consumed (its values are in registers): the signalling warp
-        // tells rank 2, off this path
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar.du_read());
-        // G13 of the previous tile has read the operand buffer
-        if (i >= 1) {
-          got = cwait<false>(bar.ga_empty(), (uint32_t)((i - 1) & 1), abort_flag, err,
-                             kErrWaitOperand);
+        if (leader) mbar_arrive(bar.w_full());
+      }
+      if (isF) {
+        // η of this thread's token row, one tile ahead (its load latency is
+        // not on the per-tile path)
+        auto eta_of = [&](int i) -> float {
+          const int64_t tok = (S_.ta + i) * BM + row;
+          return i < S_.nts && tok < n ? __ldg(&eta[tok * H + S_.head]) : 0.f;
+        };
+        float eta_next = eta_of(0);
+        for (int i = 0; i < S_.nts; ++i) {
+          const int gi = S_.base + i;  // tile index within the cluster (barrier phases)
+          const int b = gi & 1;
+          const float ne = -eta_next;  // -η (du = -W2^T v)
+          eta_next = eta_of(i + 1);
+          bool got = cwait<false>(bar.acc_full(b), (uint32_t)((gi >> 1) & 1), abort_flag, err,
+                                  kErrWaitAcc);
           __syncwarp();
           if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
-        }
-        {
-          uint8_t* r_1 = ga + row * 128;
-          uint8_t* r_3 = ga + L::XB + row * 128;
+          tc_fence_after();
+          // h1, h3 of this row for hidden units [16h, 16h + 16) of this CTA
+          uint32_t r1[16], r3[16];
+          const uint32_t tl = tmem + lane_base + b * 128 + h * 16;
+          tmem_ld_16x(tl, r1);
+          tmem_ld_16x(tl + L::FH, r3);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar.acc_empty(b));
+          // η·u needs no du: form it, keep SiLU(h1) and h3·SiLU'(h1) for later
+          float sa[16], shd[16];
+          uint32_t pu[8];
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int pos = ((2 * h + c) ^ (row & 7)) * 16;
-            *reinterpret_cast<uint4*>(r_1 + pos) =
-                make_uint4(p1[4 * c], p1[4 * c + 1], p1[4 * c + 2], p1[4 * c + 3]);
-            *reinterpret_cast<uint4*>(r_3 + pos) =
-                make_uint4(p3[4 * c], p3[4 * c + 1], p3[4 * c + 2], p3[4 * c + 3]);
-          }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, L::EPI_THREADS);
-        if (leader) mbar_arrive(bar.ga_full());
-      }
-      if (leader) {
-        bulk_wait_group0();
-        // the last multicast arrive from rank 2 has landed before this CTA may go
-        if (ok && nt > 0) final_wait(bar.au_empty(), (uint32_t)((nt - 1) & 1), err);
-      }
-    } else {
-      // rank 2: du of each tile to ranks 0 and 1
-      const uint32_t c_du_full[2] = {mapa_shared(smem_u32(bar.du_full()), 0),
-                                     mapa_shared(smem_u32(bar.du_full()), 1)};
-      const uint32_t c_du_dst[2] = {mapa_shared(smem_u32(ex), 0), mapa_shared(smem_u32(ex), 1)};
-      for (int i = 0; i < nt; ++i) {
-        const int b = i & 1;
-        bool got = cwait<false>(bar.acc_full(b), (uint32_t)((i >> 1) & 1), abort_flag, err,
-                                kErrWaitAcc);
-        __syncwarp();
-        if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
-        tc_fence_after();
-        // DU of this row for hidden units [32h, 32h + 32) of the group: rank h / 2's
-        // units [32(h % 2), 32(h % 2) + 32)
-        uint32_t r0[32];
-        tmem_ld_32x32(tmem + lane_base + b * 128 + h * 32, r0);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar.acc_empty(b));
-        uint32_t pk[16];
+          for (int e = 0; e < 16; e += 2) {
+            float o_u[2];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-        if (leader) bulk_wait_group_read0();
-        named_bar_sync(1, L::EPI_THREADS);
-        {
-          uint8_t* rp = ex + (h >> 1) * L::XB + row * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(rp + (((4 * (h & 1) + c) ^ (row & 7)) * 16)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, L::EPI_THREADS);
-        if (leader) {
-          for (int f = 0; f < 2 && ok; ++f) {
-            // rank f has read its previous du block
-            if (i >= 1 && !cwait<true>(bar.du_empty(f), (uint32_t)((i - 1) & 1), abort_flag, err,
-                                       kErrWaitOperand)) {
-              ok = false;
-              break;
+            for (int t = 0; t < 2; ++t) {
+              const float h1 = __uint_as_float(r1[e + t]);
+              const float h3 = __uint_as_float(r3[e + t]);
+              const float sgm = sigmoid_fast(h1);
+              const float a = h1 * sgm;                      // SiLU(h1)
+              sa[e + t] = a;
+              shd[e + t] = h3 * fmaf(-a, sgm, a + sgm);      // h3·SiLU'(h1), SiLU' = s + a(1 - s)
+              o_u[t] = -ne * (a * h3);
             }
-            bulk_copy_to_cluster(c_du_dst[f], ex + f * L::XB, L::XB, c_du_full[f]);
+            pu[e / 2] = pack_bf16x2(o_u[0], o_u[1]);
           }
-          bulk_commit_group();
+          // η·u to rank 2, once the previous copy has read the staging buffer
+          if (leader) bulk_wait_group_read0();
+          named_bar_sync(1, L::EPI_THREADS);
+          {
+            uint8_t* r_u = au_out + row * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              *reinterpret_cast<uint4*>(r_u + (((2 * h + c) ^ (row & 7)) * 16)) =
+                  make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, L::EPI_THREADS);
+          if (leader) {
+            // rank 2's P2 of the previous tile has read its η·u block
+            if (gi >= 1 && !cwait<true>(bar.au_empty(), (uint32_t)((gi - 1) & 1), abort_flag, err,
+                                        kErrWaitOperand)) {
+              ok = false;
+            } else {
+              bulk_copy_to_cluster(c_au_dst, au_out, L::XB, c_au_full);
+              bulk_commit_group();
+            }
+          }
+          // du of this tile from rank 2
+          got = cwait<true>(bar.du_full(), (uint32_t)(gi & 1), abort_flag, err, kErrWaitOperand);
+          __syncwarp();
+          if (named_bar_any(1, L::EPI_THREADS, !got || !ok)) { ok = false; break; }
+          // every epilogue thread is past this phase: arm the next tile's du
+          if (leader && gi + 1 < NT) mbar_arrive_expect_tx(bar.du_full(), L::XB);
+          uint32_t dv[8];
+          {
+            const uint8_t* rp = du_in + row * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const uint4 t = *reinterpret_cast<const uint4*>(rp + (((2 * h + c) ^ (row & 7)) * 16));
+              dv[4 * c] = t.x; dv[4 * c + 1] = t.y; dv[4 * c + 2] = t.z; dv[4 * c + 3] = t.w;
+            }
+          }
+          uint32_t p1[8], p3[8];  // η·dh1, η·dh3 as packed bf16 pairs
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(&dv[e / 2]);
+            const float e0 = ne * __low2float(d2), e1 = ne * __high2float(d2);  // η du
+            p1[e / 2] = pack_bf16x2(e0 * shd[e], e1 * shd[e + 1]);
+            p3[e / 2] = pack_bf16x2(e0 * sa[e], e1 * sa[e + 1]);
+          }
+          // du consumed (its values are in registers): the signalling warp
+          // tells rank 2, off this path
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar.du_read());
+          // the gradient MMAs of the previous tile have read the operand buffer
+          if (gi >= 1) {
+            got = cwait<false>(bar.ga_empty(), (uint32_t)((gi - 1) & 1), abort_flag, err,
+                               kErrWaitOperand);
+            __syncwarp();
+            if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
+          }
+          {
+            uint8_t* r_1 = ga + row * 128;
+            uint8_t* r_3 = ga + L::XB + row * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int pos = ((2 * h + c) ^ (row & 7)) * 16;
+              *reinterpret_cast<uint4*>(r_1 + pos) =
+                  make_uint4(p1[4 * c], p1[4 * c + 1], p1[4 * c + 2], p1[4 * c + 3]);
+              *reinterpret_cast<uint4*>(r_3 + pos) =
+                  make_uint4(p3[4 * c], p3[4 * c + 1], p3[4 * c + 2], p3[4 * c + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, L::EPI_THREADS);
+          if (leader) mbar_arrive(bar.ga_full());
         }
-        if (named_bar_any(1, L::EPI_THREADS, !ok)) { ok = false; break; }
+      } else {
+        // rank 2: du of each tile to ranks 0 and 1
+        for (int i = 0; i < S_.nts; ++i) {
+          const int gi = S_.base + i;
+          const int b = gi & 1;
+          bool got = cwait<false>(bar.acc_full(b), (uint32_t)((gi >> 1) & 1), abort_flag, err,
+                                  kErrWaitAcc);
+          __syncwarp();
+          if (named_bar_any(1, L::EPI_THREADS, !got)) { ok = false; break; }
+          tc_fence_after();
+          // DU of this row for hidden units [32h, 32h + 32) of the group: rank
+          // h / 2's units [32(h % 2), 32(h % 2) + 32)
+          uint32_t r0[32];
+          tmem_ld_32x32(tmem + lane_base + b * 128 + h * 32, r0);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar.acc_empty(b));
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+          if (leader) bulk_wait_group_read0();
+          named_bar_sync(1, L::EPI_THREADS);
+          {
+            uint8_t* rp = ex + (h >> 1) * L::XB + row * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(rp + (((4 * (h & 1) + c) ^ (row & 7)) * 16)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, L::EPI_THREADS);
+          if (leader) {
+            for (int f = 0; f < 2 && ok; ++f) {
+              // rank f has read its previous du block
+              if (gi >= 1 && !cwait<true>(bar.du_empty(f), (uint32_t)((gi - 1) & 1), abort_flag,
+                                          err, kErrWaitOperand)) {
+                ok = false;
+                break;
+              }
+              bulk_copy_to_cluster(f == 0 ? c_du_dst0 : c_du_dst1, ex + f * L::XB, L::XB,
+                                   f == 0 ? c_du_full0 : c_du_full1);
+            }
+            bulk_commit_group();
+          }
+          if (named_bar_any(1, L::EPI_THREADS, !ok)) { ok = false; break; }
+        }
       }
-      if (leader) bulk_wait_group0();
-    }
-    // ---------------------------------------------- gradient partial
-    const bool have = ok && nt > 0 &&
-                      cwait<false>(bar.g_full(), 0, abort_flag, err, kErrWaitAcc);
-    __syncwarp();
-    tc_fence_after();
-    const size_t mat = (size_t)hid * D;
-    if (ok) {
+      if (!ok) break;
+      // ---------------------------------------------- this segment's partial
+      const bool have = cwait<false>(bar.g_full(), (uint32_t)(sg & 1), abort_flag, err, kErrWaitAcc);
+      __syncwarp();
+      if (named_bar_any(1, L::EPI_THREADS, !have)) { ok = false; break; }
+      tc_fence_after();
+      // slot S_.p gets the piece; a group's last piece also zeroes the slots
+      // its group has no piece for
+      const int slots = S_.last ? S - S_.p : 1;
       if (isF) {
         // lanes 0..63: G1 rows, 64..127: G3 rows of this CTA's 64 hidden units
         const int blk = q < 2 ? 0 : 1;
-        const int hrow = grp * L::GH + rank * L::FH + (q & 1) * 32 + lane;
-        float* P = partials + (((size_t)s * H + head) * 3 + blk) * mat + (size_t)hrow * D;
-        TTT_DCHECK(hrow < hid, err, kErrCheckIndex);
+        const int hrow = S_.grp * L::GH + rank * L::FH + (q & 1) * 32 + lane;
+        TTT_DCHECK(hrow < hid && S_.p + slots <= S, err, kErrCheckIndex);
         for (int c0 = h * (D / 4); c0 < (h + 1) * (D / 4); c0 += 16) {
           uint32_t rr[16];
-          if (have) {
-            tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
-            tmem_ld_wait();
-          } else {
+          tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
+          tmem_ld_wait();
+          for (int z = 0; z < slots; ++z) {
+            float* P = partials + (((size_t)(S_.p + z) * H + S_.head) * 3 + blk) * mat +
+                       (size_t)hrow * D + c0;
+            float4* dst = reinterpret_cast<float4*>(P);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) rr[e] = 0u;
+            for (int v = 0; v < 4; ++v)
+              dst[v] = z == 0 ? make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
+                                            __uint_as_float(rr[4 * v + 2]),
+                                            __uint_as_float(rr[4 * v + 3]))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          float4* dst = reinterpret_cast<float4*>(P + c0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
-                                 __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
         }
       } else {
         // P2 rows = hidden units of the group, stored transposed as [d][hid]
-        const int j = grp * L::GH + row;
-        float* P = partials + (((size_t)s * H + head) * 3 + 2) * mat;
-        TTT_DCHECK(j < hid, err, kErrCheckIndex);
+        const int j = S_.grp * L::GH + row;
+        TTT_DCHECK(j < hid && S_.p + slots <= S, err, kErrCheckIndex);
         for (int c0 = h * (D / 4); c0 < (h + 1) * (D / 4); c0 += 16) {
           uint32_t rr[16];
-          if (have) {
-            tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
-            tmem_ld_wait();
-          } else {
+          tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
+          tmem_ld_wait();
+          for (int z = 0; z < slots; ++z) {
+            float* P = partials + (((size_t)(S_.p + z) * H + S_.head) * 3 + 2) * mat;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) rr[e] = 0u;
+            for (int e = 0; e < 16; ++e)
+              P[(size_t)(c0 + e) * hid + j] = z == 0 ? __uint_as_float(rr[e]) : 0.f;
           }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) P[(size_t)(c0 + e) * hid + j] = __uint_as_float(rr[e]);
         }
       }
+      // the gradient accumulator is free for the next segment
+      tc_fence_before();
+      named_bar_sync(1, L::EPI_THREADS);
+      if (leader) mbar_arrive(bar.g_empty());
+    }
+    if (leader) {
+      bulk_wait_group0();
+      // the last multicast arrive from rank 2 has landed before this CTA may go
+      if (isF && ok && NT > 0) final_wait(bar.au_empty(), (uint32_t)((NT - 1) & 1), err);
     }
   }
   tc_fence_before();
@@ -654,7 +724,7 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
 template <int D>
 cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2,
                               const float* W3, const void* K, const void* V, const float* eta,
-                              int S, int64_t chunk, float* partials, int* err, cudaStream_t st) {
+                              int NS, int S, float* partials, int* err, cudaStream_t st) {
   using L = FU<D>;
   CUtensorMap mK, mV, mKg, mVg;
   const uint64_t ld = (uint64_t)p.H * D;
@@ -662,7 +732,7 @@ cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2
     // {64 d, tokens, d-chunks of all heads}
     const uint64_t dims[3] = {(uint64_t)CH, (uint64_t)p.n, ld / CH};
     const uint64_t str[2] = {ld * 2, CH * 2};
-    const uint32_t boxf[3] = {CH, BM, 1};
+    const uint32_t boxf[3] = {CH, BM, (uint32_t)L::CPS};
     const uint32_t boxg[3] = {CH, L::TKG, (uint32_t)L::NCH};
     if (!make_map(&mK, K, 3, dims, str, boxf) || !make_map(&mV, V, 3, dims, str, boxf) ||
         !make_map(&mKg, K, 3, dims, str, boxg) || !make_map(&mVg, V, 3, dims, str, boxg))
@@ -670,9 +740,8 @@ cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2
   }
   cudaError_t e = ensure_smem_attr(fused_update_kernel<D>, L::SMEM);
   if (e != cudaSuccess) return e;
-  const int G = p.H * (p.hid / L::GH);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(3 * G * S));
+  cfg.gridDim = dim3((unsigned)(3 * NS * (p.hid / L::GH)));
   cfg.blockDim = dim3(L::THREADS);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = st;
@@ -685,22 +754,43 @@ cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2
   cfg.numAttrs = 1;
   TraceScope ts("tc_update_fused", st);
   return cudaLaunchKernelEx(&cfg, fused_update_kernel<D>, mK, mV, mKg, mVg, W1, W2, W3, eta,
-                            p.n, p.H, p.hid, S, chunk, partials, err);
+                            p.n, p.H, p.hid, NS, S, partials, err);
 }
 
 }  // namespace
 
 cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, const float* W3,
-                         const void* K, const void* V, const float* eta, int S, int64_t chunk,
+                         const void* K, const void* V, const float* eta, int NS, int S,
                          float* partials, int* err, cudaStream_t st) {
   if (p.d == 256)
-    return fused_update_impl<256>(p, W1, W2, W3, K, V, eta, S, chunk, partials, err, st);
-  return fused_update_impl<64>(p, W1, W2, W3, K, V, eta, S, chunk, partials, err, st);
+    return fused_update_impl<256>(p, W1, W2, W3, K, V, eta, NS, S, partials, err, st);
+  return fused_update_impl<64>(p, W1, W2, W3, K, V, eta, NS, S, partials, err, st);
 }
 
 // 3-CTA clusters of this kernel's size that are resident at once on a B200
 // (148 SMs in clusters of GPCs): 45, measured with
 // cudaOccupancyMaxActiveClusters; more clusters would run in a second wave.
 int fused_clusters_per_wave() { return 45; }
+
+FusedPlan fused_plan(const Problem& p) {
+  FusedPlan f{1, 1};
+  const int64_t ntg = (p.n + BM - 1) / BM;
+  const int groups = p.hid / 128;
+  const int64_t T = (int64_t)p.H * ntg;
+  if (T == 0) return f;
+  // as many sets of `groups` clusters as one wave holds, at least 4 tiles
+  // (512 tokens) per set: below that the 6.3 MB partials (4 heads of d 256)
+  // cost more than the parallelism gains
+  int64_t ns = fused_clusters_per_wave() / groups;
+  if (ns > T / 4) ns = T / 4;
+  if (ns < 1) ns = 1;
+  f.sets = (int)ns;
+  for (int64_t h = 0; h < p.H; ++h) {
+    const int pieces =
+        cluster_of((h + 1) * ntg - 1, f.sets, T) - cluster_of(h * ntg, f.sets, T) + 1;
+    if (pieces > f.splits) f.splits = pieces;
+  }
+  return f;
+}
 
 }  // namespace ttt

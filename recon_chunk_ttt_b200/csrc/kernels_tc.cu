@@ -395,8 +395,9 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   int* err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidDevice;
   if (p.n > 0) {
+    const FusedPlan f = fused_plan(p);
     const cudaError_t e =
-        fused_update(p, W1, W2, W3, K, V, eta, sp.S, sp.chunk, w.partials, err, st);
+        fused_update(p, W1, W2, W3, K, V, eta, f.sets, f.splits, w.partials, err, st);
     if (e != cudaSuccess) return e;
   } else {
     const cudaError_t e =
@@ -455,21 +456,9 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
 }  // namespace
 
 SplitPlan tc_split_plan(const Problem& p) {
-  // The fused update runs one 3-CTA cluster per (head, 128 hidden units,
-  // split); S splits of each group fill at most one wave of clusters,
-  // with at least 512 tokens per split (below that the fp32 partials, 6.3 MB
-  // per split for 4 heads of d 256, cost more than the parallelism gains).
-  // Every split is a whole number of 128-token tiles and none is empty.
-  const int groups = p.H * (p.hid / 128);
-  int S = fused_clusters_per_wave() / groups;
-  if (S < 1) S = 1;
-  const int64_t max_s = (p.n + 511) / 512;
-  if (S > max_s) S = (int)(max_s < 1 ? 1 : max_s);
-  int64_t chunk = (p.n + S - 1) / S;
-  chunk = (chunk + BM - 1) / BM * BM;
-  if (chunk < BM) chunk = BM;
-  if (p.n > 0) S = (int)((p.n + chunk - 1) / chunk);
-  return {S, chunk};
+  // The fused update's partial slots: see fused_plan.
+  const FusedPlan f = fused_plan(p);
+  return {f.splits, 0};
 }
 
 size_t tc_main_bytes(const Problem& p) {

@@ -9,7 +9,7 @@
 // library image, so the call itself allocates nothing.
 //
 // The array is a file-scope static __device__ object of TTT_STATIC_SCRATCH_BYTES
-// (64 MiB).  Every GPU that loads this part of the library holds it until the
+// (96 MiB).  Every GPU that loads this part of the library holds it until the
 // process exits.  Its contents persist from call to call; nothing in it needs
 // to start at zero because every kernel of the step writes the scratch it later
 // reads.  All calls on a device share the one array, so two calls whose work

@@ -76,18 +76,19 @@ def test_workspace_sizes(B):
 
 
 def test_split_plan(B):
-    """The token splits of the update: whole 128-token tiles, at least 512
-    tokens each, none empty, at most one wave of 3-CTA clusters (45 resident
-    on a B200) over all (head, 128-hidden-unit) groups, one split for small n."""
+    """The gradient slots of the update: sets of (hidden / 128) 3-CTA clusters,
+    as many as one wave holds (45 clusters resident on a B200: 11 sets for
+    hidden 512), split the head-major tile space evenly with at least 4 tiles
+    (512 tokens) per set; a head's pieces fill at most S slots."""
     cfg = _cfg(B)
     assert B.ttt_update_splits(cfg, 0) == 1
     assert B.ttt_update_splits(cfg, 1) == 1
     assert B.ttt_update_splits(cfg, 512) == 1
-    assert B.ttt_update_splits(cfg, 1374) == 2       # one 518 x 518 frame
-    assert B.ttt_update_splits(cfg, 961800) == 2     # 16 groups x 2 splits = 32 clusters
+    assert B.ttt_update_splits(cfg, 1374) == 4       # one 518 x 518 frame: 11 sets of 4 tiles
+    assert B.ttt_update_splits(cfg, 961800) == 4     # 11 sets over 4 heads
     assert B.ttt_update_splits(_cfg(B, heads=1), 961800) == 11
     assert B.ttt_update_splits(_cfg(B, heads=1, d=64, hidden=128), 108) == 1
-    assert B.ttt_update_splits(_cfg(B, heads=64), 961800) == 1
+    assert B.ttt_update_splits(_cfg(B, heads=64), 961800) == 2
     # Newton-Schulz: two d x hidden iterates, two d x d products and Delta per
     # matrix, on top of the update's own workspace (both precisions)
     for prec in (B.PREC_BF16_TC, B.PREC_FP32_CHECK):
@@ -230,30 +231,30 @@ def test_gate_partial_finish_reject_bad_arguments(B):
 
 
 def test_static_stream_step_limit_and_rejection(B):
-    """ttt_stream_step_static's fixed 64 MiB scratch, per configuration (the
+    """ttt_stream_step_static's fixed 96 MiB scratch, per configuration (the
     limits the header states): BF16_TC keeps its intermediates on chip, so 4
     heads of d = 256 fit for every n with and without Newton-Schulz, and for
-    every n up to 42 (ns_steps = 0) or 4 (ns_steps > 0) such heads fit; FP32_CHECK fits 2,471
-    tokens (678 with Newton-Schulz).  A call over the limit is rejected with
-    TTT_ERR_WORKSPACE before anything touches a device."""
-    cap = 64 << 20
+    every n up to 31 (ns_steps = 0) or 6 (ns_steps > 0) such heads fit;
+    FP32_CHECK fits 3,836 tokens (2,044 with Newton-Schulz).  A call over the
+    limit is rejected with TTT_ERR_WORKSPACE before anything touches a device."""
+    cap = 96 << 20
     ws = B.ttt_update_workspace_bytes
     for ns in (0, 5):
         cfg = _cfg(B, ns_steps=ns)
         assert ws(cfg, 1374) <= cap and ws(cfg, 10**9) <= cap
-    assert ws(_cfg(B, heads=42), 10**9) <= cap < ws(_cfg(B, heads=43), 1)
-    assert ws(_cfg(B, heads=4, ns_steps=5), 10**9) <= cap < ws(_cfg(B, heads=5, ns_steps=5), 10**9)
+    assert ws(_cfg(B, heads=31), 10**9) <= cap < ws(_cfg(B, heads=32), 10**9)
+    assert ws(_cfg(B, heads=6, ns_steps=5), 10**9) <= cap < ws(_cfg(B, heads=7, ns_steps=5), 10**9)
     f32 = _cfg(B, precision=B.PREC_FP32_CHECK)
     f32ns = _cfg(B, precision=B.PREC_FP32_CHECK, ns_steps=5)
-    assert ws(f32, 2471) <= cap < ws(f32, 2472)
-    assert ws(f32ns, 678) <= cap < ws(f32ns, 679)
-    assert ws(f32, 1374) <= cap < ws(f32ns, 1374)   # one frame: fits without Newton-Schulz
+    assert ws(f32, 3836) <= cap < ws(f32, 3837)
+    assert ws(f32ns, 2044) <= cap < ws(f32ns, 2045)
+    assert ws(f32, 1374) <= cap and ws(f32ns, 1374) <= cap   # one frame fits either way
     L = B.lib()
     f = L.ttt_stream_step_static
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f.argtypes = [ctypes.POINTER(B.ttt_config), P, P, P, P, P, P, P, I64, P, I64, P, P]
     f.restype = ctypes.c_int
-    for cfg, n in ((f32, 2472), (f32ns, 1374), (_cfg(B, heads=43), 10)):
+    for cfg, n in ((f32, 3837), (f32ns, 2045), (_cfg(B, heads=32), 10**6)):
         args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n, FAKE, 5, FAKE, None]
         assert f(ctypes.byref(cfg), *args) == B.TTT_ERR_WORKSPACE
     assert f(None, *[FAKE] * 7, 5, FAKE, 5, FAKE, None) == B.TTT_ERR_INVALID_ARG

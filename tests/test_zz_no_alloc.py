@@ -87,7 +87,7 @@ def test_static_scratch_rejects_oversized_problem():
     cfg = R.make_config(4, 256, 512, precision=R.PREC_FP32_CHECK)
     fn = _static_fn()
     n = 200000  # needs far more than the fixed array
-    assert R.ttt_update_workspace_bytes(cfg, n) > (64 << 20)
+    assert R.ttt_update_workspace_bytes(cfg, n) > (96 << 20)
     fake = 0x10000
     st = fn(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake, fake, n, fake, n, fake, None)
     assert st == 4, R.status_string(st)  # TTT_ERR_WORKSPACE, nothing launched
