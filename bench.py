@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--no-ns-probe", action="store_true",
                     help="skip the separate 5-step Newton-Schulz update measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--only-stream", action="store_true",
+                    help="run only the streaming measurement (stream256, one frame per "
+                         "ttt_stream_step) and print its JSON object")
     return ap.parse_args()
 
 
@@ -732,8 +735,22 @@ def kernel_source_sha(files=None) -> str:
     return h.hexdigest()[:16]
 
 
+def run_stream_only():
+    """The streaming row alone on one GPU (used to profile a frame's kernels)."""
+    import torch
+    import recon_chunk_ttt_b200 as R
+    from recon_chunk_ttt_b200 import build as B
+    B.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    print(json.dumps({"stream": stream_bench(R, torch, dev, lambda v: v)}), flush=True)
+
+
 def main():
     args = parse()
+    if args.only_stream:
+        run_stream_only()
+        return
     world, rank, local = dist_setup(args)
     w = wl.WORKLOADS[args.workload]
     if args.impl == "reference":

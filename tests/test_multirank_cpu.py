@@ -63,14 +63,14 @@ def test_reference_arm_runs_on_rank0_only():
     assert r.stdout.strip() == ""
 
 
-def test_roofline_entry_picks_the_binding_resource():
+def test_roofline_entry_rates_the_declared_resource():
+    """The bound is the algorithm's (tensor for the GEMM kernels, HBM for the
+    elementwise ones), given by the caller; the rate is work / time."""
     sys.path.insert(0, ROOT)
     import bench
     pk = {"hbm_gbs": 6549.4, "bf16_tflops": 1586.2, "bf16_tflops_sustained": 1372.0}
-    # 192 flop/B is below the ridge (1372/6.5494 = 209 flop/B): HBM bound
-    e = bench.roofline_entry("k", 192e9, 1e9, 1.0, pk)
+    e = bench.roofline_entry(192e9, 1e9, 1.0, pk, "hbm")
     assert e["bound"] == "hbm" and e["unit"] == "GB/s"
     assert e["achieved"] == pytest.approx(1e9 / 1e-3 / 1e9)
-    # 768 flop/B: tensor bound
-    e = bench.roofline_entry("k", 768e9, 1e9, 1.0, pk)
+    e = bench.roofline_entry(768e9, 1e9, 1.0, pk, "tensor")
     assert e["bound"] == "tensor" and e["achieved"] == pytest.approx(768.0)
