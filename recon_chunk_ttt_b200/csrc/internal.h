@@ -75,16 +75,17 @@ cudaError_t tc_apply(const Problem& p, const __nv_bfloat16_raw* shadow, const vo
                      cudaStream_t st);
 // Fused update kernel (kernels_fused.cu): fp32 weights W1, W3 [H][hid][d],
 // W2 [H][d][hid] in (rounded to bf16 inside); the S partial slots of the
-// plan out ([S][H][3][hid*d]).  The head-major tile space is split evenly
-// over `sets` sets of hid/128 3-CTA clusters (one per group of 128 hidden
-// units); a head's gradient arrives in at most `splits` pieces (slots),
-// unused slots are zero.
+// plan out ([S][H][3][hid*d]).  The head-major tile space is split over
+// `sets` sets of hid/128 3-CTA clusters (one per group of 128 hidden units):
+// evenly over the whole space (sets_per_head = 0), or, for few tiles per
+// head, sets_per_head sets per head; a head's gradient arrives in at most
+// `splits` pieces (slots), unused slots are zero.
 struct FusedPlan {
-  int sets, splits;
+  int sets, sets_per_head, splits;
 };
 FusedPlan fused_plan(const Problem& p);
 cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, const float* W3,
-                         const void* K, const void* V, const float* eta, int NS, int S,
+                         const void* K, const void* V, const float* eta, const FusedPlan& f,
                          float* partials, int* err, cudaStream_t st);
 // Clusters of the fused update that fill one wave of the GPU.
 int fused_clusters_per_wave();

@@ -153,6 +153,10 @@ __device__ __forceinline__ void final_wait(uint64_t* bar, uint32_t parity, int* 
 // goes to partial slot p; slots a head has no piece for are written as zeros
 // by the set holding its last piece.  All of it is a function of (n, shape,
 // NS), so the split sums are fixed.
+// For small n (few tiles per head) a range that crosses a head would pay a
+// second weight staging and gradient drain on a short critical path, so the
+// sets are instead aligned to heads: SPH sets per head, each a contiguous
+// part of one head's tiles (one segment, piece = part).
 struct Seg {
   int head, grp;     // group of the segment
   int64_t ta;        // first tile of the segment within its group
@@ -164,6 +168,10 @@ struct Seg {
 __host__ __device__ __forceinline__ int64_t range_lo(int c, int NC, int64_t T) {
   return (int64_t)c * T / NC;
 }
+// Start of set c's range when the sets are aligned to heads, SPH per head.
+__host__ __device__ __forceinline__ int64_t aligned_lo(int c, int SPH, int64_t ntg) {
+  return (int64_t)(c / SPH) * ntg + (int64_t)(c % SPH) * ntg / SPH;
+}
 // The set whose range holds tile index x of the head-major space.
 __host__ __device__ __forceinline__ int cluster_of(int64_t x, int NC, int64_t T) {
   int c = (int)(x * NC / T);
@@ -171,7 +179,21 @@ __host__ __device__ __forceinline__ int cluster_of(int64_t x, int NC, int64_t T)
   while (c + 1 < NC && range_lo(c + 1, NC, T) <= x) ++c;
   return c;
 }
-__device__ __forceinline__ Seg make_seg(int c, int NC, int64_t T, int64_t ntg, int grp, int sg) {
+__device__ __forceinline__ Seg make_seg(int c, int NC, int SPH, int64_t T, int64_t ntg, int grp,
+                                        int sg) {
+  if (SPH > 0) {
+    // head-aligned: one segment, piece = part of the head
+    const int64_t a = aligned_lo(c, SPH, ntg), b = aligned_lo(c + 1, SPH, ntg);
+    Seg s;
+    s.head = c / SPH;
+    s.grp = grp;
+    s.ta = a - (int64_t)s.head * ntg;
+    s.nts = (int)(b - a);
+    s.base = 0;
+    s.p = c % SPH;
+    s.last = s.p == SPH - 1;
+    return s;
+  }
   const int64_t lo = range_lo(c, NC, T), hi = range_lo(c + 1, NC, T);
   const int64_t g = lo / ntg + sg;  // head
   const int64_t a = g * ntg > lo ? g * ntg : lo;
@@ -194,7 +216,7 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
                         const __grid_constant__ CUtensorMap mVg,
                         const float* __restrict__ W1, const float* __restrict__ W2,
                         const float* __restrict__ W3, const float* __restrict__ eta,
-                        int64_t n, int H, int hid, int NS, int S,
+                        int64_t n, int H, int hid, int NS, int SPH, int S,
                         float* __restrict__ partials, int* err) {
   using L = FU<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -210,10 +232,11 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
   const int set = blockIdx.x / 3 / groups, grp = blockIdx.x / 3 % groups;
   const int64_t ntg = (n + BM - 1) / BM;
   const int64_t T = (int64_t)H * ntg;
-  const int64_t lo = range_lo(set, NS, T), hi = range_lo(set + 1, NS, T);
+  const int64_t lo = SPH > 0 ? aligned_lo(set, SPH, ntg) : range_lo(set, NS, T);
+  const int64_t hi = SPH > 0 ? aligned_lo(set + 1, SPH, ntg) : range_lo(set + 1, NS, T);
   const int NT = (int)(hi - lo);                        // tiles of this cluster
-  const int nseg = NT > 0 ? (int)((hi - 1) / ntg - lo / ntg + 1) : 0;
-  auto seg = [&](int sg) { return make_seg(set, NS, T, ntg, grp, sg); };
+  const int nseg = NT <= 0 ? 0 : SPH > 0 ? 1 : (int)((hi - 1) / ntg - lo / ntg + 1);
+  auto seg = [&](int sg) { return make_seg(set, NS, SPH, T, ntg, grp, sg); };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NKF; ++i) {
@@ -453,34 +476,54 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
         // swizzled operand layout; 16-byte granule g of a 128-byte row r sits
         // at g ^ (r % 8).  Every MMA that read the previous weights is done
         // (the previous segment's gradient was drained after g_full).
+        // Both roles stage 2 * 64 * D / 8 (F) or D * 128 / 8 (rank 2) 8-element
+        // granules: the same count, NG per thread; all of a thread's loads are
+        // issued before its stores so their latencies overlap.
+        constexpr int NG = (L::GH * D / 8) / L::EPI_THREADS;
+        static_assert(NG * L::EPI_THREADS == L::GH * D / 8, "granules per thread");
+        float4 wa[NG], wb[NG];
         if (isF) {
           // rows 0..63: W1, 64..127: W3 (hidden units of this CTA); a warp
           // reads one d-row of 32 granules (D = 256) at a time
           constexpr int GPR = D / 8;  // granules per weight row
-          for (int x = et; x < 2 * L::FH * GPR; x += L::EPI_THREADS) {
-            const int r = x / GPR, gg = x % GPR, c = gg / 8, g = gg % 8;
+#pragma unroll
+          for (int k = 0; k < NG; ++k) {
+            const int x = et + k * L::EPI_THREADS;
+            const int r = x / GPR, gg = x % GPR;
             const float* src = (r < L::FH ? W1 : W3) + (size_t)S_.head * mat +
                                (size_t)(S_.grp * L::GH + rank * L::FH + (r % L::FH)) * D + gg * 8;
-            const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+            wa[k] = __ldg(reinterpret_cast<const float4*>(src));
+            wb[k] = __ldg(reinterpret_cast<const float4*>(src + 4));
+          }
+#pragma unroll
+          for (int k = 0; k < NG; ++k) {
+            const int x = et + k * L::EPI_THREADS;
+            const int r = x / GPR, gg = x % GPR, c = gg / 8, g = gg % 8;
             *reinterpret_cast<uint4*>(smem + L::OFF_W + c * L::CHUNK + r * 128 +
                                       ((g ^ (r & 7)) * 16)) =
-                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                           pack_bf16x2(b.z, b.w));
+                make_uint4(pack_bf16x2(wa[k].x, wa[k].y), pack_bf16x2(wa[k].z, wa[k].w),
+                           pack_bf16x2(wb[k].x, wb[k].y), pack_bf16x2(wb[k].z, wb[k].w));
           }
         } else {
           // W2[head][c][grp*128 + j]: d-row c, hidden units j of the group, as
           // two blocks of 64 units; a half-warp reads one d-row (512 bytes)
-          for (int x = et; x < D * (L::GH / 8); x += L::EPI_THREADS) {
-            const int c = x / (L::GH / 8), gg = x % (L::GH / 8), blk = gg / 8, g = gg % 8;
+#pragma unroll
+          for (int k = 0; k < NG; ++k) {
+            const int x = et + k * L::EPI_THREADS;
+            const int c = x / (L::GH / 8), gg = x % (L::GH / 8);
             const float* src =
                 W2 + (size_t)S_.head * mat + (size_t)c * hid + S_.grp * L::GH + gg * 8;
-            const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
+            wa[k] = __ldg(reinterpret_cast<const float4*>(src));
+            wb[k] = __ldg(reinterpret_cast<const float4*>(src + 4));
+          }
+#pragma unroll
+          for (int k = 0; k < NG; ++k) {
+            const int x = et + k * L::EPI_THREADS;
+            const int c = x / (L::GH / 8), gg = x % (L::GH / 8), blk = gg / 8, g = gg % 8;
             *reinterpret_cast<uint4*>(smem + L::OFF_W + blk * L::W2BLK + c * 128 +
                                       ((g ^ (c & 7)) * 16)) =
-                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                           pack_bf16x2(b.z, b.w));
+                make_uint4(pack_bf16x2(wa[k].x, wa[k].y), pack_bf16x2(wa[k].z, wa[k].w),
+                           pack_bf16x2(wb[k].x, wb[k].y), pack_bf16x2(wb[k].z, wb[k].w));
           }
         }
         fence_proxy_async_smem();
@@ -724,7 +767,8 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
 template <int D>
 cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2,
                               const float* W3, const void* K, const void* V, const float* eta,
-                              int NS, int S, float* partials, int* err, cudaStream_t st) {
+                              int NS, int SPH, int S, float* partials, int* err,
+                              cudaStream_t st) {
   using L = FU<D>;
   CUtensorMap mK, mV, mKg, mVg;
   const uint64_t ld = (uint64_t)p.H * D;
@@ -754,17 +798,19 @@ cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2
   cfg.numAttrs = 1;
   TraceScope ts("tc_update_fused", st);
   return cudaLaunchKernelEx(&cfg, fused_update_kernel<D>, mK, mV, mKg, mVg, W1, W2, W3, eta,
-                            p.n, p.H, p.hid, NS, S, partials, err);
+                            p.n, p.H, p.hid, NS, SPH, S, partials, err);
 }
 
 }  // namespace
 
 cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, const float* W3,
-                         const void* K, const void* V, const float* eta, int NS, int S,
+                         const void* K, const void* V, const float* eta, const FusedPlan& f,
                          float* partials, int* err, cudaStream_t st) {
   if (p.d == 256)
-    return fused_update_impl<256>(p, W1, W2, W3, K, V, eta, NS, S, partials, err, st);
-  return fused_update_impl<64>(p, W1, W2, W3, K, V, eta, NS, S, partials, err, st);
+    return fused_update_impl<256>(p, W1, W2, W3, K, V, eta, f.sets, f.sets_per_head, f.splits,
+                                  partials, err, st);
+  return fused_update_impl<64>(p, W1, W2, W3, K, V, eta, f.sets, f.sets_per_head, f.splits,
+                               partials, err, st);
 }
 
 // 3-CTA clusters of this kernel's size that are resident at once on a B200
@@ -773,11 +819,23 @@ cudaError_t fused_update(const Problem& p, const float* W1, const float* W2, con
 int fused_clusters_per_wave() { return 45; }
 
 FusedPlan fused_plan(const Problem& p) {
-  FusedPlan f{1, 1};
+  FusedPlan f{1, 0, 1};
   const int64_t ntg = (p.n + BM - 1) / BM;
   const int groups = p.hid / 128;
   const int64_t T = (int64_t)p.H * ntg;
   if (T == 0) return f;
+  // Few tiles per head (up to 64: 8,192 tokens): sets aligned to heads, as
+  // many per head as one wave holds, at least 4 tiles each.
+  const int per_wave = fused_clusters_per_wave() / groups;
+  if (ntg <= 64 && per_wave >= p.H) {
+    int64_t sph = per_wave / p.H;
+    if (sph > ntg / 4) sph = ntg / 4;
+    if (sph < 1) sph = 1;
+    f.sets_per_head = (int)sph;
+    f.sets = (int)(sph * p.H);
+    f.splits = (int)sph;
+    return f;
+  }
   // as many sets of `groups` clusters as one wave holds, at least 4 tiles
   // (512 tokens) per set: below that the 6.3 MB partials (4 heads of d 256)
   // cost more than the parallelism gains

@@ -397,7 +397,7 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
   if (p.n > 0) {
     const FusedPlan f = fused_plan(p);
     const cudaError_t e =
-        fused_update(p, W1, W2, W3, K, V, eta, f.sets, f.splits, w.partials, err, st);
+        fused_update(p, W1, W2, W3, K, V, eta, f, w.partials, err, st);
     if (e != cudaSuccess) return e;
   } else {
     const cudaError_t e =

@@ -79,12 +79,15 @@ def test_split_plan(B):
     """The gradient slots of the update: sets of (hidden / 128) 3-CTA clusters,
     as many as one wave holds (45 clusters resident on a B200: 11 sets for
     hidden 512), split the head-major tile space evenly with at least 4 tiles
-    (512 tokens) per set; a head's pieces fill at most S slots."""
+    (512 tokens) per set, or, with at most 64 tiles per head, are aligned to
+    heads (one slot per set of a head); a head's pieces fill at most S slots."""
     cfg = _cfg(B)
     assert B.ttt_update_splits(cfg, 0) == 1
     assert B.ttt_update_splits(cfg, 1) == 1
     assert B.ttt_update_splits(cfg, 512) == 1
-    assert B.ttt_update_splits(cfg, 1374) == 4       # one 518 x 518 frame: 11 sets of 4 tiles
+    assert B.ttt_update_splits(cfg, 8192) == 2       # 64 tiles per head, aligned
+    assert B.ttt_update_splits(cfg, 8193) == 4       # 65 tiles per head: 11 sets over 4 heads
+    assert B.ttt_update_splits(cfg, 1374) == 2       # one 518 x 518 frame: 2 sets per head
     assert B.ttt_update_splits(cfg, 961800) == 4     # 11 sets over 4 heads
     assert B.ttt_update_splits(_cfg(B, heads=1), 961800) == 11
     assert B.ttt_update_splits(_cfg(B, heads=1, d=64, hidden=128), 108) == 1
