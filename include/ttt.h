@@ -46,7 +46,8 @@
  *                 layout as W1, W3, W2 (W1 block, then W3, then W2);
  *                 ttt_shadow_bytes() bytes.
  *  - Device pointers must be 16-byte aligned (tensor-memory-access rule).
- *  - Supported shapes: (d, hidden) = (64, 128) or (256, 512), heads >= 1.
+ *  - Supported shapes: (d, hidden) = (64, 128) or (256, 512), heads >= 1
+ *    (linear mode: (64, 64) or (256, 256)).
  *  - n = 0 or eta = 0 gives Ŵ = W.  Outputs may alias the weight inputs
  *    (in-place update); K, V, Q, eta and O must not alias outputs.
  *  - Results are deterministic run to run (fixed-order reductions, no
@@ -75,7 +76,19 @@ typedef enum {
   TTT_ERR_DEVICE = 6             /* a kernel gave up a bounded wait         */
 } ttt_status;
 
-enum { TTT_MLP_SWIGLU = 0 };
+/* Fast-weight form.  TTT_MLP_SWIGLU: the layer above.  TTT_MLP_LINEAR:
+ * f_W(k) = W k with one d x d matrix per head (67656.sbs reading notes,
+ * section "为什么它像 attention（线性情形的直观推导）"), for which one step has
+ * the closed form Ŵ = W + Σ_i η_i v_i k_i^T (before the renormalisation) and
+ * the read o = Ŵ q is an un-normalised linear attention.  In linear mode
+ * hidden must equal d, ns_steps must be 0, W is passed as W1 ([H][d][d],
+ * row = output), W2 and W3 (and W2_out, W3_out) are unused and may be NULL,
+ * the shadow holds the one bf16 matrix (H * d * d * 2 bytes) and partials
+ * are [H][1][d*d] holding Σ η v k^T (= -g).  Its two contractions run on
+ * CUDA cores with fp32 arithmetic in both precisions (BF16_TC reads bf16
+ * tokens and the bf16 shadow and writes bf16 outputs); it is a reference
+ * mode for that closed form, not the benchmarked layer. */
+enum { TTT_MLP_SWIGLU = 0, TTT_MLP_LINEAR = 1 };
 enum { TTT_RENORM_OFF = 0, TTT_RENORM_ROW = 1, TTT_RENORM_FROB = 2 };
 enum { TTT_PREC_BF16_TC = 0, TTT_PREC_FP32_CHECK = 1 };
 enum { TTT_MAX_NS_STEPS = 32 };
@@ -84,7 +97,7 @@ typedef struct {
   int32_t heads;     /* H, number of independent fast-weight MLPs          */
   int32_t d;         /* head dimension (64 or 256)                         */
   int32_t hidden;    /* fast-weight hidden width (128 or 512)              */
-  int32_t mlp;       /* TTT_MLP_SWIGLU                                     */
+  int32_t mlp;       /* TTT_MLP_SWIGLU or TTT_MLP_LINEAR                   */
   int32_t renorm;    /* TTT_RENORM_*                                       */
   int32_t ns_steps;  /* Newton–Schulz steps on g: 0 (off) .. TTT_MAX_NS_STEPS */
   int32_t precision; /* TTT_PREC_BF16_TC: bf16 tensor-core operands, fp32
@@ -99,7 +112,8 @@ const char* ttt_status_string(ttt_status s);
  * (0 if the config is invalid). */
 size_t ttt_update_workspace_bytes(const ttt_config* cfg, int64_t n_tokens);
 
-/* Bytes of the bf16 weight shadow (3 * H * d * hidden * 2). */
+/* Bytes of the bf16 weight shadow (3 * H * d * hidden * 2; linear mode
+ * H * d * d * 2). */
 size_t ttt_shadow_bytes(const ttt_config* cfg);
 
 /* Number of token splits S the update of n tokens reduces: the gradient is

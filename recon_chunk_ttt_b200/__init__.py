@@ -23,7 +23,7 @@ _EXPORTS = {
     "ttt_update_partial", "ttt_update_finish", "ttt_gate", "GATE_EPS", "ttt_update_splits",
     "ttt_selftest_wait_timeout", "DEVICE_ERR_SELFTEST", "TTT_OK", "TTT_ERR_INVALID_ARG",
     "TTT_ERR_UNSUPPORTED_SHAPE", "TTT_ERR_ALIGNMENT", "TTT_ERR_WORKSPACE", "TTT_ERR_CUDA",
-    "TTT_ERR_DEVICE",
+    "TTT_ERR_DEVICE", "MLP_SWIGLU", "MLP_LINEAR",
 }
 
 

@@ -21,7 +21,7 @@ LIB_PATH = os.environ.get("RECON_CHUNK_TTT_LIB") or os.path.join(_HERE, "libttt.
 TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED_SHAPE, TTT_ERR_ALIGNMENT, \
     TTT_ERR_WORKSPACE, TTT_ERR_CUDA, TTT_ERR_DEVICE = range(7)
 MAX_NS_STEPS = 32  # TTT_MAX_NS_STEPS
-MLP_SWIGLU = 0
+MLP_SWIGLU, MLP_LINEAR = 0, 1
 RENORM_OFF, RENORM_ROW, RENORM_FROB = 0, 1, 2
 PREC_BF16_TC, PREC_FP32_CHECK = 0, 1
 
@@ -160,8 +160,8 @@ def ttt_update(cfg: ttt_config, W1, W2, W3, K, V, eta, W1_out=None, W2_out=None,
     """Ŵ = renorm(W - ∇_W Σ η_i (-f_W(k_i)^T v_i)); returns (W1_out, W2_out, W3_out)."""
     n = int(K.shape[0]) if K is not None else 0
     W1_out = torch.empty_like(W1) if W1_out is None else W1_out
-    W2_out = torch.empty_like(W2) if W2_out is None else W2_out
-    W3_out = torch.empty_like(W3) if W3_out is None else W3_out
+    W2_out = torch.empty_like(W2) if W2_out is None and W2 is not None else W2_out
+    W3_out = torch.empty_like(W3) if W3_out is None and W3 is not None else W3_out
     if workspace is None:
         workspace = alloc_workspace(cfg, n, W1.device)
     nbytes = workspace.numel() * workspace.element_size()
@@ -251,7 +251,7 @@ def ttt_update_finish(cfg: ttt_config, W1, W2, W3, partials, W1_out=None, W2_out
     """Ŵ from the ranks' partials ([ranks, partial_floats], summed in rank
     order); returns (W1_out, W2_out, W3_out)."""
     ranks = int(partials.shape[0]) if partials.dim() == 2 else 1
-    outs = [o if o is not None else torch.empty_like(w)
+    outs = [o if o is not None or w is None else torch.empty_like(w)
             for o, w in ((W1_out, W1), (W2_out, W2), (W3_out, W3))]
     if workspace is None:
         workspace = torch.empty(max(ttt_finish_workspace_bytes(cfg), 1), dtype=torch.uint8,

@@ -12,8 +12,13 @@
 
 namespace ttt {
 
+// Fast-weight forms (ttt_config.mlp).
+constexpr int kMlpSwiGLU = 0;
+constexpr int kMlpLinear = 1;
+
 // Problem description after validation.
 struct Problem {
+  int mlp;    // kMlpSwiGLU or kMlpLinear (then hid == d and W1 is the d x d W)
   int H, d, hid;
   int64_t n;  // tokens (update) or queries (apply)
   int renorm;
@@ -61,8 +66,22 @@ cudaError_t ns_then_renorm(const Problem& p, int S, const float* partials, void*
                            float* scratch, cudaStream_t st);
 // out[i] = sum over s = 0..S-1 of partials[s * count + i], in that order.
 cudaError_t sum_splits(int S, size_t count, const float* partials, float* out, cudaStream_t st);
+// W2 and W3 may be NULL (linear fast weights: only the W1 block is written).
 cudaError_t pack_shadow(int H, int d, int hid, const float* W1, const float* W2,
                         const float* W3, __nv_bfloat16_raw* shadow, cudaStream_t st);
+
+// ---- linear fast weights f_W(k) = W k (kernels_linear.cu) ------------------
+// Partials [S][H][d*d] hold P = Σ η v k^T (= -g); the update adds them.
+SplitPlan linear_split_plan(const Problem& p);
+size_t linear_workspace_bytes(const Problem& p);
+cudaError_t linear_update(const Problem& p, bool bf16_tokens, const float* W, const void* K,
+                          const void* V, const float* eta, float* Wo,
+                          __nv_bfloat16_raw* shadow, void* ws, cudaStream_t st,
+                          float* partial_out = nullptr);
+// BF16_TC (bf16 = true) reads the bf16 shadow of W, FP32_CHECK the fp32 W.
+cudaError_t linear_apply(const Problem& p, bool bf16, const float* W,
+                         const __nv_bfloat16_raw* shadow, const void* Q, void* O,
+                         cudaStream_t st);
 
 // ---- bf16 tensor-core path (tcgen05) --------------------------------------
 SplitPlan tc_split_plan(const Problem& p);

@@ -140,22 +140,31 @@ __device__ __forceinline__ void renorm_row(const float* __restrict__ P0, size_t 
   }
 }
 
+// nblk = 3: the SwiGLU layer (blocks W1, W3, W2 per head, partials P1 = G1,
+// P3 = G3, P2 = -G2).  nblk = 1: linear fast weights (W1 = W, d x d, partial
+// P = -g = Σ η v k^T, added).
 __global__ void __launch_bounds__(256, 2) reduce_renorm_kernel(
-    const float* __restrict__ partials, int S, int H, int d, int hid, int mode,
+    const float* __restrict__ partials, int S, int H, int d, int hid, int nblk, int mode,
     const float* W1, const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
     __nv_bfloat16_raw* __restrict__ shadow, double* __restrict__ scratch) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= H * (2 * hid + d)) return;
-  const RowRef r = decode_row(warp, d, hid);
+  const int per = nblk == 3 ? 2 * hid + d : d;
+  if (warp >= H * per) return;
+  RowRef r;
+  if (nblk == 3) {
+    r = decode_row(warp, d, hid);
+  } else {
+    r.head = warp / d; r.blk = 0; r.row = warp % d; r.len = d;
+  }
   const size_t mat = (size_t)hid * d;
   const float* W = r.blk == 0 ? W1 : r.blk == 1 ? W3 : W2;
   float* Wo = r.blk == 0 ? W1o : r.blk == 1 ? W3o : W2o;
   const size_t base = (size_t)r.head * mat + (size_t)r.row * r.len;
-  // P1, P3 are G1, G3 (subtract); P2 is -G2 (add).  Partial block = blk.
-  const double sign = r.blk == 2 ? 1.0 : -1.0;
-  const size_t sstride = (size_t)H * 3 * mat;  // one split
-  const float* P = partials + ((size_t)r.head * 3 + r.blk) * mat + (size_t)r.row * r.len;
+  // P1, P3 are G1, G3 (subtract); P2 is -G2 and the linear P is -g (add).
+  const double sign = r.blk == 2 || nblk == 1 ? 1.0 : -1.0;
+  const size_t sstride = (size_t)H * nblk * mat;  // one split
+  const float* P = partials + ((size_t)r.head * nblk + r.blk) * mat + (size_t)r.row * r.len;
   // the shadow (W1 | W3 | W2 blocks) is written here unless the Frobenius
   // scale still has to be applied
   __nv_bfloat16_raw* sh = shadow != nullptr && mode != 2 ? shadow + (size_t)r.blk * H * mat
@@ -180,10 +189,10 @@ __global__ void __launch_bounds__(256, 2) reduce_renorm_kernel(
 // Frobenius mode: one block per (head, matrix).  Sums the per-row squares in
 // row order, then rescales the matrix in place and writes the shadow.
 __global__ void __launch_bounds__(256) frob_scale_kernel(
-    int H, int d, int hid, const double* __restrict__ scratch, float* W1o, float* W2o,
+    int H, int d, int hid, int nblk, const double* __restrict__ scratch, float* W1o, float* W2o,
     float* W3o, __nv_bfloat16_raw* __restrict__ shadow) {
-  const int head = blockIdx.x / 3, blk = blockIdx.x % 3;
-  const int per = 2 * hid + d;
+  const int head = blockIdx.x / nblk, blk = blockIdx.x % nblk;
+  const int per = nblk == 3 ? 2 * hid + d : d;
   const int r0 = head * per + (blk == 0 ? 0 : blk == 1 ? hid : 2 * hid);
   const int rows = blk == 2 ? d : hid;
   __shared__ double sc;
@@ -213,8 +222,8 @@ __global__ void pack_shadow_kernel(size_t mat_total, const float* __restrict__ W
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < mat_total;
        i += (size_t)gridDim.x * blockDim.x) {
     shadow[i] = to_bf16_raw(W1[i]);
-    shadow[mat_total + i] = to_bf16_raw(W3[i]);
-    shadow[2 * mat_total + i] = to_bf16_raw(W2[i]);
+    if (W3 != nullptr) shadow[mat_total + i] = to_bf16_raw(W3[i]);
+    if (W2 != nullptr) shadow[2 * mat_total + i] = to_bf16_raw(W2[i]);
   }
 }
 
@@ -256,15 +265,17 @@ __global__ void selftest_timeout_kernel(long long limit, int* err) {
 cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const float* W1,
                           const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
                           __nv_bfloat16_raw* shadow, float* scratch, cudaStream_t st) {
-  const int rows = p.H * (2 * p.hid + p.d);
+  const int nblk = p.mlp == kMlpLinear ? 1 : 3;
+  const int rows = p.H * (nblk == 3 ? 2 * p.hid + p.d : p.d);
   const int blocks = (rows * 32 + 255) / 256;
   TraceScope ts("reduce_renorm", st);
-  reduce_renorm_kernel<<<blocks, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, p.renorm, W1, W2,
-                                              W3, W1o, W2o, W3o, shadow,
+  reduce_renorm_kernel<<<blocks, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, nblk, p.renorm, W1,
+                                              W2, W3, W1o, W2o, W3o, shadow,
                                               reinterpret_cast<double*>(scratch));
   if (p.renorm == 2)
-    frob_scale_kernel<<<p.H * 3, 256, 0, st>>>(p.H, p.d, p.hid, reinterpret_cast<double*>(scratch),
-                                              W1o, W2o, W3o, shadow);
+    frob_scale_kernel<<<p.H * nblk, 256, 0, st>>>(p.H, p.d, p.hid, nblk,
+                                                 reinterpret_cast<double*>(scratch), W1o, W2o,
+                                                 W3o, shadow);
   return cudaGetLastError();
 }
 

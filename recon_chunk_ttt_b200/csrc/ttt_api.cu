@@ -17,18 +17,35 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 ttt_status check_cfg(const ttt_config* cfg) {
   if (cfg == nullptr) return TTT_ERR_INVALID_ARG;
   if (cfg->heads < 1 || cfg->heads > 4096) return TTT_ERR_INVALID_ARG;
-  if (cfg->mlp != TTT_MLP_SWIGLU) return TTT_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->mlp != TTT_MLP_SWIGLU && cfg->mlp != TTT_MLP_LINEAR) return TTT_ERR_INVALID_ARG;
   if (cfg->renorm < TTT_RENORM_OFF || cfg->renorm > TTT_RENORM_FROB) return TTT_ERR_INVALID_ARG;
   if (cfg->precision != TTT_PREC_BF16_TC && cfg->precision != TTT_PREC_FP32_CHECK)
     return TTT_ERR_INVALID_ARG;
   if (cfg->ns_steps < 0 || cfg->ns_steps > TTT_MAX_NS_STEPS) return TTT_ERR_INVALID_ARG;
+  if (cfg->mlp == TTT_MLP_LINEAR) {
+    // f_W(k) = W k with W d x d (carried in W1): hidden must equal d, and the
+    // Newton-Schulz switch belongs to the SwiGLU layer
+    if (!((cfg->d == 64 || cfg->d == 256) && cfg->hidden == cfg->d) || cfg->ns_steps != 0)
+      return TTT_ERR_UNSUPPORTED_SHAPE;
+    return TTT_OK;
+  }
   const bool ok = (cfg->d == 64 && cfg->hidden == 128) || (cfg->d == 256 && cfg->hidden == 512);
   if (!ok) return TTT_ERR_UNSUPPORTED_SHAPE;
   return TTT_OK;
 }
 
+bool is_linear(const ttt_config* cfg) { return cfg->mlp == TTT_MLP_LINEAR; }
+
+// Workspace of the update of n tokens for a valid config.
+size_t update_workspace(const ttt_config* cfg, const Problem& p) {
+  if (is_linear(cfg)) return ttt::linear_workspace_bytes(p);
+  return cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_workspace_bytes(p)
+                                               : ttt::tc_workspace_bytes(p);
+}
+
 Problem make_problem(const ttt_config* cfg, int64_t n) {
   Problem p;
+  p.mlp = cfg->mlp;
   p.H = cfg->heads;
   p.d = cfg->d;
   p.hid = cfg->hidden;
@@ -63,14 +80,12 @@ const char* ttt_status_string(ttt_status s) {
 
 size_t ttt_update_workspace_bytes(const ttt_config* cfg, int64_t n_tokens) {
   if (check_cfg(cfg) != TTT_OK || n_tokens < 0 || n_tokens > kMaxTokens) return 0;
-  const Problem p = make_problem(cfg, n_tokens);
-  return cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_workspace_bytes(p)
-                                               : ttt::tc_workspace_bytes(p);
+  return update_workspace(cfg, make_problem(cfg, n_tokens));
 }
 
 size_t ttt_shadow_bytes(const ttt_config* cfg) {
   if (check_cfg(cfg) != TTT_OK) return 0;
-  return (size_t)3 * cfg->heads * cfg->d * cfg->hidden * 2;
+  return (size_t)(is_linear(cfg) ? 1 : 3) * cfg->heads * cfg->d * cfg->hidden * 2;
 }
 
 ttt_status ttt_update(const ttt_config* cfg, const float* W1, const float* W2, const float* W3,
@@ -80,17 +95,20 @@ ttt_status ttt_update(const ttt_config* cfg, const float* W1, const float* W2, c
   ttt_status s = check_cfg(cfg);
   if (s != TTT_OK) return s;
   if (n < 0 || n > kMaxTokens) return TTT_ERR_INVALID_ARG;
-  if (!W1 || !W2 || !W3 || !W1_out || !W2_out || !W3_out) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !W1_out) return TTT_ERR_INVALID_ARG;
+  if (!is_linear(cfg) && (!W2 || !W3 || !W2_out || !W3_out)) return TTT_ERR_INVALID_ARG;
   if (n > 0 && (!K || !V || !eta)) return TTT_ERR_INVALID_ARG;
   const void* ptrs[] = {W1, W2, W3, K, V, eta, W1_out, W2_out, W3_out, shadow, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   const Problem p = make_problem(cfg, n);
-  const size_t need = cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_workspace_bytes(p)
-                                                            : ttt::tc_workspace_bytes(p);
+  const size_t need = update_workspace(cfg, p);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto* sh = static_cast<__nv_bfloat16_raw*>(shadow);
+  if (is_linear(cfg))
+    return cuda_status(ttt::linear_update(p, cfg->precision == TTT_PREC_BF16_TC, W1, K, V, eta,
+                                          W1_out, sh, workspace, st));
   if (cfg->precision == TTT_PREC_FP32_CHECK)
     return cuda_status(ttt::f32_update(p, W1, W2, W3, static_cast<const float*>(K),
                                        static_cast<const float*>(V), eta, W1_out, W2_out, W3_out,
@@ -107,7 +125,7 @@ ttt_status ttt_apply(const ttt_config* cfg, const float* W1, const float* W2, co
   if (m < 0 || m > kMaxTokens) return TTT_ERR_INVALID_ARG;
   if (m > 0 && (!Q || !O)) return TTT_ERR_INVALID_ARG;
   if (cfg->precision == TTT_PREC_FP32_CHECK) {
-    if (!W1 || !W2 || !W3) return TTT_ERR_INVALID_ARG;
+    if (!W1 || (!is_linear(cfg) && (!W2 || !W3))) return TTT_ERR_INVALID_ARG;
   } else if (!shadow) {
     return TTT_ERR_INVALID_ARG;
   }
@@ -116,6 +134,9 @@ ttt_status ttt_apply(const ttt_config* cfg, const float* W1, const float* W2, co
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   const Problem p = make_problem(cfg, m);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (is_linear(cfg))
+    return cuda_status(ttt::linear_apply(p, cfg->precision == TTT_PREC_BF16_TC, W1,
+                                         static_cast<const __nv_bfloat16_raw*>(shadow), Q, O, st));
   if (cfg->precision == TTT_PREC_FP32_CHECK)
     return cuda_status(ttt::f32_apply(p, W1, W2, W3, static_cast<const float*>(Q),
                                       static_cast<float*>(O), st));
@@ -127,10 +148,11 @@ ttt_status ttt_pack_shadow(const ttt_config* cfg, const float* W1, const float* 
                            const float* W3, void* shadow, ttt_stream_t stream) {
   ttt_status s = check_cfg(cfg);
   if (s != TTT_OK) return s;
-  if (!W1 || !W2 || !W3 || !shadow) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !shadow || (!is_linear(cfg) && (!W2 || !W3))) return TTT_ERR_INVALID_ARG;
   const void* ptrs[] = {W1, W2, W3, shadow};
   for (const void* p : ptrs)
-    if (!aligned16(p)) return TTT_ERR_ALIGNMENT;
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  if (is_linear(cfg)) W2 = W3 = nullptr;
   return cuda_status(ttt::pack_shadow(cfg->heads, cfg->d, cfg->hidden, W1, W2, W3,
                                       static_cast<__nv_bfloat16_raw*>(shadow),
                                       reinterpret_cast<cudaStream_t>(stream)));
@@ -176,13 +198,14 @@ ttt_status ttt_gate(const ttt_config* cfg, const void* Wg, const void* O_prime, 
 int32_t ttt_update_splits(const ttt_config* cfg, int64_t n_tokens) {
   if (check_cfg(cfg) != TTT_OK || n_tokens < 0 || n_tokens > kMaxTokens) return 0;
   const Problem p = make_problem(cfg, n_tokens);
+  if (is_linear(cfg)) return ttt::linear_split_plan(p).S;
   return cfg->precision == TTT_PREC_FP32_CHECK ? ttt::f32_split_plan(p).S
                                                : ttt::tc_split_plan(p).S;
 }
 
 size_t ttt_partial_floats(const ttt_config* cfg) {
   if (check_cfg(cfg) != TTT_OK) return 0;
-  return (size_t)3 * cfg->heads * cfg->d * cfg->hidden;
+  return (size_t)(is_linear(cfg) ? 1 : 3) * cfg->heads * cfg->d * cfg->hidden;
 }
 
 size_t ttt_finish_workspace_bytes(const ttt_config* cfg) {
@@ -199,16 +222,19 @@ ttt_status ttt_update_partial(const ttt_config* cfg, const float* W1, const floa
   ttt_status s = check_cfg(cfg);
   if (s != TTT_OK) return s;
   if (n < 0 || n > kMaxTokens) return TTT_ERR_INVALID_ARG;
-  if (!W1 || !W2 || !W3 || !partial) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !partial || (!is_linear(cfg) && (!W2 || !W3))) return TTT_ERR_INVALID_ARG;
   if (n > 0 && (!K || !V || !eta)) return TTT_ERR_INVALID_ARG;
   const void* ptrs[] = {W1, W2, W3, K, V, eta, partial, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   const Problem p = make_problem(cfg, n);
   const bool tc = cfg->precision == TTT_PREC_BF16_TC;
-  const size_t need = tc ? ttt::tc_workspace_bytes(p) : ttt::f32_workspace_bytes(p);
+  const size_t need = update_workspace(cfg, p);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (is_linear(cfg))
+    return cuda_status(ttt::linear_update(p, tc, W1, K, V, eta, nullptr, nullptr, workspace, st,
+                                          partial));
   if (!tc)
     return cuda_status(ttt::f32_update(p, W1, W2, W3, static_cast<const float*>(K),
                                        static_cast<const float*>(V), eta, nullptr, nullptr,
@@ -224,7 +250,8 @@ ttt_status ttt_update_finish(const ttt_config* cfg, const float* W1, const float
   ttt_status s = check_cfg(cfg);
   if (s != TTT_OK) return s;
   if (ranks < 1 || ranks > 65536) return TTT_ERR_INVALID_ARG;
-  if (!W1 || !W2 || !W3 || !partials || !W1_out || !W2_out || !W3_out) return TTT_ERR_INVALID_ARG;
+  if (!W1 || !partials || !W1_out) return TTT_ERR_INVALID_ARG;
+  if (!is_linear(cfg) && (!W2 || !W3 || !W2_out || !W3_out)) return TTT_ERR_INVALID_ARG;
   const void* ptrs[] = {W1, W2, W3, partials, W1_out, W2_out, W3_out, shadow, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
@@ -251,7 +278,7 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
   if (n < 0 || n > kMaxTokens || chunk < 1) return TTT_ERR_INVALID_ARG;
   if (order != TTT_ORDER_UPDATE_THEN_APPLY && order != TTT_ORDER_APPLY_THEN_UPDATE)
     return TTT_ERR_INVALID_ARG;
-  if (!W1 || !W2 || !W3) return TTT_ERR_INVALID_ARG;
+  if (!W1 || (!is_linear(cfg) && (!W2 || !W3))) return TTT_ERR_INVALID_ARG;
   const bool tc = cfg->precision == TTT_PREC_BF16_TC;
   if (tc && !shadow) return TTT_ERR_INVALID_ARG;
   if (n == 0) return TTT_OK;
@@ -266,7 +293,7 @@ ttt_status ttt_chunked(const ttt_config* cfg, float* W1, float* W2, float* W3, v
   for (int64_t i = 0; i < nchunks; ++i) any_update |= update_mask == nullptr || update_mask[i] != 0;
   if (any_update) {
     const Problem p = make_problem(cfg, first);
-    const size_t need = tc ? ttt::tc_workspace_bytes(p) : ttt::f32_workspace_bytes(p);
+    const size_t need = update_workspace(cfg, p);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   }
   // Every chunk's pointers keep the base alignment (token rows are multiples

@@ -75,6 +75,26 @@ def test_workspace_sizes(B):
     assert B.ttt_update_splits(_cfg(B, d=100), 10) == 0
 
 
+def test_linear_mode_validation_and_sizes(B):
+    """Linear fast weights (f_W(k) = W k): hidden must equal d, no
+    Newton-Schulz; one d x d matrix per head in W1 (W2, W3 may be NULL), a
+    one-matrix shadow and partial; an unknown form is an invalid argument."""
+    lin = _cfg(B, hidden=256, mlp=B.MLP_LINEAR)
+    assert B.ttt_shadow_bytes(lin) == 4 * 256 * 256 * 2
+    assert B.ttt_partial_floats(lin) == 4 * 256 * 256
+    assert B.ttt_update_workspace_bytes(lin, 1000) >= B.ttt_update_splits(lin, 1000) * 4 * 256 * 256 * 4
+    assert B.ttt_update_workspace_bytes(_cfg(B, mlp=B.MLP_LINEAR), 10) == 0       # hidden != d
+    assert B.ttt_update_workspace_bytes(_cfg(B, d=64, hidden=64, mlp=B.MLP_LINEAR), 10) > 0
+    assert _update(B, _cfg(B, mlp=B.MLP_LINEAR)) == B.TTT_ERR_UNSUPPORTED_SHAPE
+    assert _update(B, _cfg(B, hidden=256, mlp=B.MLP_LINEAR, ns_steps=2)) == B.TTT_ERR_UNSUPPORTED_SHAPE
+    assert _update(B, _cfg(B, mlp=2)) == B.TTT_ERR_INVALID_ARG
+    # W2, W3 and their outputs are not needed in linear mode: validation runs
+    # on to the workspace check
+    assert _update(B, lin, W2=None, W3=None, W2o=None, W3o=None, ws_bytes=100) == B.TTT_ERR_WORKSPACE
+    assert _update(B, lin, W1=None) == B.TTT_ERR_INVALID_ARG
+    assert _update(B, _cfg(B), W2=None) == B.TTT_ERR_INVALID_ARG                  # SwiGLU needs W2
+
+
 def test_split_plan(B):
     """The gradient slots of the update: sets of (hidden / 128) 3-CTA clusters,
     as many as one wave holds (45 clusters resident on a B200: 11 sets for
