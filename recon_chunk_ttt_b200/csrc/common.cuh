@@ -312,6 +312,30 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream serialization attribute may start before the kernel ahead of it in
+// the stream has finished; grid_dep_wait() returns once that kernel has
+// completed and its memory operations are visible, and must come before any
+// read of its results (or of anything the host or earlier work wrote).
+// grid_dep_launch() lets the next kernel start once every CTA of this grid has
+// issued it (or exited); it is issued after this CTA holds its resources
+// (shared memory, TMEM), so the next kernel's CTAs can only take what is left.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Loads from a shared::cluster address (this or another CTA of the cluster).
+// Not ordered against other memory operations by the compiler: callers put
+// them between cluster barriers.
+__device__ __forceinline__ void ld_shared_cluster_v4(uint32_t caddr, float* x) {
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3])
+               : "r"(caddr));
+}
+__device__ __forceinline__ void ld_shared_cluster_v2(uint32_t caddr, float* x) {
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(x[0]), "=f"(x[1]) : "r"(caddr));
+}
 // Every thread of every CTA of the cluster; memory operations before it
 // (including ones on other CTAs' shared memory) are performed before any
 // thread of the cluster passes it.

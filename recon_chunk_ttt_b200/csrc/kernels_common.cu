@@ -147,6 +147,8 @@ __global__ void __launch_bounds__(256, 2) reduce_renorm_kernel(
     const float* __restrict__ partials, int S, int H, int d, int hid, int nblk, int mode,
     const float* W1, const float* W2, const float* W3, float* W1o, float* W2o, float* W3o,
     __nv_bfloat16_raw* __restrict__ shadow, double* __restrict__ scratch) {
+  grid_dep_launch();
+  grid_dep_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int per = nblk == 3 ? 2 * hid + d : d;
@@ -269,9 +271,21 @@ cudaError_t reduce_renorm(const Problem& p, int S, const float* partials, const 
   const int rows = p.H * (nblk == 3 ? 2 * p.hid + p.d : p.d);
   const int blocks = (rows * 32 + 255) / 256;
   TraceScope ts("reduce_renorm", st);
-  reduce_renorm_kernel<<<blocks, 256, 0, st>>>(partials, S, p.H, p.d, p.hid, nblk, p.renorm, W1,
-                                              W2, W3, W1o, W2o, W3o, shadow,
-                                              reinterpret_cast<double*>(scratch));
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, reduce_renorm_kernel, partials, S, p.H, p.d,
+                                             p.hid, nblk, (int)p.renorm, W1, W2, W3, W1o, W2o,
+                                             W3o, shadow, reinterpret_cast<double*>(scratch));
+    if (e != cudaSuccess) return e;
+  }
   if (p.renorm == 2)
     frob_scale_kernel<<<p.H * nblk, 256, 0, st>>>(p.H, p.d, p.hid, nblk,
                                                  reinterpret_cast<double*>(scratch), W1o, W2o,

@@ -283,6 +283,8 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();
+  grid_dep_wait();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ forward ring
@@ -706,25 +708,38 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
       // its group has no piece for
       const int slots = S_.last ? S - S_.p : 1;
       if (isF) {
-        // lanes 0..63: G1 rows, 64..127: G3 rows of this CTA's 64 hidden units
+        // lanes 0..63: G1 rows, 64..127: G3 rows of this CTA's 64 hidden units.
+        // Each warp's 32 rows x 16 columns pass through its own 2 KB of the
+        // gradient operand buffer (idle once the gradient is complete), so
+        // that a store instruction writes 64 contiguous bytes of 8 rows
+        // rather than 16 bytes of 32 rows.
         const int blk = q < 2 ? 0 : 1;
-        const int hrow = S_.grp * L::GH + rank * L::FH + (q & 1) * 32 + lane;
-        TTT_DCHECK(hrow < hid && S_.p + slots <= S, err, kErrCheckIndex);
+        const int hrow0 = S_.grp * L::GH + rank * L::FH + (q & 1) * 32;
+        TTT_DCHECK(hrow0 + 32 <= hid && S_.p + slots <= S, err, kErrCheckIndex);
+        uint8_t* stg = ga + (warp - 3) * 2048;  // [32 rows][4 chunks of 16 B]
         for (int c0 = h * (D / 4); c0 < (h + 1) * (D / 4); c0 += 16) {
           uint32_t rr[16];
           tmem_ld_16x(tmem + lane_base + L::TM_G + c0, rr);
           tmem_ld_wait();
-          for (int z = 0; z < slots; ++z) {
-            float* P = partials + (((size_t)(S_.p + z) * H + S_.head) * 3 + blk) * mat +
-                       (size_t)hrow * D + c0;
-            float4* dst = reinterpret_cast<float4*>(P);
+          // row `lane`: chunk j at position j ^ ((lane >> 1) & 3)
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = z == 0 ? make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
-                                            __uint_as_float(rr[4 * v + 2]),
-                                            __uint_as_float(rr[4 * v + 3]))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) * 16)) =
+                make_uint4(rr[4 * j], rr[4 * j + 1], rr[4 * j + 2], rr[4 * j + 3]);
+          __syncwarp();
+          const int j = lane & 3;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = k * 8 + (lane >> 2);
+            const uint4 v =
+                *reinterpret_cast<const uint4*>(stg + r * 64 + ((j ^ ((r >> 1) & 3)) * 16));
+            for (int z = 0; z < slots; ++z) {
+              float* P = partials + (((size_t)(S_.p + z) * H + S_.head) * 3 + blk) * mat +
+                         (size_t)(hrow0 + r) * D + c0 + 4 * j;
+              *reinterpret_cast<uint4*>(P) = z == 0 ? v : make_uint4(0u, 0u, 0u, 0u);
+            }
           }
+          __syncwarp();
         }
       } else {
         // P2 rows = hidden units of the group, stored transposed as [d][hid]
@@ -789,13 +804,15 @@ cudaError_t fused_update_impl(const Problem& p, const float* W1, const float* W2
   cfg.blockDim = dim3(L::THREADS);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 3;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   TraceScope ts("tc_update_fused", st);
   return cudaLaunchKernelEx(&cfg, fused_update_kernel<D>, mK, mV, mKg, mVg, W1, W2, W3, eta,
                             p.n, p.H, p.hid, NS, SPH, S, partials, err);

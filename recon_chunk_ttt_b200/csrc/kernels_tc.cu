@@ -65,8 +65,14 @@ struct AP {
   static constexpr uint32_t TM_Q = 128;                  // the q tile (A of F) in TMEM
 };
 
-// Persistent: CTA b takes (query tile, head) items b, b + grid, ...  Per item
-// and 64-wide hidden slice js: F(js) = Q [W1s; W3s]^T into TMEM buffer js&1,
+// Persistent: CTA b takes (query tile, head) items b, b + grid, ...  With
+// P > 1 (few items: the launch is one cluster of P CTAs per item) the CTA of
+// cluster rank r takes the hidden slices [r nsl / P, (r + 1) nsl / P) of item
+// blockIdx.x / P and writes its partial O (fp32) to its own shared memory;
+// after a cluster barrier the CTA of rank o sums rows [o 128 / P,
+// (o + 1) 128 / P) of the P partials in rank order (distributed shared
+// memory loads) into O.  Per
+// item and 64-wide hidden slice js: F(js) = Q [W1s; W3s]^T into TMEM buffer js&1,
 // the epilogue turns it into u = SiLU(h1) ⊙ h3 (bf16, shared memory), and
 // O += u W2s^T.  The q chunks are released one by one during the
 // last slice so the next item's q streams in early; O is drained while the
@@ -76,7 +82,7 @@ template <int D>
 __global__ void __launch_bounds__(AP<D>::THREADS, 1)
     apply_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mW13,
                  const __grid_constant__ CUtensorMap mW2,
-                 int64_t m, int H, int hid, __nv_bfloat16* __restrict__ O, int* err) {
+                 int64_t m, int H, int hid, int P, __nv_bfloat16* __restrict__ O, int* err) {
   using L = AP<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -99,6 +105,11 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
   const int w13_stages = L::NCH / L::CH_PER_STAGE;
   const int64_t nqt = (m + BM - 1) / BM;
   const int64_t items = nqt * H;
+  // this CTA's items (first, first + stride, ...) and hidden slices [js0, js0 + ns)
+  const int part = (int)(blockIdx.x % (unsigned)P);
+  const int64_t first = blockIdx.x / P, stride = gridDim.x / P;
+  const int js0 = part * nsl / P;
+  const int ns = (part + 1) * nsl / P - js0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NSTAGE; ++i) {
@@ -129,6 +140,8 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();
+  grid_dep_wait();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -145,7 +158,7 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       ++issued;
       if (++stage == L::NSTAGE) { stage = 0; phase ^= 1; }
     };
-    for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
+    for (int64_t it = first, i = 0; it < items && ok; it += stride, ++i) {
       const int64_t qt = it / H;
       const int head = (int)(it % H);
       for (int c = 0; c < L::NCH && ok; ++c) {
@@ -179,11 +192,11 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
         tma_load_2d(st, &mW2, &full[stage], js * HS, head * D);
         advance();
       };
-      for (int js = 0; js < nsl && ok; ++js) {
-        load_w13(js);
-        if (js >= 2 && ok) load_w2(js - 2);
+      for (int js = 0; js < ns && ok; ++js) {
+        load_w13(js0 + js);
+        if (js >= 2 && ok) load_w2(js0 + js - 2);
       }
-      for (int j = nsl >= 2 ? nsl - 2 : 0; j < nsl && ok; ++j) load_w2(j);
+      for (int j = ns >= 2 ? ns - 2 : 0; j < ns && ok; ++j) load_w2(js0 + j);
     }
     drain_ring(full, L::NSTAGE, issued, err);
     for (int c = 0; c < L::NCH; ++c) drain_ring(&q_full[c], 1, qloads, err);
@@ -224,9 +237,9 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       umma_commit(&u_empty[b]);
       return true;
     };
-    for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
-      for (int js = 0; js < nsl && ok; ++js) {
-        const int64_t g = i * nsl + js;
+    for (int64_t it = first, i = 0; it < items && ok; it += stride, ++i) {
+      for (int js = 0; js < ns && ok; ++js) {
+        const int64_t g = i * ns + js;
         // one F buffer: wait until the epilogue has drained F(g - 1) (which
         // also means every earlier F MMA, and so every read of the q tile in
         // TMEM, has completed)
@@ -274,8 +287,8 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       }
       if (!ok) break;
       bool tail_ok = true;
-      for (int j = nsl >= 2 ? nsl - 2 : 0; j < nsl && tail_ok; ++j)
-        tail_ok = do_o(i * nsl + j, j, i);
+      for (int j = ns >= 2 ? ns - 2 : 0; j < ns && tail_ok; ++j)
+        tail_ok = do_o(i * ns + j, j, i);
       if (!tail_ok) break;
       umma_commit(o_full);
     }
@@ -288,12 +301,12 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
     const int ch = (warp - 2) / 4;  // hidden columns [32ch, 32ch+32) of a slice
     const int row = q * 32 + lane;
     bool ok = true;
-    for (int64_t it = blockIdx.x, i = 0; it < items && ok; it += gridDim.x, ++i) {
+    for (int64_t it = first, i = 0; it < items && ok; it += stride, ++i) {
       const int64_t qt = it / H;
       const int head = (int)(it % H);
       const int64_t qi = qt * BM + row;
-      for (int js = 0; js < nsl && ok; ++js) {
-        const int64_t g = i * nsl + js;
+      for (int js = 0; js < ns && ok; ++js) {
+        const int64_t g = i * ns + js;
         const int b = (int)(g & 1);
         const uint32_t par = (uint32_t)((g >> 1) & 1);
         const bool got = mbar_wait(&f_full[0], (uint32_t)(g & 1), abort_flag, err, kErrWaitAcc);
@@ -335,6 +348,7 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
       const bool got_o = mbar_wait(o_full, (uint32_t)(i & 1), abort_flag, err, kErrWaitAcc);
       __syncwarp();
       if (!got_o) break;
+      if (P > 1) break;  // one item; its partial O leaves after the loop
       tc_fence_after();
       const uint32_t to = tmem + ((uint32_t)(q * 32) << 16) + 256;
       for (int c0 = ch * (D / 2); c0 < (ch + 1) * (D / 2); c0 += 32) {
@@ -360,6 +374,81 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (P > 1) {
+    // Every CTA of the cluster is past its last MMA (its epilogue saw
+    // o_full): its q and operand buffers are idle.  The partial O goes to
+    // this CTA's own buffers, row r at r * D * 4 bytes, fp32, 16-byte chunk c
+    // of the row at (c & ~7) | ((c ^ r) & 7).
+    tc_fence_after();
+    if (warp >= 2) {
+      const int q = warp & 3, ch = (warp - 2) / 4, row = q * 32 + lane;
+      uint8_t* prow = smem + L::OFF_Q + (size_t)row * D * 4;
+      const uint32_t to = tmem + ((uint32_t)(q * 32) << 16) + 256;
+      for (int c0 = ch * (D / 2); c0 < (ch + 1) * (D / 2); c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld_32x32(to + c0, rr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          *reinterpret_cast<uint4*>(prow + ((c0 / 4) + (v ^ (row & 7))) * 16) =
+              make_uint4(rr[4 * v], rr[4 * v + 1], rr[4 * v + 2], rr[4 * v + 3]);
+      }
+    }
+    tc_fence_before();
+    // every partial of the cluster is written
+    cluster_sync_all();
+    const int64_t qt = first / H;
+    const int head = (int)(first % H);
+    const int r0 = part * BM / P, nr = (part + 1) * BM / P - r0;
+    constexpr int VPL = D / 32;  // floats of a row per lane (8 or 2)
+    const int nw = (int)(blockDim.x / 32);
+    const uint32_t local = smem_u32(smem + L::OFF_Q);
+    for (int lr = warp; lr < nr; lr += nw) {
+      const int r = r0 + lr;
+      const int64_t qi = qt * BM + r;
+      if (qi >= m) break;
+      // all P loads of the row in flight before the sum
+      float x[8][VPL];
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        if (p < P) {
+          const uint32_t base = mapa_shared(local, (uint32_t)p) + (uint32_t)r * D * 4;
+          if constexpr (VPL == 8) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int c = 2 * lane + k;
+              ld_shared_cluster_v4(base + (uint32_t)(((c & ~7) | ((c ^ r) & 7)) * 16),
+                                   &x[p][4 * k]);
+            }
+          } else {
+            const int c = lane >> 1;
+            ld_shared_cluster_v2(
+                base + (uint32_t)(((c & ~7) | ((c ^ r) & 7)) * 16 + (lane & 1) * 8), x[p]);
+          }
+        }
+      }
+      // rank order
+      float acc[VPL];
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) acc[e] = x[0][e];
+#pragma unroll
+      for (int p = 1; p < 8; ++p)
+        if (p < P)
+#pragma unroll
+          for (int e = 0; e < VPL; ++e) acc[e] += x[p][e];
+      TTT_DCHECK(head < H && lane * VPL + VPL <= D, err, kErrCheckIndex);
+      __nv_bfloat16* dst = O + qi * (int64_t)H * D + (int64_t)head * D + lane * VPL;
+      if constexpr (VPL == 8) {
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0], acc[1]);
+      }
+    }
+    // no CTA leaves while another may still read its shared memory
+    cluster_sync_all();
+  }
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
@@ -410,6 +499,43 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
                         W2, W3, W1o, W2o, W3o, shadow, w.scratch, st);
 }
 
+// Clusters of P apply CTAs that fit on the GPU at once (queried once per P).
+template <int D>
+int apply_clusters_per_wave(int P) {
+  static int cache[9] = {};
+  if (cache[P] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P);
+    cfg.blockDim = dim3(AP<D>::THREADS);
+    cfg.dynamicSmemBytes = AP<D>::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, apply_kernel<D>, &cfg) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      n = -1;
+    }
+    cache[P] = n;
+  }
+  return cache[P];
+}
+
+// Hidden-slice parts per (query tile, head): 1 (persistent CTAs) unless the
+// items fill at most half a wave; then 2, if all the clusters fit on the GPU
+// at once.  Measured at 1,374 queries x 4 heads (d 256): 16.8 us with one
+// part, 15.1 with two, 15.9 with three (the partial sums cross the cluster
+// at about 20 GB/s per SM, which eats the gain of shorter slice chains).
+template <int D>
+int apply_parts(int64_t items, int nsl) {
+  if (nsl >= 2 && 2 * items <= num_sms() && items <= apply_clusters_per_wave<D>(2)) return 2;
+  return 1;
+}
+
 template <int D>
 cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, const void* Q,
                           void* O, cudaStream_t st) {
@@ -443,14 +569,25 @@ cudaError_t tc_apply_impl(const Problem& p, const __nv_bfloat16_raw* shadow, con
   cudaError_t e = ensure_smem_attr(apply_kernel<D>, AP<D>::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t items = (p.n + BM - 1) / BM * p.H;
+  const int P = apply_parts<D>(items, p.hid / HS);
   const int sms = num_sms();
-  const unsigned grid = (unsigned)(items < sms ? items : sms);
-  {
-    TraceScope ts("tc_apply", st);
-    apply_kernel<D><<<grid, AP<D>::THREADS, AP<D>::SMEM, st>>>(
-        mQ, mW13, mW2, p.n, p.H, p.hid, static_cast<__nv_bfloat16*>(O), err);
-  }
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P > 1 ? (unsigned)(items * P) : (unsigned)(items < sms ? items : sms));
+  cfg.blockDim = dim3(AP<D>::THREADS);
+  cfg.dynamicSmemBytes = AP<D>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)P;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = P > 1 ? 2 : 1;
+  TraceScope ts("tc_apply", st);
+  return cudaLaunchKernelEx(&cfg, apply_kernel<D>, mQ, mW13, mW2, p.n, p.H, p.hid, P,
+                            static_cast<__nv_bfloat16*>(O), err);
 }
 
 }  // namespace

@@ -10,7 +10,7 @@ import oracle as O
 from recon_chunk_ttt_b200 import workloads as wl
 
 from helpers import (TOL_F32, TOL_TC, as_output_type, gpu_inputs, oracle_update_apply,
-                     rel_errors, run_update_apply, to_dev)
+                     rel_errors, rel_fro_heads, run_update_apply, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -301,3 +301,26 @@ def test_bounded_wait_runs_out_and_reports():
     ref = oracle_update_apply(x, R.PREC_BF16_TC, R.RENORM_ROW)
     assert max(rel_errors(gpu, ref, x)) <= TOL_TC
     assert R.ttt_check_device_error() == 0
+
+
+@pytest.mark.parametrize("m,H,d,hid", [(1, 4, 256, 512), (700, 4, 256, 512), (1374, 4, 256, 512),
+                                       (2600, 4, 256, 512), (300, 2, 64, 128), (5000, 1, 64, 128)])
+def test_apply_hidden_parts_vs_oracle(m, H, d, hid):
+    """The apply alone, at query counts whose (tile, head) items fill less
+    than a wave (one cluster per item, the hidden slices split over its CTAs,
+    partial outputs summed in rank order) and more (persistent CTAs): against
+    the oracle's apply of the bf16 weights, per head, and bitwise equal on a
+    second run."""
+    x = wl.random_layer(300 + m, m, H, d, hid)
+    cfg = R.make_config(H, d, hid)
+    Wd = [to_dev(a, torch.float32) for a in (x.W1, x.W2, x.W3)]
+    shadow = R.ttt_pack_shadow(cfg, *Wd)
+    Qd = to_dev(x.Q, torch.bfloat16)
+    O1 = R.ttt_apply(cfg, Qd, shadow=shadow)
+    O2 = R.ttt_apply(cfg, Qd, shadow=shadow)
+    R.ttt_check_device_error()
+    assert torch.equal(O1, O2)
+    Wb = [wl.bf16_round(a) for a in (x.W1, x.W2, x.W3)]
+    ref = O.ttt_apply(*Wb, wl.bf16_round(x.Q))
+    got = O1.float().cpu().double().numpy()
+    assert rel_fro_heads(got, ref, H, token_major=True) <= TOL_TC
