@@ -17,8 +17,11 @@
 //     DU   = V W2s^T                   M = 128 tokens, N = 128, into TMEM (2 buffers)
 //     epilogue: du (bf16) to ranks 0 and 1
 //     P2  += (η·u)^T V                 M = 128 hidden, N = d, in TMEM
-// The gradient MMAs of tile i run after the forward MMAs of tile i+1, so the
-// epilogues and exchanges of a tile overlap the next tile's MMAs.  At the end
+// The forward and the gradient MMAs have an issuing thread each, so the
+// wait of one for its operands (the forward tile, or the epilogue's η-scaled
+// block and the gradient ring) does not hold up the other; the forward MMAs
+// run ahead, and a tile's epilogue and exchanges overlap the next tile's
+// forward MMAs.  At the end
 // each CTA writes its slice of the split's fp32 partial ([S][H][3][hid*d],
 // blocks G1, G3, P2 as [d][hid]); a fixed-order reduction over the splits
 // follows in another kernel, so results are bitwise reproducible.
@@ -75,9 +78,11 @@ struct FU {
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static constexpr int EPI_WARPS = 16;          // four per TMEM lane quadrant
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
-  // kf producer, MMA, kg producer, epilogue warps, then one signalling warp
-  static constexpr int THREADS = 96 + EPI_THREADS + 32;
+  // kf producer, forward MMA issuer, kg producer, epilogue warps, one
+  // signalling warp, gradient MMA issuer
+  static constexpr int THREADS = 96 + EPI_THREADS + 64;
   static constexpr int SIGNAL_WARP = 3 + EPI_WARPS;
+  static constexpr int GMMA_WARP = SIGNAL_WARP + 1;   // gradient MMA issuer
   static constexpr uint32_t TMEM_COLS = 512;    // forward buffers at 0 and 128, gradient at 256
   static constexpr uint32_t TM_G = 256;
 };
@@ -104,6 +109,7 @@ struct Bars {
   __device__ uint64_t* du_empty(int f) { return x(11 + f); }  // D: rank f read its du
   __device__ uint64_t* du_read() { return x(13); }    // F: every epilogue warp read du
   __device__ uint64_t* g_empty() { return x(14); }    // gradient accumulator drained
+  __device__ uint64_t* done_g() { return x(15); }
 };
 
 // Give up: device error word, and the abort flag of every CTA of the cluster.
@@ -257,6 +263,7 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     mbar_init(bar.g_full(), 1);
     mbar_init(bar.g_empty(), 1);
     mbar_init(bar.done(), 1);
+    mbar_init(bar.done_g(), 1);
     mbar_init(bar.au_empty(), 1);
     mbar_init(bar.du_full(), 1);
     mbar_init(bar.du_empty(0), 1);
@@ -344,100 +351,117 @@ __global__ void __launch_bounds__(FU<D>::THREADS, 1)
     }
     drain_ring(bar.kg_full(0), L::NKG, issued, err);
   } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------ MMA issuer
+    // ------------------------------------------------ forward MMA issuer
     // F: B = [W1s; W3s] rows, K-major; D: B = W2 columns of the group,
     // MN-major (two blocks of 64 hidden units x d rows)
     const uint32_t idF = idesc_bf16_f32(BM, 128, false, !isF);
-    const uint32_t idG = idesc_bf16_f32(BM, D, true, true);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t ga = sbase + L::OFF_GA;
-    int fs = 0, gs = 0;
-    uint32_t fph = 0, gph = 0;
+    int fs = 0;
+    uint32_t fph = 0;
     bool ok = true;
     for (int sg = 0; sg < nseg && ok; ++sg) {
       const Seg S_ = seg(sg);
-      // this segment's weights are staged; the previous gradient is drained
-      if (!cwait<false>(bar.w_full(), (uint32_t)(sg & 1), abort_flag, err, kErrWaitFull) ||
-          (sg >= 1 && !cwait<false>(bar.g_empty(), (uint32_t)((sg - 1) & 1), abort_flag, err,
-                                    kErrWaitAccFree))) {
+      // this segment's weights are staged
+      if (!cwait<false>(bar.w_full(), (uint32_t)(sg & 1), abort_flag, err, kErrWaitFull)) {
         ok = false;
         break;
       }
-      // Per tile i: the forward MMAs of tile i, then the gradient MMAs of
-      // tile i - 1 (whose operand the epilogue has been forming meanwhile).
-      for (int i = 0; i <= S_.nts && ok; ++i) {
-        if (i < S_.nts) {
-          const int gi = S_.base + i;
-          const int b = gi & 1;
-          if (!cwait<false>(bar.acc_empty(b), ((gi >> 1) & 1) ^ 1, abort_flag, err,
-                            kErrWaitAccFree)) {
+      for (int i = 0; i < S_.nts && ok; ++i) {
+        const int gi = S_.base + i;
+        const int b = gi & 1;
+        if (!cwait<false>(bar.acc_empty(b), ((gi >> 1) & 1) ^ 1, abort_flag, err,
+                          kErrWaitAccFree)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dF = tmem + b * 128;
+        for (int c0 = 0; c0 < L::NCH && ok; c0 += L::CPS) {
+          if (!cwait<false>(bar.kf_full(fs), fph, abort_flag, err, kErrWaitFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t dF = tmem + b * 128;
-          for (int c0 = 0; c0 < L::NCH && ok; c0 += L::CPS) {
-            if (!cwait<false>(bar.kf_full(fs), fph, abort_flag, err, kErrWaitFull)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            for (int cc = 0; cc < L::CPS; ++cc) {
-              const int c = c0 + cc;
-              const uint32_t a = sbase + L::OFF_KF + fs * L::KF_STAGE + cc * L::CHUNK;
+          for (int cc = 0; cc < L::CPS; ++cc) {
+            const int c = c0 + cc;
+            const uint32_t a = sbase + L::OFF_KF + fs * L::KF_STAGE + cc * L::CHUNK;
 #pragma unroll
-              for (int kk = 0; kk < CH / 16; ++kk) {
-                const uint64_t db =
-                    isF ? sdesc_sw128(sbase + L::OFF_W + c * L::CHUNK + kk * KSTEP_BYTES, 16, 1024)
-                        : sdesc_sw128(sbase + L::OFF_W + (c * CH + kk * 16) * 128, L::W2BLK, 1024);
-                umma_bf16(dF, sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024), db, idF,
-                          (c | kk) != 0);
-              }
+            for (int kk = 0; kk < CH / 16; ++kk) {
+              const uint64_t db =
+                  isF ? sdesc_sw128(sbase + L::OFF_W + c * L::CHUNK + kk * KSTEP_BYTES, 16, 1024)
+                      : sdesc_sw128(sbase + L::OFF_W + (c * CH + kk * 16) * 128, L::W2BLK, 1024);
+              umma_bf16(dF, sdesc_sw128(a + kk * KSTEP_BYTES, 16, 1024), db, idF,
+                        (c | kk) != 0);
             }
-            umma_commit(bar.kf_empty(fs));
-            if (++fs == L::NKF) { fs = 0; fph ^= 1; }
           }
-          if (!ok) break;
-          umma_commit(bar.acc_full(b));
+          umma_commit(bar.kf_empty(fs));
+          if (++fs == L::NKF) { fs = 0; fph ^= 1; }
         }
-        if (i >= 1) {
-          const int j = S_.base + i - 1;
-          const bool got =
-              isF ? cwait<false>(bar.ga_full(), (uint32_t)(j & 1), abort_flag, err, kErrWaitOperand)
-                  : cwait<true>(bar.ga_full(), (uint32_t)(j & 1), abort_flag, err, kErrWaitOperand);
-          if (!got) { ok = false; break; }
-          if (!isF && j + 1 < NT) mbar_arrive_expect_tx(bar.ga_full(), 2 * L::XB);
-          tc_fence_after();
-          for (int st = 0; st < BM / L::TKG && ok; ++st) {
-            if (!cwait<false>(bar.kg_full(gs), gph, abort_flag, err, kErrWaitFull)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t kg = sbase + L::OFF_KG + gs * L::KG_STAGE;
-#pragma unroll
-            for (int kk = 0; kk < L::TKG / 16; ++kk) {
-              // A: MN-major, 2 blocks of 64 rows (LBO), 16 tokens per K step;
-              // B: MN-major, NCH blocks of 64 d (LBO = TKG rows x 128 B)
-              const uint64_t da = sdesc_sw128(ga + (st * L::TKG + kk * 16) * 128, L::XB, 1024);
-              const uint64_t db = sdesc_sw128(kg + kk * 16 * 128, L::TKG * 128, 1024);
-              umma_bf16(tmem + L::TM_G, da, db, idG, ((i - 1) | st | kk) != 0);
-            }
-            umma_commit(bar.kg_empty(gs));
-            if (++gs == L::NKG) { gs = 0; gph ^= 1; }
-          }
-          if (!ok) break;
-          if (isF)
-            umma_commit(bar.ga_empty());
-          else
-            umma_commit_cluster(bar.au_empty(), (uint16_t)0x3);  // ranks 0 and 1 may refill
-        }
+        if (!ok) break;
+        umma_commit(bar.acc_full(b));
       }
-      if (ok) umma_commit(bar.g_full());
     }
     umma_commit(bar.done());
     volatile int never = 0;
     mbar_wait(bar.done(), 0, &never, err, kErrWaitFinal);
+  } else if (warp == L::GMMA_WARP) {
+    // ------------------------------------------------ gradient MMA issuer
+    // (lane 0; the other lanes of the warp have no role)
+   if (lane == 0) {
+    // Its own thread, so that its operand waits (the epilogue's η-scaled
+    // block, the gradient ring) overlap the forward issuer's.
+    const uint32_t idG = idesc_bf16_f32(BM, D, true, true);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t ga = sbase + L::OFF_GA;
+    int gs = 0;
+    uint32_t gph = 0;
+    bool ok = true;
+    for (int sg = 0; sg < nseg && ok; ++sg) {
+      const Seg S_ = seg(sg);
+      // the previous segment's gradient is drained
+      if (sg >= 1 && !cwait<false>(bar.g_empty(), (uint32_t)((sg - 1) & 1), abort_flag, err,
+                                   kErrWaitAccFree)) {
+        ok = false;
+        break;
+      }
+      for (int i = 0; i < S_.nts && ok; ++i) {
+        const int j = S_.base + i;
+        const bool got =
+            isF ? cwait<false>(bar.ga_full(), (uint32_t)(j & 1), abort_flag, err, kErrWaitOperand)
+                : cwait<true>(bar.ga_full(), (uint32_t)(j & 1), abort_flag, err, kErrWaitOperand);
+        if (!got) { ok = false; break; }
+        if (!isF && j + 1 < NT) mbar_arrive_expect_tx(bar.ga_full(), 2 * L::XB);
+        tc_fence_after();
+        for (int st = 0; st < BM / L::TKG && ok; ++st) {
+          if (!cwait<false>(bar.kg_full(gs), gph, abort_flag, err, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kg = sbase + L::OFF_KG + gs * L::KG_STAGE;
+#pragma unroll
+          for (int kk = 0; kk < L::TKG / 16; ++kk) {
+            // A: MN-major, 2 blocks of 64 rows (LBO), 16 tokens per K step;
+            // B: MN-major, NCH blocks of 64 d (LBO = TKG rows x 128 B)
+            const uint64_t da = sdesc_sw128(ga + (st * L::TKG + kk * 16) * 128, L::XB, 1024);
+            const uint64_t db = sdesc_sw128(kg + kk * 16 * 128, L::TKG * 128, 1024);
+            umma_bf16(tmem + L::TM_G, da, db, idG, (i | st | kk) != 0);
+          }
+          umma_commit(bar.kg_empty(gs));
+          if (++gs == L::NKG) { gs = 0; gph ^= 1; }
+        }
+        if (!ok) break;
+        if (isF)
+          umma_commit(bar.ga_empty());
+        else
+          umma_commit_cluster(bar.au_empty(), (uint16_t)0x3);  // ranks 0 and 1 may refill
+      }
+      if (ok) umma_commit(bar.g_full());
+    }
+    umma_commit(bar.done_g());
+    volatile int never = 0;
+    mbar_wait(bar.done_g(), 0, &never, err, kErrWaitFinal);
+   }
   } else if (warp == L::SIGNAL_WARP) {
     // ------------------------------------------------ F: du consumed -> rank 2
     // A remote arrive with cluster-scope release costs about a microsecond on
