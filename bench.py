@@ -538,9 +538,16 @@ def shard_probe(R, torch, dev, cfg, K, V, eta, Win, Wout, shadow, ws, stream, T,
     e1.record(stream)
     torch.cuda.synchronize(dev)
     R.ttt_check_device_error()
-    ms = rank_max(e0.elapsed_time(e1) / reps)
-    return {"ranks": world, "tokens_per_rank": b - a, "tokens": T, "ms_per_layer_update": ms,
-            "update_tokens_per_s_one_scene": T / (ms / 1e3),
+    return shard_fields(world, b - a, T, rank_max(e0.elapsed_time(e1) / reps))
+
+
+def shard_fields(world: int, tokens_per_rank: int, T: int, ms: float) -> dict:
+    """The token-sharded update's line: ms is already the max over ranks; the
+    throughput is the one scene's T tokens over that time (strong scaling:
+    the scene is fixed, the ranks share it)."""
+    return {"ranks": world, "tokens_per_rank": tokens_per_rank, "tokens": T,
+            "ms_per_layer_update": ms, "update_tokens_per_s_one_scene": T / (ms / 1e3),
+            "scaling": "strong",
             "exchange": "NCCL all-gather of one fp32 partial per rank" if world > 1 else "none"}
 
 

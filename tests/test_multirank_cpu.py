@@ -2,7 +2,9 @@
 
 Each rank runs its own scene (weak scaling, no data-path collective); the step
 time is the max over ranks and the whole-job value sums the ranks' tokens.  The
-reference arm runs on rank 0 only.
+token-sharded update's field (one scene split over the ranks) takes the
+slowest rank's time and counts the scene's tokens once.  The reference arm
+runs on rank 0 only.
 """
 import json
 import os
@@ -35,8 +37,15 @@ def _worker(rank, world, port, out_dir):
         ms_local = [10.0, 12.5][rank]
         ms = bench.max_over_ranks(ms_local, w, torch.device("cpu"))
         value = bench.aggregate_value(w, 961800, 24, ms)
+        # the token-sharded update of one scene: each rank times its own
+        # partial + exchange + finish; the line takes the slowest rank
+        from recon_chunk_ttt_b200.sharded import shard_range
+        a, b = shard_range(961800, r, w)
+        sh = bench.shard_fields(w, b - a, 961800,
+                                bench.max_over_ranks([4.0, 4.5][rank], w, torch.device("cpu")))
         with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
-            json.dump({"world": w, "rank": r, "local": local, "ms": ms, "value": value}, f)
+            json.dump({"world": w, "rank": r, "local": local, "ms": ms, "value": value,
+                       "shard": sh}, f)
     finally:
         dist.destroy_process_group()
 
@@ -51,6 +60,11 @@ def test_two_gloo_ranks_take_max_time_and_sum_tokens(tmp_path):
         assert d["world"] == 2 and d["rank"] == r and d["local"] == r
         assert d["ms"] == 12.5
         assert d["value"] == pytest.approx(2 * 961800 * 24 / 0.0125)
+        sh = d["shard"]
+        assert sh["ranks"] == 2 and sh["tokens"] == 961800 and sh["scaling"] == "strong"
+        assert sh["tokens_per_rank"] == 480900
+        assert sh["ms_per_layer_update"] == 4.5
+        assert sh["update_tokens_per_s_one_scene"] == pytest.approx(961800 / 0.0045)
 
 
 def test_reference_arm_runs_on_rank0_only():
