@@ -50,14 +50,16 @@ struct FU {
   static constexpr int NCH = D / CH;            // 64-wide d chunks
   static constexpr int GH = 128;                // hidden units per cluster
   static constexpr int FH = 64;                 // hidden units per F CTA
-  // Ring shapes (measured at scene700 size): the forward ring holds one whole
-  // k (or v) tile in one 64 KB TMA box, the gradient ring two 16 KB stages.
-  // A thread's TMA boxes complete one after another, so fewer, larger boxes
-  // deliver more bytes per unit of time.
+  // Ring shapes (measured at scene700 size, with separate forward and
+  // gradient issuers): the forward ring holds one k (or v) tile as two 32 KB
+  // boxes (half of d each), so the next tile's first half loads while this
+  // tile's second half is multiplied (2.5 % faster than one 64 KB box, 3-4 %
+  // faster than four 16 KB boxes); the gradient ring two 16 KB stages (one
+  // 32 KB or four 8 KB stages: 3-4 % slower).
   static constexpr int TKG = 32;                // tokens per gradient stage
-  static constexpr int NKF = 1;                 // forward ring stages
+  static constexpr int NKF = 2;                 // forward ring stages
   static constexpr int NKG = 2;                 // gradient ring: [TKG tokens x d] stages
-  static constexpr int CPS_ = 4;                // d-chunks per forward stage (one TMA box)
+  static constexpr int CPS_ = 2;                // d-chunks per forward stage (one TMA box)
   static constexpr int CPS = CPS_ < NCH ? CPS_ : NCH;
   static_assert(NCH % CPS == 0, "chunks per stage");
   static constexpr int CHUNK = BM * 128;        // 16 KB: 128 rows x 64 bf16
