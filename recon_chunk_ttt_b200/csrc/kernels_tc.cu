@@ -45,7 +45,8 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, u
 }
 
 // ----------------------------------------------------------------------------
-// apply kernel: O = W2 [SiLU(W1 q) ⊙ W3 q], one (query tile, head) per CTA
+// apply kernel: O = W2 [SiLU(W1 q) ⊙ W3 q], one (query tile, head) per CTA,
+// or per cluster of P CTAs when the items are few
 // ----------------------------------------------------------------------------
 template <int D>
 struct AP {
@@ -68,10 +69,12 @@ struct AP {
 // Persistent: CTA b takes (query tile, head) items b, b + grid, ...  With
 // P > 1 (few items: the launch is one cluster of P CTAs per item) the CTA of
 // cluster rank r takes the hidden slices [r nsl / P, (r + 1) nsl / P) of item
-// blockIdx.x / P and writes its partial O (fp32) to its own shared memory;
-// after a cluster barrier the CTA of rank o sums rows [o 128 / P,
-// (o + 1) 128 / P) of the P partials in rank order (distributed shared
-// memory loads) into O.  Per
+// blockIdx.x / P and, once its own MMAs are done, writes its partial O
+// (fp32) into its own q and operand buffers; after a cluster barrier the CTA
+// of rank o sums rows [o 128 / P, (o + 1) 128 / P) of the P partials in rank
+// order (distributed shared memory loads, all P of a row in flight at once)
+// into O, and a second barrier keeps every CTA alive until its partial has
+// been read.  Per
 // item and 64-wide hidden slice js: F(js) = Q [W1s; W3s]^T into TMEM buffer js&1,
 // the epilogue turns it into u = SiLU(h1) ⊙ h3 (bf16, shared memory), and
 // O += u W2s^T.  The q chunks are released one by one during the
@@ -375,10 +378,10 @@ __global__ void __launch_bounds__(AP<D>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (P > 1) {
-    // Every CTA of the cluster is past its last MMA (its epilogue saw
-    // o_full): its q and operand buffers are idle.  The partial O goes to
-    // this CTA's own buffers, row r at r * D * 4 bytes, fp32, 16-byte chunk c
-    // of the row at (c & ~7) | ((c ^ r) & 7).
+    // This CTA is past its last MMA (its epilogue saw o_full) and its last
+    // load (the producer drained its rings): its q and operand buffers are
+    // idle.  The partial O goes there, row r at r * D * 4 bytes, fp32,
+    // 16-byte chunk c of the row at (c & ~7) | ((c ^ r) & 7).
     tc_fence_after();
     if (warp >= 2) {
       const int q = warp & 3, ch = (warp - 2) / 4, row = q * 32 + lane;
