@@ -36,6 +36,15 @@
  *  - Every call is asynchronous on `stream` (NULL = the legacy default
  *    stream); arguments are validated on the host before anything is
  *    enqueued, so an error status means nothing was launched.
+ *  - The update, reduce/renorm and apply kernels are launched as
+ *    programmatic dependents (CUDA programmatic dependent launch): each
+ *    waits for the complete, visible results of the work ahead of it on the
+ *    stream before reading anything, and lets the next kernel on the stream
+ *    start its launch early.  A caller's kernel that follows on the same
+ *    stream and is itself launched with programmatic stream serialization
+ *    must wait for its dependency (cudaGridDependencySynchronize) before
+ *    reading this library's outputs; any other following work is ordered
+ *    as usual.
  *  - Layouts are dense, row-major, per head h = 0..H-1:
  *        W1, W3 : float [H][hidden][d]      W2 : float [H][d][hidden]
  *        K, V, Q: [n][H*d] token-major, bf16 (precision BF16_TC) or
