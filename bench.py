@@ -407,8 +407,7 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int):
     roof["traffic_over_algorithmic_bytes"] = (roof["traffic"] / roof["algorithmic_bytes_per_launch"]
                                               if roof["traffic"] else None)
     upd_ms = trace.get("tc_update_fused", (0, 0.0))[1]
-    upd_all_ms = upd_ms + trace.get("tc_convert_weights", (0, 0.0))[1] + \
-        trace.get("reduce_renorm", (0, 0.0))[1]
+    upd_all_ms = upd_ms + trace.get("reduce_renorm", (0, 0.0))[1]
     upd_flops = kw["tc_update_fused"]["flops"] * T * H * reps
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
