@@ -14,8 +14,9 @@ Sources (pages on the web, cited by title and section):
             ray-map queries) and section 3 "Streaming Reconstruction".
   [notes]   67656.sbs reading notes "ZipMap：基于 Test-Time Training 的线性时间
             有状态 3D 重建", section "TTT 模块：核心公式" (virtual objective,
-            one gradient step with per-token eta, SwiGLU, the linear-case
-            derivation) and "流式更新（streaming）".
+            one gradient step with per-token eta, SwiGLU), section
+            "为什么它像 attention（线性情形的直观推导）" (the linear case) and
+            "流式更新（streaming）".
   [survey]  mhpn.cn survey of TTSA3R / LaCT / ZipMap / LoGeR, part "二、LaCT,
             2、架构" (update = summed chunk gradient, then L2 normalisation).
 
