@@ -14,6 +14,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_util.cuh"
@@ -502,11 +504,17 @@ cudaError_t tc_update_impl(const Problem& p, const float* W1, const float* W2, c
                         W2, W3, W1o, W2o, W3o, shadow, w.scratch, st);
 }
 
-// Clusters of P apply CTAs that fit on the GPU at once (queried once per P).
+// Clusters of P apply CTAs that fit on the current GPU at once (queried once
+// per device and P).
 template <int D>
 int apply_clusters_per_wave(int P) {
-  static int cache[9] = {};
-  if (cache[P] == 0) {
+  static std::mutex mu;
+  static int cache[64][9] = {};
+  int dev = 0;
+  if (P < 1 || P > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  std::lock_guard<std::mutex> lk(mu);
+  int (&c)[9] = cache[dev];
+  if (c[P] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)P);
     cfg.blockDim = dim3(AP<D>::THREADS);
@@ -523,9 +531,9 @@ int apply_clusters_per_wave(int P) {
       (void)cudaGetLastError();
       n = -1;
     }
-    cache[P] = n;
+    c[P] = n;
   }
-  return cache[P];
+  return c[P];
 }
 
 // Hidden-slice parts per (query tile, head): 1 (persistent CTAs) unless the
